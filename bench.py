@@ -1,0 +1,406 @@
+"""Benchmark of the fused attention forward pass on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one pass of the decode sweep (B=1, Hq=64, Hkv in {4, 8}, L=1,
+S in {256 ... 32768}, Dqk=192 / Dv=128, bf16, causal): twelve attention calls
+through the C ABI, each a split-KV pass plus a log-sum-exp combine chosen by
+the router.  The headline is KV HBM GB/s (KV bytes the calls must read /
+device time).  L2 is flushed (a 2x L2-sized buffer is written) before every
+call, outside the timed kernels.  The same JSON line also carries the
+prefill configurations (TFLOP/s against the tensor peak), the verify sweep
+and the encoder shapes as secondary objects, the roofline of the dominant
+kernel, an end-to-end number through the public API with host buffers, and
+the fp64 CPU oracle timed on a bounded sample.
+
+With N > 1 (torchrun, one process per GPU) every rank runs the same sweep
+on its own GPU: the (batch, KV head) units are independent, so there is no
+collective on the data path ("scaling": "weak"); timing is the max over
+ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from scaled_dot_product_13_b200 import inputs as I  # noqa: E402
+from scaled_dot_product_13_b200.accounting import flops, io_bytes, kv_bytes  # noqa: E402
+
+METRIC = "prefill TFLOP/s & decode KV HBM GB/s on 1 B200, % of roofline; µs per SDPA call"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def ncu_traffic(kernel_file: str, tag: str):
+    """Per-launch DRAM bytes from a committed ncu summary, only while the
+    kernel source it was taken on is unchanged (sha256 recorded beside it)."""
+    prof = os.path.join(ROOT, "profiles", "traffic.md")
+    try:
+        text = open(prof).read()
+    except OSError:
+        return None
+    src = open(os.path.join(ROOT, "scaled_dot_product_13_b200", "csrc", kernel_file), "rb").read()
+    sha = hashlib.sha256(src).hexdigest()[:16]
+    for m in re.finditer(r"^traffic (\S+) (\S+) bytes_per_launch=(\d+) source_sha256=(\w+)",
+                         text, re.M):
+        if m.group(1) == tag and m.group(2) == kernel_file and m.group(4) == sha:
+            return int(m.group(3))
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+class Case:
+    """One attention problem resident on the device, ready to call."""
+
+    def __init__(self, sdpa, p: I.Problem, device):
+        self.p = p
+        q, k, v = I.make_qkv(p)
+        self.q, self.k, self.v = q.to(device), k.to(device), v.to(device)
+        self.out = torch.empty(p.B, p.Hq, p.L, p.Dv, dtype=p.torch_dtype, device=device)
+        self.info = sdpa.plan(p.B, p.Hq, p.Hkv, p.L, p.S, p.Dqk, p.Dv, p.causal, p.window, p.dtype)
+        nb = self.info["workspace_bytes"]
+        self.ws = torch.empty(max(nb, 4) // 4, dtype=torch.float32, device=device) if nb else None
+        self.kv_bytes = kv_bytes(p)
+        self.flops = flops(p)
+        self.io_bytes = io_bytes(p)
+
+    def call(self, sdpa):
+        sdpa.forward_ws(self.q, self.k, self.v, self.ws, scale=self.p.sm_scale,
+                        causal=self.p.causal, window_size=self.p.window, out=self.out)
+
+
+class HostCase:
+    """A problem's seeded inputs on the host (for the CPU oracle)."""
+
+    def __init__(self, p: I.Problem):
+        self.p = p
+        self.q, self.k, self.v = I.make_qkv(p)
+        self.kv_bytes = kv_bytes(p)
+
+
+def time_cases(sdpa, cases, steps, warmup, flush, sync_all):
+    """Per call: flush L2 (untimed), then time the call and its main kernel
+    with CUDA events on the current stream.  Returns per-case lists (ms)."""
+    call_ms = [[] for _ in cases]
+    main_ms = [[] for _ in cases]
+    stream = torch.cuda.current_stream()
+    for it in range(warmup + steps):
+        evs = []
+        for c in cases:
+            flush.zero_()
+            e0, e1, m0, m1 = (torch.cuda.Event(enable_timing=True) for _ in range(4))
+            e0.record(stream)
+            sdpa.time_next_main_kernel(m0, m1)
+            c.call(sdpa)
+            e1.record(stream)
+            evs.append((e0, e1, m0, m1))
+        if it == warmup - 1:
+            sync_all()
+        if it >= warmup:
+            torch.cuda.synchronize()
+            for i, (e0, e1, m0, m1) in enumerate(evs):
+                call_ms[i].append(e0.elapsed_time(e1))
+                main_ms[i].append(m0.elapsed_time(m1))
+    return call_ms, main_ms
+
+
+def time_e2e(sdpa, cases, steps, warmup, device):
+    """Public API with host buffers: pinned host -> device copy of q, k, v,
+    the call, device -> host copy of out; all inside the timed region."""
+    hosts = []
+    for c in cases:
+        hosts.append(tuple(t.cpu().pin_memory() for t in (c.q, c.k, c.v)) +
+                     (torch.empty(c.out.shape, dtype=c.out.dtype).pin_memory(),))
+    stream = torch.cuda.current_stream()
+    tot = []
+    h2d = d2h = 0
+    for it in range(warmup + steps):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for c, (hq, hk, hv, ho) in zip(cases, hosts):
+            qd = hq.to(device, non_blocking=True)
+            kd = hk.to(device, non_blocking=True)
+            vd = hv.to(device, non_blocking=True)
+            out = sdpa.forward(qd, kd, vd, scale=c.p.sm_scale, causal=c.p.causal,
+                               window_size=c.p.window)
+            ho.copy_(out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if it >= warmup:
+            tot.append(e0.elapsed_time(e1))
+    for c in cases:
+        h2d += sum(t.numel() * t.element_size() for t in (c.q, c.k, c.v))
+        d2h += c.out.numel() * c.out.element_size()
+    return tot, h2d, d2h
+
+
+def oracle_sample(cases, budget_s=12.0):
+    """The fp64 CPU oracle as it stands, on a bounded sample of the decode
+    sweep: every call of the sweep, repeated while the budget lasts (one
+    full pass at least).  Returns (KV GB/s, seconds, cores, calls)."""
+    from oracle import sdpa_oracle
+
+    cores = os.cpu_count() or 1
+    host = [(tuple(t.cpu() for t in (c.q, c.k, c.v)), c) for c in cases]
+    t0 = time.perf_counter()
+    nbytes, calls = 0.0, 0
+    while True:
+        for (q, k, v), c in host:
+            sdpa_oracle(q, k, v, c.p.sm_scale, c.p.causal, c.p.window, nthreads=cores)
+            nbytes += c.kv_bytes
+            calls += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return nbytes / dt / 1e9, dt, cores, calls
+
+
+def secondary(sdpa, probs, steps, warmup, flush, sync_all, device, peaks, kind):
+    """Time a list of problems (one call each per step); return a summary."""
+    cases = [Case(sdpa, p, device) for p in probs]
+    call_ms, main_ms = time_cases(sdpa, cases, steps, warmup, flush, sync_all)
+    pts = []
+    for c, cm, mm in zip(cases, call_ms, main_ms):
+        us = 1e3 * statistics.median(cm)
+        d = {"name": c.p.name, "us": round(us, 2), "path": c.info["path"],
+             "splits": c.info["splits"]}
+        if kind == "tflops":
+            tf = c.flops / (us * 1e-6) / 1e12
+            d.update({"tflops": round(tf, 1),
+                      "frac_tensor": round(tf / peaks["bf16_tflops"], 4)})
+        d["kv_gbs"] = round(c.kv_bytes / (us * 1e-6) / 1e9, 1)
+        d["frac_hbm"] = round(d["kv_gbs"] / peaks["hbm_gbs"], 4)
+        pts.append(d)
+    del cases
+    torch.cuda.empty_cache()
+    return pts
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the prefill / verify / encoder objects")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import torch.distributed as dist  # noqa: F811
+        import datetime
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+
+    probs = I.decode_problems()
+    peaks, peak_src = load_peaks()
+    workload = {"workload": "decode split-KV sweep: B=1, Hq=64, Hkv in {4,8}, L=1, "
+                            "S in {256,1024,4096,8192,16384,32768}, Dqk=192, Dv=128, bf16, causal",
+                "calls_per_step": len(probs), "l2": "flushed before every call (2x L2 write)",
+                "parallelism": f"replicas x{world} (independent KV-head units, no collective)"}
+
+    if args.impl == "reference":
+        if rank == 0:
+            host_cases = [HostCase(p) for p in probs]
+            for _ in range(args.warmup):
+                oracle_sample(host_cases[:1], budget_s=0.0)
+            vals, secs = [], 0.0
+            cores = os.cpu_count() or 1
+            for _ in range(args.steps):
+                v_, dt, cores, _ = oracle_sample(host_cases, budget_s=0.0)
+                vals.append(v_)
+                secs += dt
+            val = statistics.median(vals)
+            line = {"impl": "reference", "metric": METRIC, "value": round(val, 4),
+                    "unit": "GB/s (KV, decode)", "n_gpus": args.gpus, "steps": args.steps,
+                    "warmup": args.warmup, "ms_per_step": round(1e3 * secs / args.steps, 3),
+                    "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                    "dtype": "f64", "data": "synthetic N(0,1), seeded", "config": workload,
+                    "cpu_baseline": {"kind": "oracle", "value": round(val, 4),
+                                     "unit": "GB/s (KV, decode)", "cores": cores,
+                                     "sample": "one full pass of the 12-call decode sweep per step"},
+                    "e2e": {"value": round(val, 4), "unit": "GB/s (KV, decode)",
+                            "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            print(json.dumps(line), flush=True)
+        if dist is not None:
+            dist.destroy_process_group()
+        return
+
+    import scaled_dot_product_13_b200 as sdpa
+
+    sdpa.load_library()
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=device)
+
+    def sync_all():
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+            torch.cuda.synchronize()
+
+    cases = [Case(sdpa, p, device) for p in probs]
+    sync_all()
+    sampler = ClockSampler(device.index if device.index is not None else 0)
+    # warm-up steps run inside time_cases; the sampler covers the timed steps
+    sampler.start()
+    call_ms, main_ms = time_cases(sdpa, cases, args.steps, args.warmup, flush, sync_all)
+    sync_all()
+    clocks = sampler.stop()
+    sdpa.device_status(clear=False)
+
+    per_step_ms = [sum(cm[s] for cm in call_ms) for s in range(args.steps)]
+    local_ms = float(np.mean(per_step_ms))
+    local_total = float(sum(per_step_ms))
+    if dist is not None:
+        t = torch.tensor([local_total], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    else:
+        total_ms = local_total
+    step_bytes = sum(c.kv_bytes for c in cases)
+    value = world * step_bytes * args.steps / (total_ms * 1e-3) / 1e9
+
+    # roofline of the dominant kernel: the split-KV pass of the largest call
+    big = max(range(len(cases)), key=lambda i: cases[i].kv_bytes)
+    main_us = 1e3 * float(np.mean(main_ms[big]))
+    achieved = cases[big].kv_bytes / (main_us * 1e-6) / 1e9
+    traffic = ncu_traffic("splitkv.cuh", cases[big].p.name)
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": traffic, "kernel": "splitkv_kernel",
+                "launch": cases[big].p.name, "peak_source": peak_src,
+                "algorithmic_bytes_per_launch": cases[big].kv_bytes}
+    points = []
+    for c, cm, mm in zip(cases, call_ms, main_ms):
+        us = 1e3 * statistics.median(cm)
+        points.append({"name": c.p.name, "us": round(us, 2),
+                       "us_p10": round(1e3 * float(np.percentile(cm, 10)), 2),
+                       "us_p90": round(1e3 * float(np.percentile(cm, 90)), 2),
+                       "main_kernel_us": round(1e3 * statistics.median(mm), 2),
+                       "kv_gbs": round(c.kv_bytes / (us * 1e-6) / 1e9, 1),
+                       "frac_hbm": round(c.kv_bytes / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
+                       "splits": c.info["splits"], "ctas": c.info["ctas"]})
+    launches = sum(c.info["launches"] for c in cases) * args.steps
+
+    e2e_ms, h2d, d2h = time_e2e(sdpa, cases, max(3, args.steps // 4), 2, device)
+    e2e_val = step_bytes / (float(np.mean(e2e_ms)) * 1e-3) / 1e9 * world
+    del cases
+    torch.cuda.empty_cache()
+
+    extra = {}
+    if not args.no_secondary:
+        sec_steps = max(3, min(args.steps, 10))
+        extra["prefill"] = secondary(sdpa, I.window_problems() + I.encoder_problems(), sec_steps,
+                                     3, flush, sync_all, device, peaks, "tflops")
+        extra["verify"] = secondary(sdpa, I.verify_problems(), sec_steps, 3, flush, sync_all,
+                                    device, peaks, "tflops")
+        extra["tiny"] = secondary(sdpa, [I.tiny_problem()], sec_steps, 3, flush, sync_all,
+                                  device, peaks, "tflops")
+
+    line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s (KV, decode)",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic N(0,1), seeded (no model weights)", "config": workload,
+            "roofline": roofline, "clocks": clocks, "gpu_launches": launches,
+            "e2e": {"value": round(e2e_val, 2), "unit": "GB/s (KV, decode)",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": round(float(np.mean(e2e_ms)), 3)},
+            "points": points}
+    line.update(extra)
+    if rank == 0 and world == 1:
+        host_cases = [HostCase(p) for p in I.decode_problems()]
+        val, secs, cores, calls = oracle_sample(host_cases, budget_s=10.0)
+        line["cpu_baseline"] = {"value": round(val, 4), "unit": "GB/s (KV, decode)",
+                                "cores": cores, "kind": "oracle",
+                                "sample": f"{calls} decode calls of the sweep ({secs:.1f} s, fp64)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

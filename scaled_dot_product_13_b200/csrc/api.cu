@@ -1,0 +1,561 @@
+// C ABI of libsdpa: argument validation, the router (planner), workspace
+// handling, TMA descriptor encoding and launch sequencing.
+//
+// The router never falls back to a non-fused path: a problem either maps to a
+// fused kernel instance or the call fails with a message that names the
+// violated constraint (mlx PR #4185, "API": force_fused raises with the
+// unsupported constraint; "Kernel support": the dispatch-time check that
+// prevents silent zero output).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "launch.h"
+#include "ptx.cuh"
+
+// Device watchdog word (see sdpa_device_status).
+__device__ unsigned int g_sdpa_watchdog_word;
+
+namespace sdpa {
+
+namespace {
+
+thread_local std::string t_last_error;
+thread_local cudaEvent_t t_ev_start = nullptr, t_ev_stop = nullptr;
+std::atomic<uint64_t> g_wait_limit_ns{0};
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;  // 2 s
+
+sdpa_status fail(sdpa_status st, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return st;
+}
+
+sdpa_status fail_str(sdpa_status st, const std::string &msg) {
+  t_last_error = msg;
+  return st;
+}
+
+uint64_t wait_limit() {
+  const uint64_t v = g_wait_limit_ns.load();
+  return v ? v : kDefaultWaitLimitNs;
+}
+
+// ---------------------------------------------------------------------------
+// validation
+// ---------------------------------------------------------------------------
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + nb && b0 < a0 + na;
+}
+
+sdpa_status validate_shape(const Problem &p) {
+  if (p.B < 1 || p.Hq < 1 || p.Hkv < 1 || p.L < 1 || p.S < 1)
+    return fail(SDPA_ERR_INVALID_ARG,
+                "B, Hq, Hkv, L, S must all be >= 1 (got B=%d Hq=%d Hkv=%d L=%d S=%d)", p.B, p.Hq,
+                p.Hkv, p.L, p.S);
+  if (p.Hq % p.Hkv != 0)
+    return fail(SDPA_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", p.Hq, p.Hkv);
+  if (p.dtype != SDPA_BF16 && p.dtype != SDPA_F16)
+    return fail(SDPA_ERR_UNSUPPORTED, "dtype %d is not supported (bf16 = 0, f16 = 1)",
+                (int)p.dtype);
+  if (p.causal != 0 && p.causal != 1)
+    return fail(SDPA_ERR_INVALID_ARG, "causal must be 0 or 1 (got %d)", p.causal);
+  if (p.causal && p.L > p.S)
+    return fail(SDPA_ERR_INVALID_ARG,
+                "causal attention needs L <= S (got L=%d > S=%d): queries are aligned to the "
+                "end of the keys, so the first rows would see no key",
+                p.L, p.S);
+  if (p.window < 0)
+    return fail(SDPA_ERR_INVALID_ARG, "window_size must be >= 0 (got %d)", p.window);
+  if (p.window > 0 && !p.causal)
+    return fail(SDPA_ERR_UNSUPPORTED,
+                "window_size > 0 is defined only together with causal masking (got causal=0, "
+                "window_size=%d)",
+                p.window);
+  if (!std::isfinite(p.scale))
+    return fail(SDPA_ERR_INVALID_ARG, "scale must be finite");
+  for (int d : {p.Dqk, p.Dv}) {
+    if (d < 8 || d > 256 || d % 8 != 0)
+      return fail(SDPA_ERR_UNSUPPORTED,
+                  "head dims must be multiples of 8 in [8, 256] (got Dqk=%d, Dv=%d)", p.Dqk,
+                  p.Dv);
+  }
+  const long long rows = (long long)p.B * p.Hq * p.L;
+  if (rows > 0x7fffffffLL || (long long)p.B * p.Hkv * p.S > 0x7fffffffLL)
+    return fail(SDPA_ERR_UNSUPPORTED,
+                "B*Hq*L and B*Hkv*S must each stay below 2^31 (got %lld and %lld)", rows,
+                (long long)p.B * p.Hkv * p.S);
+  return SDPA_OK;
+}
+
+sdpa_status validate_pointers(const Problem &p, const void *q, const void *k, const void *v,
+                              const void *out) {
+  if (!q || !k || !v || !out)
+    return fail(SDPA_ERR_INVALID_ARG, "q, k, v and out must be non-NULL device pointers");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return fail(SDPA_ERR_INVALID_ARG, "q, k, v and out must be 16-byte aligned");
+  const size_t nq = (size_t)p.B * p.Hq * p.L * p.Dqk * 2;
+  const size_t nk = (size_t)p.B * p.Hkv * p.S * p.Dqk * 2;
+  const size_t nv = (size_t)p.B * p.Hkv * p.S * p.Dv * 2;
+  const size_t no = (size_t)p.B * p.Hq * p.L * p.Dv * 2;
+  if (overlaps(out, no, q, nq) || overlaps(out, no, k, nk) || overlaps(out, no, v, nv))
+    return fail(SDPA_ERR_INVALID_ARG, "out must not overlap q, k or v");
+  return SDPA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// router
+// ---------------------------------------------------------------------------
+int pick_pair(int dqk, int dv) {
+  for (int i = 0; i < kNumDimPairs; ++i)
+    if (kDimPairs[i].dqk >= dqk && kDimPairs[i].dv >= dv) return i;
+  return -1;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_splits,
+                      Plan *out) {
+  Plan pl;
+  memset(&pl, 0, sizeof(pl));
+  pl.pair = pick_pair(pb.Dqk, pb.Dv);
+  if (pl.pair < 0)
+    return fail(SDPA_ERR_UNSUPPORTED, "no kernel instance covers Dqk=%d, Dv=%d", pb.Dqk, pb.Dv);
+  if (force_path != SDPA_PATH_AUTO && force_path != SDPA_PATH_SPLITKV &&
+      force_path != SDPA_PATH_TC)
+    return fail(SDPA_ERR_INVALID_ARG, "unknown path %d", force_path);
+  if (force_splits < 0) return fail(SDPA_ERR_INVALID_ARG, "force_splits must be >= 0");
+  if (num_sms < 1) num_sms = 148;
+  const int g = pb.Hq / pb.Hkv;
+  pl.rows = g * pb.L;
+
+  if (force_path == SDPA_PATH_TC)
+    return fail(SDPA_ERR_UNSUPPORTED, "the tcgen05 tile path is not available in this build");
+  pl.path = SDPA_PATH_SPLITKV;
+  if (pl.rows <= 16) {
+    pl.wr = 1; pl.wk = 4;
+  } else if (pl.rows <= 32) {
+    pl.wr = 2; pl.wk = 2;
+  } else {
+    pl.wr = 4; pl.wk = 1;
+  }
+  pl.row_tile = 16 * pl.wr;
+  pl.key_block = kSplitKvBN;
+
+  pl.row_tiles = (pl.rows + pl.row_tile - 1) / pl.row_tile;
+  // keys visible to at least one row: [kbeg, S); the last row sits at S-1
+  const int off = pb.S - pb.L;
+  const int kbeg = pb.window > 0 ? std::max(0, off - pb.window + 1) : 0;
+  const int bn = pl.key_block;
+  pl.split_base = (kbeg / bn) * bn;
+  const int nkb = (pb.S + bn - 1) / bn - kbeg / bn;
+  const long long base = (long long)pb.B * pb.Hkv * pl.row_tiles;
+  int splits;
+  if (force_splits > 0) {
+    splits = std::min(force_splits, nkb);
+  } else if (base >= num_sms) {
+    splits = 1;
+  } else {
+    splits = (int)std::max(1LL, num_sms / base);
+    splits = std::min(splits, nkb);
+  }
+  const int bps = (nkb + splits - 1) / splits;
+  if (force_splits == 0) splits = (nkb + bps - 1) / bps;
+  pl.splits = splits;
+  pl.keys_per_split = bps * bn;
+  pl.ctas = base * splits;
+  if (pl.ctas > 0x7fffffffLL)
+    return fail(SDPA_ERR_UNSUPPORTED, "problem needs %lld CTAs, above the grid limit", pl.ctas);
+  pl.launches = splits > 1 ? 2 : 1;
+  if (splits > 1) {
+    const size_t rows_total = (size_t)pb.B * pb.Hq * pb.L;
+    pl.ws_o_bytes = align256(rows_total * pb.Dv * sizeof(float) * splits);
+    pl.ws_lse_bytes = align256(rows_total * sizeof(float) * splits);
+  }
+  pl.ws_bytes = pl.ws_o_bytes + pl.ws_lse_bytes;
+  *out = pl;
+  return SDPA_OK;
+}
+
+void fill_info(const Plan &pl, sdpa_plan_info *info) {
+  info->path = pl.path;
+  info->splits = pl.splits;
+  info->rows = pl.rows;
+  info->row_tile = pl.row_tile;
+  info->row_tiles = pl.row_tiles;
+  info->key_block = pl.key_block;
+  info->keys_per_split = pl.keys_per_split;
+  info->ctas = (int)pl.ctas;
+  info->launches = pl.launches;
+  info->dqk_pad = kDimPairs[pl.pair].dqk;
+  info->dv_pad = kDimPairs[pl.pair].dv;
+  info->workspace_bytes = pl.ws_bytes;
+}
+
+// ---------------------------------------------------------------------------
+// device state
+// ---------------------------------------------------------------------------
+constexpr int kMaxDevices = 64;
+std::mutex g_dev_mu;
+unsigned int *g_wd_ptr[kMaxDevices];
+int g_num_sms[kMaxDevices];
+
+sdpa_status device_state(int *dev_out, int *sms_out, unsigned int **wd_out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess)
+    return fail(SDPA_ERR_CUDA, "no usable CUDA device: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return fail(SDPA_ERR_CUDA, "device index %d too large", dev);
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (!g_wd_ptr[dev]) {
+    cudaDeviceProp prop;
+    e = cudaGetDeviceProperties(&prop, dev);
+    if (e != cudaSuccess)
+      return fail(SDPA_ERR_CUDA, "cudaGetDeviceProperties: %s", cudaGetErrorString(e));
+    if (prop.major != 10 || prop.minor != 0)
+      return fail(SDPA_ERR_UNSUPPORTED,
+                  "libsdpa is built for sm_100a (B200); device %d is sm_%d%d", dev, prop.major,
+                  prop.minor);
+    void *ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_sdpa_watchdog_word);
+    if (e != cudaSuccess)
+      return fail(SDPA_ERR_CUDA, "cudaGetSymbolAddress(watchdog): %s", cudaGetErrorString(e));
+    g_num_sms[dev] = prop.multiProcessorCount;
+    g_wd_ptr[dev] = static_cast<unsigned int *>(ptr);
+  }
+  *dev_out = dev;
+  *sms_out = g_num_sms[dev];
+  *wd_out = g_wd_ptr[dev];
+  return SDPA_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// ---------------------------------------------------------------------------
+// the call
+// ---------------------------------------------------------------------------
+sdpa_status run(const Problem &pb, const void *q, const void *k, const void *v, void *out,
+                int force_path, int force_splits, void *ws, size_t ws_bytes, bool own_ws,
+                cudaStream_t stream) {
+  sdpa_status st = validate_shape(pb);
+  if (st != SDPA_OK) return st;
+  st = validate_pointers(pb, q, k, v, out);
+  if (st != SDPA_OK) return st;
+  int dev, sms;
+  unsigned int *wd;
+  st = device_state(&dev, &sms, &wd);
+  if (st != SDPA_OK) return st;
+  Plan pl;
+  st = make_plan(pb, sms, force_path, force_splits, &pl);
+  if (st != SDPA_OK) return st;
+
+  bool allocated = false;
+  if (pl.ws_bytes > 0) {
+    if (own_ws) {
+      cudaError_t e = cudaMallocAsync(&ws, pl.ws_bytes, stream);
+      if (e != cudaSuccess)
+        return fail(SDPA_ERR_CUDA, "cudaMallocAsync(%zu bytes) for the split workspace: %s",
+                    pl.ws_bytes, cudaGetErrorString(e));
+      allocated = true;
+    } else {
+      if (ws == nullptr || ws_bytes < pl.ws_bytes)
+        return fail(SDPA_ERR_RESOURCES, "workspace of %zu bytes needed, %zu given", pl.ws_bytes,
+                    ws == nullptr ? (size_t)0 : ws_bytes);
+      if (!aligned16(ws)) return fail(SDPA_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+    }
+  }
+  Launch ln;
+  ln.pb = pb;
+  ln.plan = pl;
+  ln.q = q; ln.k = k; ln.v = v; ln.out = out;
+  ln.part_o = static_cast<float *>(ws);
+  ln.part_lse = ws ? reinterpret_cast<float *>(static_cast<char *>(ws) + pl.ws_o_bytes) : nullptr;
+  ln.lse_out = nullptr;
+  ln.wd_word = wd;
+  ln.wd_limit_ns = wait_limit();
+  ln.stream = stream;
+
+  std::string err;
+  cudaEvent_t ev0 = t_ev_start, ev1 = t_ev_stop;
+  t_ev_start = t_ev_stop = nullptr;
+  if (ev0) cudaEventRecord(ev0, stream);
+  st = launch_splitkv(ln, &err);
+  if (ev1) cudaEventRecord(ev1, stream);
+  if (st == SDPA_OK && pl.splits > 1) st = launch_combine(ln, &err);
+  if (allocated) {
+    cudaError_t e = cudaFreeAsync(ws, stream);
+    if (st == SDPA_OK && e != cudaSuccess) {
+      err = std::string("cudaFreeAsync: ") + cudaGetErrorString(e);
+      st = SDPA_ERR_CUDA;
+    }
+  }
+  if (st != SDPA_OK) return fail_str(st, err);
+  return SDPA_OK;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// shared helpers declared in launch.h
+// ---------------------------------------------------------------------------
+bool encode_tma(CUtensorMap *map, sdpa_dtype dt, int rank, const void *base,
+                const uint64_t *dims, const uint64_t *strides_bytes, const uint32_t *box,
+                std::string *err) {
+  auto fn = encode_fn();
+  if (!fn) {
+    *err = "cuTensorMapEncodeTiled is not available from the driver";
+    return false;
+  }
+  cuuint64_t gdim[5], gstr[4];
+  cuuint32_t bdim[5], estr[5];
+  for (int i = 0; i < rank; ++i) {
+    gdim[i] = dims[i];
+    bdim[i] = box[i];
+    estr[i] = 1;
+  }
+  for (int i = 0; i < rank - 1; ++i) gstr[i] = strides_bytes[i];
+  CUresult r = fn(map, dt == SDPA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                  (cuuint32_t)rank, const_cast<void *>(base), gdim, gstr, bdim, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    char buf[160];
+    snprintf(buf, sizeof(buf), "cuTensorMapEncodeTiled failed (CUresult %d, rank %d)", (int)r,
+             rank);
+    *err = buf;
+    return false;
+  }
+  return true;
+}
+
+sdpa_status prepare_kernel(const void *func, int threads, size_t smem, const char *name,
+                           std::string *err) {
+  // (device, function) pairs already checked
+  static std::mutex mu;
+  static const void *done_fn[512];
+  static int done_dev[512];
+  static int ndone = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    for (int i = 0; i < ndone; ++i)
+      if (done_fn[i] == func && done_dev[i] == dev) return SDPA_OK;
+  }
+  cudaFuncAttributes attr;
+  cudaError_t e = cudaFuncGetAttributes(&attr, func);
+  if (e != cudaSuccess) {
+    *err = std::string(name) + ": cudaFuncGetAttributes: " + cudaGetErrorString(e);
+    return SDPA_ERR_CUDA;
+  }
+  int max_optin = 0;
+  cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  char buf[256];
+  if (attr.maxThreadsPerBlock < threads) {
+    snprintf(buf, sizeof(buf), "%s: compiled kernel allows %d threads per block, launch needs %d",
+             name, attr.maxThreadsPerBlock, threads);
+    *err = buf;
+    return SDPA_ERR_RESOURCES;
+  }
+  if ((size_t)attr.sharedSizeBytes + smem > (size_t)max_optin) {
+    snprintf(buf, sizeof(buf), "%s: needs %zu bytes of shared memory, device allows %d", name,
+             (size_t)attr.sharedSizeBytes + smem, max_optin);
+    *err = buf;
+    return SDPA_ERR_RESOURCES;
+  }
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) {
+    *err = std::string(name) + ": cudaFuncSetAttribute: " + cudaGetErrorString(e);
+    return SDPA_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lk(mu);
+  if (ndone < 512) {
+    done_fn[ndone] = func;
+    done_dev[ndone] = dev;
+    ++ndone;
+  }
+  return SDPA_OK;
+}
+
+// Watchdog self-test kernel: waits on an mbarrier that nothing ever arrives
+// on; the bounded wait must expire and record its code.
+__global__ void watchdog_selftest_kernel(Watchdog wd, int *result) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const bool ok = mbar_wait(&bar, 0, wd, kWdTmaFull);
+  if (threadIdx.x == 0) *result = ok ? 1 : 0;
+}
+
+}  // namespace sdpa
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+using namespace sdpa;
+
+static Problem make_problem(int B, int Hq, int Hkv, int L, int S, int Dqk, int Dv, float scale,
+                            int causal, int window, sdpa_dtype dtype) {
+  Problem p;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = L; p.S = S; p.Dqk = Dqk; p.Dv = Dv;
+  p.scale = scale; p.causal = causal; p.window = window; p.dtype = dtype;
+  return p;
+}
+
+extern "C" {
+
+sdpa_status sdpa_forward(const void *q, const void *k, const void *v, void *out, int B, int Hq,
+                         int Hkv, int L, int S, int Dqk, int Dv, float scale, int causal,
+                         int window_size, sdpa_dtype dtype, sdpa_stream_t stream) {
+  t_last_error.clear();
+  return run(make_problem(B, Hq, Hkv, L, S, Dqk, Dv, scale, causal, window_size, dtype), q, k, v,
+             out, SDPA_PATH_AUTO, 0, nullptr, 0, true, (cudaStream_t)stream);
+}
+
+size_t sdpa_workspace_bytes(int B, int Hq, int Hkv, int L, int S, int Dqk, int Dv, int causal,
+                            int window_size, sdpa_dtype dtype) {
+  t_last_error.clear();
+  Problem pb = make_problem(B, Hq, Hkv, L, S, Dqk, Dv, 1.0f, causal, window_size, dtype);
+  if (validate_shape(pb) != SDPA_OK) return 0;
+  int dev, sms;
+  unsigned int *wd;
+  if (device_state(&dev, &sms, &wd) != SDPA_OK) return 0;
+  Plan pl;
+  if (make_plan(pb, sms, SDPA_PATH_AUTO, 0, &pl) != SDPA_OK) return 0;
+  return pl.ws_bytes;
+}
+
+sdpa_status sdpa_forward_ws(const void *q, const void *k, const void *v, void *out, int B,
+                            int Hq, int Hkv, int L, int S, int Dqk, int Dv, float scale,
+                            int causal, int window_size, sdpa_dtype dtype, void *workspace,
+                            size_t workspace_bytes, sdpa_stream_t stream) {
+  t_last_error.clear();
+  return run(make_problem(B, Hq, Hkv, L, S, Dqk, Dv, scale, causal, window_size, dtype), q, k, v,
+             out, SDPA_PATH_AUTO, 0, workspace, workspace_bytes, false, (cudaStream_t)stream);
+}
+
+sdpa_status sdpa_plan(int B, int Hq, int Hkv, int L, int S, int Dqk, int Dv, int causal,
+                      int window_size, sdpa_dtype dtype, int num_sms, int force_path,
+                      int force_splits, sdpa_plan_info *info) {
+  t_last_error.clear();
+  if (!info) return fail(SDPA_ERR_INVALID_ARG, "info must be non-NULL");
+  Problem pb = make_problem(B, Hq, Hkv, L, S, Dqk, Dv, 1.0f, causal, window_size, dtype);
+  sdpa_status st = validate_shape(pb);
+  if (st != SDPA_OK) return st;
+  Plan pl;
+  st = make_plan(pb, num_sms, force_path, force_splits, &pl);
+  if (st != SDPA_OK) return st;
+  fill_info(pl, info);
+  return SDPA_OK;
+}
+
+sdpa_status sdpa_forward_planned(const void *q, const void *k, const void *v, void *out, int B,
+                                 int Hq, int Hkv, int L, int S, int Dqk, int Dv, float scale,
+                                 int causal, int window_size, sdpa_dtype dtype, int force_path,
+                                 int force_splits, void *workspace, size_t workspace_bytes,
+                                 sdpa_stream_t stream) {
+  t_last_error.clear();
+  return run(make_problem(B, Hq, Hkv, L, S, Dqk, Dv, scale, causal, window_size, dtype), q, k, v,
+             out, force_path, force_splits, workspace, workspace_bytes, false,
+             (cudaStream_t)stream);
+}
+
+sdpa_status sdpa_device_status(int clear) {
+  t_last_error.clear();
+  int dev, sms;
+  unsigned int *wd;
+  sdpa_status st = device_state(&dev, &sms, &wd);
+  if (st != SDPA_OK) return st;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess)
+    return fail(SDPA_ERR_CUDA, "cudaDeviceSynchronize: %s", cudaGetErrorString(e));
+  unsigned int word = 0;
+  e = cudaMemcpy(&word, wd, sizeof(word), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return fail(SDPA_ERR_CUDA, "reading the watchdog word: %s", cudaGetErrorString(e));
+  if (clear && word != 0) {
+    const unsigned int zero = 0;
+    e = cudaMemcpy(wd, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return fail(SDPA_ERR_CUDA, "clearing the watchdog word: %s", cudaGetErrorString(e));
+  }
+  if (word != 0)
+    return fail(SDPA_ERR_TIMEOUT, "a kernel gave up on a bounded wait (watchdog code %u)", word);
+  return SDPA_OK;
+}
+
+void sdpa_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns); }
+
+void sdpa_time_next_main_kernel(void *start_event, void *stop_event) {
+  t_ev_start = static_cast<cudaEvent_t>(start_event);
+  t_ev_stop = static_cast<cudaEvent_t>(stop_event);
+}
+
+sdpa_status sdpa_watchdog_selftest(uint64_t limit_ns, int *waited_out) {
+  t_last_error.clear();
+  int dev, sms;
+  unsigned int *wd;
+  sdpa_status st = device_state(&dev, &sms, &wd);
+  if (st != SDPA_OK) return st;
+  int *d_res = nullptr;
+  cudaError_t e = cudaMalloc(&d_res, sizeof(int));
+  if (e != cudaSuccess) return fail(SDPA_ERR_CUDA, "cudaMalloc: %s", cudaGetErrorString(e));
+  Watchdog w;
+  w.word = wd;
+  w.limit_ns = limit_ns ? limit_ns : 100000000ull;
+  watchdog_selftest_kernel<<<1, 32>>>(w, d_res);
+  e = cudaGetLastError();
+  int res = -1;
+  if (e == cudaSuccess) e = cudaMemcpy(&res, d_res, sizeof(int), cudaMemcpyDeviceToHost);
+  cudaFree(d_res);
+  if (e != cudaSuccess) return fail(SDPA_ERR_CUDA, "selftest: %s", cudaGetErrorString(e));
+  if (waited_out) *waited_out = res;
+  return SDPA_OK;
+}
+
+const char *sdpa_status_string(sdpa_status s) {
+  switch (s) {
+    case SDPA_OK: return "SDPA_OK";
+    case SDPA_ERR_INVALID_ARG: return "SDPA_ERR_INVALID_ARG";
+    case SDPA_ERR_UNSUPPORTED: return "SDPA_ERR_UNSUPPORTED";
+    case SDPA_ERR_RESOURCES: return "SDPA_ERR_RESOURCES";
+    case SDPA_ERR_CUDA: return "SDPA_ERR_CUDA";
+    case SDPA_ERR_TIMEOUT: return "SDPA_ERR_TIMEOUT";
+  }
+  return "SDPA_ERR_UNKNOWN";
+}
+
+const char *sdpa_last_error_message(void) { return t_last_error.c_str(); }
+
+int sdpa_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,80 @@
+// Host-side declarations shared by the C-ABI layer and the per-kernel launch
+// units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <string>
+
+#include "../../include/sdpa.h"
+
+namespace sdpa {
+
+// Head-dim pairs a kernel instance is compiled for.  A problem runs on the
+// cheapest pair that covers it; TMA zero-fills the columns in between.
+struct DimPair {
+  int dqk, dv;
+};
+constexpr DimPair kDimPairs[] = {{64, 64},   {80, 80},   {128, 128},
+                                 {192, 128}, {192, 192}, {256, 256}};
+constexpr int kNumDimPairs = sizeof(kDimPairs) / sizeof(kDimPairs[0]);
+
+// Key block of the split-KV kernel (keys per pipeline stage).
+constexpr int kSplitKvBN = 64;
+
+struct Problem {
+  int B, Hq, Hkv, L, S, Dqk, Dv;
+  float scale;
+  int causal, window;
+  sdpa_dtype dtype;
+};
+
+struct Plan {
+  int path;            // SDPA_PATH_SPLITKV or SDPA_PATH_TC
+  int pair;            // index into kDimPairs
+  int rows;            // g * L
+  int wr, wk;          // split-KV warp layout (rows x key slices)
+  int row_tile;
+  int row_tiles;
+  int key_block;
+  int split_base;      // first key of split 0 (block aligned)
+  int keys_per_split;
+  int splits;
+  long long ctas;
+  int launches;
+  size_t ws_o_bytes, ws_lse_bytes, ws_bytes;
+};
+
+// Everything a kernel launch needs.
+struct Launch {
+  Problem pb;
+  Plan plan;
+  const void *q, *k, *v;
+  void *out;
+  float *part_o, *part_lse;
+  float *lse_out;          // optional final LSE [B*Hq*L] (nullptr = not wanted)
+  unsigned int *wd_word;
+  uint64_t wd_limit_ns;
+  cudaStream_t stream;
+};
+
+// Encode a tiled TMA descriptor (128-byte swizzle, zero fill out of bounds).
+// rank 2 or 3; dims/strides in elements/bytes as cuTensorMapEncodeTiled wants.
+bool encode_tma(CUtensorMap *map, sdpa_dtype dt, int rank, const void *base,
+                const uint64_t *dims, const uint64_t *strides_bytes, const uint32_t *box,
+                std::string *err);
+
+// Per-path launchers (return SDPA_OK or an error with *err set).
+sdpa_status launch_splitkv(const Launch &ln, std::string *err);
+sdpa_status launch_combine(const Launch &ln, std::string *err);
+
+// Checks that a kernel fits the device (threads, shared memory) before its
+// first launch, and raises its dynamic shared-memory limit.  Cached per
+// device and kernel.
+sdpa_status prepare_kernel(const void *func, int threads, size_t smem, const char *name,
+                           std::string *err);
+
+}  // namespace sdpa

@@ -1,0 +1,89 @@
+// Kernel parameter block shared by the attention kernels.
+#pragma once
+
+#include <stdint.h>
+
+#include "ptx.cuh"
+
+namespace sdpa {
+
+// One attention call, as the kernels see it.
+//
+// Packed rows: for batch b and KV head h, the g = Hq/Hkv query heads that
+// read h are consecutive, so their g*L query rows form one contiguous slab of
+// R = g*L rows in q and out (row r = j*L + i is query i of head h*g + j).  A
+// CTA owns a tile of consecutive slab rows and one range of keys.  Query i
+// sits at key position i + off with off = S - L.
+struct AttnParams {
+  int B, Hq, Hkv, L, S, Dqk, Dv;
+  int R;              // packed rows per (b, KV head) = g * L
+  int off;            // S - L
+  int causal;         // 0/1
+  int window;         // 0 = none
+  float scale_log2;   // scale * log2(e)
+  int row_tiles;      // row tiles per (b, KV head)
+  int splits;         // key splits
+  int split_base;     // first key of split 0 (a multiple of the key block)
+  int keys_per_split; // multiple of the kernel's key block
+  void *out;          // [B*Hq*L][Dv] in the I/O type (written when splits == 1)
+  float *part_o;      // [splits][B*Hq*L][Dv] fp32, normalised per split
+  float *part_lse;    // [splits][B*Hq*L] fp32 natural-log LSE, -inf if empty
+  Watchdog wd;
+};
+
+// Range of positions covered by the valid rows of a tile.
+struct TileRows {
+  int row0;       // first slab row of the tile
+  int nvalid;     // rows of the tile inside the slab
+  int pos_min;    // smallest key position of a valid row
+  int pos_max;    // largest
+};
+
+__device__ __forceinline__ TileRows tile_rows(const AttnParams &p, int row_tile, int rows_per_tile) {
+  TileRows t;
+  t.row0 = row_tile * rows_per_tile;
+  t.nvalid = min(rows_per_tile, p.R - t.row0);
+  const int i0 = t.row0 % p.L;
+  const int i1 = (t.row0 + t.nvalid - 1) % p.L;
+  if (t.nvalid >= p.L || i1 < i0) {  // the tile wraps over a whole head's rows
+    t.pos_min = p.off;
+    t.pos_max = p.L - 1 + p.off;
+  } else {
+    t.pos_min = i0 + p.off;
+    t.pos_max = i1 + p.off;
+  }
+  return t;
+}
+
+// Key range [k_lo, k_hi) a tile must visit, rounded out to whole key blocks
+// of `bn`, then clipped to the split's range [split*kps, (split+1)*kps).
+// Causal: keys above the last row's position are skipped (kb_lim).  Window:
+// whole blocks left of the first row's window edge are skipped (kb_start)
+// (mlx PR #3552, "Implementation").
+__device__ __forceinline__ void tile_key_range(const AttnParams &p, const TileRows &t, int bn,
+                                               int split, int &k_lo, int &k_hi) {
+  const int kend = p.causal ? min(p.S, t.pos_max + 1) : p.S;
+  const int kbeg = p.window > 0 ? max(0, t.pos_min - p.window + 1) : 0;
+  const int lo = (kbeg / bn) * bn;
+  const int hi = ((kend + bn - 1) / bn) * bn;
+  const int s_lo = p.split_base + split * p.keys_per_split;
+  const int s_hi = s_lo + p.keys_per_split;
+  k_lo = max(lo, s_lo);
+  k_hi = min(hi, s_hi);
+  if (k_hi < k_lo) k_hi = k_lo;
+}
+
+// Does key block [k0, k0+bn) need per-element masking for any row of the tile?
+__device__ __forceinline__ bool block_needs_mask(const AttnParams &p, const TileRows &t, int k0,
+                                                 int bn) {
+  if (k0 + bn > p.S) return true;                                  // tail past S
+  if (p.causal && k0 + bn - 1 > t.pos_min) return true;            // diagonal
+  if (p.window > 0 && k0 <= t.pos_max - p.window) return true;     // window left edge
+  return false;
+}
+
+__device__ __forceinline__ bool key_visible(const AttnParams &p, int pos, int col) {
+  return col < p.S && (!p.causal || col <= pos) && (p.window == 0 || pos - col < p.window);
+}
+
+}  // namespace sdpa

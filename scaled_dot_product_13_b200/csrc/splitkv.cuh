@@ -1,0 +1,408 @@
+// Split-KV attention pass on warp-level tensor-core tiles (m16n8k16).
+//
+// This is the decode / short-query path: the g*L query rows that share one KV
+// head are packed into 16-row warp tiles, so one pass over that head's keys
+// serves all of them, and the keys are split across CTAs so the work stays
+// parallel over S even when B*Hkv is small (mlx issue #3826: the verify
+// window lost its split over S and paid a padded 64-row tile per head; the
+// fix there was a split over S with a log-sum-exp merge).  It is also a
+// complete, general path: any L, causal and window masks, any head dims up
+// to 256.
+//
+// CTA = (row tile, split, batch*KV head).  Warps: WR x WK consumer warps (WR
+// row groups of 16 rows, WK slices of each key block) and one producer warp
+// that streams Q once and K/V key blocks through an NST-stage ring with TMA
+// (128-byte swizzled boxes of 64 columns, zero fill past S and past D).
+// Each consumer keeps an fp32 online softmax (running max m, running sum l,
+// rescaled O) in registers; P is rounded to the 16-bit input type for the
+// P*V tile.  The WK slices are merged in shared memory at the end; the
+// result goes to `out` (one split) or to fp32 partials + LSE (several).
+#pragma once
+
+#include "params.cuh"
+
+namespace sdpa {
+
+template <int DQK, int DV, int BN, int WR, int WK, int NST>
+struct SplitKvCfg {
+  static constexpr int kRT = 16 * WR;             // rows per CTA
+  static constexpr int kKW = BN / WK;             // keys per warp per block
+  static constexpr int kQBoxes = (DQK + 63) / 64; // 64-column TMA boxes
+  static constexpr int kVBoxes = (DV + 63) / 64;
+  static constexpr int kConsumers = WR * WK;
+  static constexpr int kThreads = (kConsumers + 1) * 32;
+  static constexpr uint32_t kQBytes = kQBoxes * kRT * 128;
+  static constexpr uint32_t kKBytes = kQBoxes * BN * 128;
+  static constexpr uint32_t kVBytes = kVBoxes * BN * 128;
+  static constexpr uint32_t kStageBytes = kKBytes + kVBytes;
+  static constexpr uint32_t kRingBytes = NST * kStageBytes;
+  // merge buffer (reuses the ring): per consumer warp, O fragments + m + l
+  static constexpr uint32_t kMergeBytes = kConsumers * 32 * (DV / 2 + 4) * 4;
+  static constexpr uint32_t kBarOffset =
+      kQBytes + (kRingBytes > kMergeBytes ? kRingBytes : kMergeBytes);
+  static constexpr uint32_t kSmemBytes = kBarOffset + (2 * NST + 1) * 8 + 1024;  // + align slack
+  static_assert(DQK % 16 == 0 && DV % 16 == 0, "head dims padded to 16");
+  static_assert(kKW % 16 == 0, "each warp takes whole 16-key chunks");
+  static_assert(BN % 8 == 0 && BN <= 256, "TMA box height");
+  static_assert((kRT * 128) % 1024 == 0 && (BN * 128) % 1024 == 0, "swizzle atoms");
+};
+
+template <bool kBF16, int DQK, int DV, int BN, int WR, int WK, int NST>
+__global__ void __launch_bounds__(SplitKvCfg<DQK, DV, BN, WR, WK, NST>::kThreads, 1)
+    splitkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+  using Cfg = SplitKvCfg<DQK, DV, BN, WR, WK, NST>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+  uint8_t *sQ = smem;
+  uint8_t *sRing = smem + Cfg::kQBytes;
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + Cfg::kBarOffset);
+  uint64_t *empty = full + NST;
+  uint64_t *qbar = empty + NST;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // --- work item -----------------------------------------------------------
+  int bid = blockIdx.x;
+  const int row_tile = bid % p.row_tiles;
+  bid /= p.row_tiles;
+  const int split = bid % p.splits;
+  const int bh = bid / p.splits;  // b * Hkv + kv head
+  const TileRows tr = tile_rows(p, row_tile, Cfg::kRT);
+  int k_lo, k_hi;
+  tile_key_range(p, tr, BN, split, k_lo, k_hi);
+  const int nblocks = (k_hi - k_lo) / BN;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], Cfg::kConsumers);
+    }
+    mbar_init(qbar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  if (warp == Cfg::kConsumers) {
+    // ===================== producer warp =====================
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      const int grow0 = bh * p.R + tr.row0;
+      mbar_arrive_expect_tx(qbar, Cfg::kQBytes);
+#pragma unroll
+      for (int bx = 0; bx < Cfg::kQBoxes; ++bx)
+        tma_load_2d(sQ + bx * Cfg::kRT * 128, &tm_q, qbar, bx * 64, grow0);
+      int issued = 0;
+      for (int t = 0; t < nblocks; ++t) {
+        const int s = t % NST;
+        const uint32_t ph = (uint32_t)(t / NST) & 1u;
+        if (!mbar_wait(&empty[s], ph ^ 1u, p.wd, kWdTmaEmpty)) break;
+        uint8_t *sK = sRing + s * Cfg::kStageBytes;
+        uint8_t *sV = sK + Cfg::kKBytes;
+        mbar_arrive_expect_tx(&full[s], Cfg::kStageBytes);
+        const int k0 = k_lo + t * BN;
+#pragma unroll
+        for (int bx = 0; bx < Cfg::kQBoxes; ++bx)
+          tma_load_3d(sK + bx * BN * 128, &tm_k, &full[s], bx * 64, k0, bh);
+#pragma unroll
+        for (int bx = 0; bx < Cfg::kVBoxes; ++bx)
+          tma_load_3d(sV + bx * BN * 128, &tm_v, &full[s], bx * 64, k0, bh);
+        issued = t + 1;
+      }
+      // Drain: no copy may still be landing in shared memory when the CTA
+      // exits (matters only when a wait gave up).
+      mbar_wait_drain(qbar, 0, p.wd);
+      for (int t = issued - NST > 0 ? issued - NST : 0; t < issued; ++t)
+        mbar_wait_drain(&full[t % NST], (uint32_t)(t / NST) & 1u, p.wd);
+    }
+    return;
+  }
+
+  // ===================== consumer warps =====================
+  const int rw = warp % WR;   // row group
+  const int kw = warp / WR;   // key slice
+  const int kw0 = kw * Cfg::kKW;
+  constexpr int kNT = Cfg::kKW / 8;   // n8 tiles of scores per warp
+  constexpr int kOT = DV / 8;         // n8 tiles of output
+  constexpr int kKS = DQK / 16;       // k16 steps of Q K^T
+
+  // the two rows this thread holds (local to the CTA tile) and their positions
+  const int lr_a = rw * 16 + (lane >> 2);
+  const int lr_b = lr_a + 8;
+  const int pos_a = ((tr.row0 + lr_a) % p.L) + p.off;
+  const int pos_b = ((tr.row0 + lr_b) % p.L) + p.off;
+
+  float o[kOT][4];
+#pragma unroll
+  for (int i = 0; i < kOT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+  float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
+
+  bool ok = mbar_wait(qbar, 0, p.wd, kWdTmaFull);
+  const uint32_t sQa = smem_u32(sQ);
+
+  for (int t = 0; ok && t < nblocks; ++t) {
+    const int s = t % NST;
+    const uint32_t ph = (uint32_t)(t / NST) & 1u;
+    if (!mbar_wait(&full[s], ph, p.wd, kWdTmaFull)) {
+      ok = false;
+      break;
+    }
+    const uint32_t sK = smem_u32(sRing + s * Cfg::kStageBytes);
+    const uint32_t sV = sK + Cfg::kKBytes;
+    const int k0 = k_lo + t * BN;
+
+    // ---- S = Q K^T for this warp's 16 rows x kKW keys ----
+    float sc[kNT][4];
+#pragma unroll
+    for (int i = 0; i < kNT; ++i) sc[i][0] = sc[i][1] = sc[i][2] = sc[i][3] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < kKS; ++ks) {
+      uint32_t a0, a1, a2, a3;
+      {
+        const int m = lane >> 3;
+        const uint32_t row = rw * 16 + (m & 1) * 8 + (lane & 7);
+        const uint32_t chunk = ks * 2 + (m >> 1);
+        ldsm_x4(sQa + (chunk >> 3) * (Cfg::kRT * 128) + sw128_offset(row, chunk & 7), a0, a1, a2,
+                a3);
+      }
+#pragma unroll
+      for (int n2 = 0; n2 < kNT / 2; ++n2) {
+        const int m = lane >> 3;
+        const uint32_t key = kw0 + n2 * 16 + (m >> 1) * 8 + (lane & 7);
+        const uint32_t chunk = ks * 2 + (m & 1);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(sK + (chunk >> 3) * (BN * 128) + sw128_offset(key, chunk & 7), b0, b1, b2, b3);
+        mma_16816<kBF16>(sc[2 * n2], a0, a1, a2, a3, b0, b1);
+        mma_16816<kBF16>(sc[2 * n2 + 1], a0, a1, a2, a3, b2, b3);
+      }
+    }
+
+    // ---- scale into the log2 domain, mask, online softmax ----
+#pragma unroll
+    for (int i = 0; i < kNT; ++i) {
+      sc[i][0] *= p.scale_log2;
+      sc[i][1] *= p.scale_log2;
+      sc[i][2] *= p.scale_log2;
+      sc[i][3] *= p.scale_log2;
+    }
+    if (block_needs_mask(p, tr, k0, BN)) {
+#pragma unroll
+      for (int i = 0; i < kNT; ++i) {
+        const int col = k0 + kw0 + i * 8 + (lane & 3) * 2;
+        if (!key_visible(p, pos_a, col)) sc[i][0] = -INFINITY;
+        if (!key_visible(p, pos_a, col + 1)) sc[i][1] = -INFINITY;
+        if (!key_visible(p, pos_b, col)) sc[i][2] = -INFINITY;
+        if (!key_visible(p, pos_b, col + 1)) sc[i][3] = -INFINITY;
+      }
+    }
+    float mx_a = -INFINITY, mx_b = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < kNT; ++i) {
+      mx_a = fmaxf(mx_a, fmaxf(sc[i][0], sc[i][1]));
+      mx_b = fmaxf(mx_b, fmaxf(sc[i][2], sc[i][3]));
+    }
+    mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 1));
+    mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 2));
+    mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 1));
+    mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 2));
+    const float mn_a = fmaxf(m_a, mx_a);
+    const float mn_b = fmaxf(m_b, mx_b);
+    // a row with nothing visible yet keeps m = -inf; use 0 as its reference
+    const float ref_a = mn_a == -INFINITY ? 0.f : mn_a;
+    const float ref_b = mn_b == -INFINITY ? 0.f : mn_b;
+    const float al_a = fast_exp2(m_a - ref_a);
+    const float al_b = fast_exp2(m_b - ref_b);
+    m_a = mn_a;
+    m_b = mn_b;
+    float rs_a = 0.f, rs_b = 0.f;
+#pragma unroll
+    for (int i = 0; i < kNT; ++i) {
+      sc[i][0] = fast_exp2(sc[i][0] - ref_a);
+      sc[i][1] = fast_exp2(sc[i][1] - ref_a);
+      sc[i][2] = fast_exp2(sc[i][2] - ref_b);
+      sc[i][3] = fast_exp2(sc[i][3] - ref_b);
+      rs_a += sc[i][0] + sc[i][1];
+      rs_b += sc[i][2] + sc[i][3];
+    }
+    l_a = l_a * al_a + rs_a;
+    l_b = l_b * al_b + rs_b;
+#pragma unroll
+    for (int i = 0; i < kOT; ++i) {
+      o[i][0] *= al_a;
+      o[i][1] *= al_a;
+      o[i][2] *= al_b;
+      o[i][3] *= al_b;
+    }
+
+    // ---- O += P V ----
+#pragma unroll
+    for (int kc = 0; kc < kNT / 2; ++kc) {
+      const uint32_t a0 = pack2<kBF16>(sc[2 * kc][0], sc[2 * kc][1]);
+      const uint32_t a1 = pack2<kBF16>(sc[2 * kc][2], sc[2 * kc][3]);
+      const uint32_t a2 = pack2<kBF16>(sc[2 * kc + 1][0], sc[2 * kc + 1][1]);
+      const uint32_t a3 = pack2<kBF16>(sc[2 * kc + 1][2], sc[2 * kc + 1][3]);
+#pragma unroll
+      for (int n2 = 0; n2 < kOT / 2; ++n2) {
+        const int m = lane >> 3;
+        const uint32_t key = kw0 + kc * 16 + (m & 1) * 8 + (lane & 7);
+        const uint32_t chunk = n2 * 2 + (m >> 1);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(sV + (chunk >> 3) * (BN * 128) + sw128_offset(key, chunk & 7), b0, b1, b2, b3);
+        mma_16816<kBF16>(o[2 * n2], a0, a1, a2, a3, b0, b1);
+        mma_16816<kBF16>(o[2 * n2 + 1], a0, a1, a2, a3, b2, b3);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+  }
+
+  // row sums: reduce the per-thread partials over the quad
+  l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
+  l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
+  l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
+  l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
+
+  if constexpr (WK > 1) {
+    // ---- merge the key slices through shared memory (ring is free now) ----
+    // layout: [warp][element][lane] floats, element = 0..DV/2-1 for O, then m_a, m_b, l_a, l_b
+    float *buf = reinterpret_cast<float *>(sRing);
+    constexpr int kE = DV / 2 + 4;
+    asm volatile("bar.sync 1, %0;" ::"n"(Cfg::kConsumers * 32) : "memory");
+    if (kw != 0) {
+      float *mine = buf + warp * kE * 32;
+#pragma unroll
+      for (int i = 0; i < kOT; ++i)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) mine[(i * 4 + e) * 32 + lane] = o[i][e];
+      mine[(DV / 2 + 0) * 32 + lane] = m_a;
+      mine[(DV / 2 + 1) * 32 + lane] = m_b;
+      mine[(DV / 2 + 2) * 32 + lane] = l_a;
+      mine[(DV / 2 + 3) * 32 + lane] = l_b;
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(Cfg::kConsumers * 32) : "memory");
+    if (kw != 0) return;
+    float mm_a = m_a, mm_b = m_b;
+#pragma unroll
+    for (int k = 1; k < WK; ++k) {
+      const float *other = buf + (k * WR + rw) * kE * 32;
+      mm_a = fmaxf(mm_a, other[(DV / 2 + 0) * 32 + lane]);
+      mm_b = fmaxf(mm_b, other[(DV / 2 + 1) * 32 + lane]);
+    }
+    const float rf_a = mm_a == -INFINITY ? 0.f : mm_a;
+    const float rf_b = mm_b == -INFINITY ? 0.f : mm_b;
+    float w_a = fast_exp2(m_a - rf_a), w_b = fast_exp2(m_b - rf_b);
+    l_a *= w_a;
+    l_b *= w_b;
+#pragma unroll
+    for (int i = 0; i < kOT; ++i) {
+      o[i][0] *= w_a;
+      o[i][1] *= w_a;
+      o[i][2] *= w_b;
+      o[i][3] *= w_b;
+    }
+#pragma unroll
+    for (int k = 1; k < WK; ++k) {
+      const float *other = buf + (k * WR + rw) * kE * 32;
+      const float ow_a = fast_exp2(other[(DV / 2 + 0) * 32 + lane] - rf_a);
+      const float ow_b = fast_exp2(other[(DV / 2 + 1) * 32 + lane] - rf_b);
+      l_a += ow_a * other[(DV / 2 + 2) * 32 + lane];
+      l_b += ow_b * other[(DV / 2 + 3) * 32 + lane];
+#pragma unroll
+      for (int i = 0; i < kOT; ++i) {
+        o[i][0] += ow_a * other[(i * 4 + 0) * 32 + lane];
+        o[i][1] += ow_a * other[(i * 4 + 1) * 32 + lane];
+        o[i][2] += ow_b * other[(i * 4 + 2) * 32 + lane];
+        o[i][3] += ow_b * other[(i * 4 + 3) * 32 + lane];
+      }
+    }
+    m_a = mm_a;
+    m_b = mm_b;
+  }
+
+  // ---- epilogue ----
+  const float inv_a = l_a > 0.f ? 1.f / l_a : 0.f;
+  const float inv_b = l_b > 0.f ? 1.f / l_b : 0.f;
+  const bool va = lr_a < tr.nvalid, vb = lr_b < tr.nvalid;
+  const long grow_a = (long)bh * p.R + tr.row0 + lr_a;
+  const long grow_b = grow_a + 8;
+  const int c0 = (lane & 3) * 2;
+  if (p.splits == 1) {
+    uint32_t *out32 = reinterpret_cast<uint32_t *>(p.out);
+#pragma unroll
+    for (int i = 0; i < kOT; ++i) {
+      const int col = i * 8 + c0;
+      if (col < p.Dv) {
+        if (va) out32[(grow_a * p.Dv + col) >> 1] = pack2<kBF16>(o[i][0] * inv_a, o[i][1] * inv_a);
+        if (vb) out32[(grow_b * p.Dv + col) >> 1] = pack2<kBF16>(o[i][2] * inv_b, o[i][3] * inv_b);
+      }
+    }
+  } else {
+    const long total_rows = (long)p.B * p.Hq * p.L;
+    float *po = p.part_o + (long)split * total_rows * p.Dv;
+#pragma unroll
+    for (int i = 0; i < kOT; ++i) {
+      const int col = i * 8 + c0;
+      if (col < p.Dv) {
+        if (va)
+          *reinterpret_cast<float2 *>(po + grow_a * p.Dv + col) =
+              make_float2(o[i][0] * inv_a, o[i][1] * inv_a);
+        if (vb)
+          *reinterpret_cast<float2 *>(po + grow_b * p.Dv + col) =
+              make_float2(o[i][2] * inv_b, o[i][3] * inv_b);
+      }
+    }
+    if ((lane & 3) == 0) {
+      constexpr float kLn2 = 0.693147180559945309f;
+      float *pl = p.part_lse + (long)split * total_rows;
+      if (va) pl[grow_a] = l_a > 0.f ? (m_a + log2f(l_a)) * kLn2 : -INFINITY;
+      if (vb) pl[grow_b] = l_b > 0.f ? (m_b + log2f(l_b)) * kLn2 : -INFINITY;
+    }
+  }
+  (void)ok;
+}
+
+// ---------------------------------------------------------------------------
+// Log-sum-exp combine of split partials (mlx issue #3826: split over S, then
+// a log-sum-exp merge; mlx PR #3637: the 2-pass kernel's aggregation).
+// One warp per output row:
+//   LSE = max_s LSE_s + ln sum_s exp(LSE_s - max),  O = sum_s exp(LSE_s - LSE) O_s
+// Splits that saw no visible key carry LSE_s = -inf and weight 0.
+// ---------------------------------------------------------------------------
+template <bool kBF16>
+__global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ part_o,
+                                                      const float *__restrict__ part_lse,
+                                                      void *__restrict__ out, float *lse_out,
+                                                      long total_rows, int Dv, int splits) {
+  const long row = (long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= total_rows) return;
+  float mx = -INFINITY;
+  for (int s = lane; s < splits; s += 32) mx = fmaxf(mx, part_lse[(long)s * total_rows + row]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  const float ref = mx == -INFINITY ? 0.f : mx;
+  float den = 0.f;
+  for (int s = lane; s < splits; s += 32) den += __expf(part_lse[(long)s * total_rows + row] - ref);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  for (int d = lane; d < Dv; d += 32) {
+    float acc = 0.f;
+    for (int s = 0; s < splits; ++s) {
+      const float w = __expf(part_lse[(long)s * total_rows + row] - ref);
+      acc += w * part_o[((long)s * total_rows + row) * Dv + d];
+    }
+    acc *= inv;
+    if constexpr (kBF16)
+      reinterpret_cast<__nv_bfloat16 *>(out)[row * Dv + d] = __float2bfloat16_rn(acc);
+    else
+      reinterpret_cast<__half *>(out)[row * Dv + d] = __float2half_rn(acc);
+  }
+  if (lse_out != nullptr && lane == 0) lse_out[row] = den > 0.f ? ref + logf(den) : -INFINITY;
+}
+
+}  // namespace sdpa

@@ -1,0 +1,144 @@
+"""C-ABI library: loads, exports what the header declares, validates on the
+host and plans without a GPU (CPU only; no compute call is made)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import scaled_dot_product_13_b200 as sdpa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    text = open(os.path.join(ROOT, "include", "sdpa.h")).read()
+    return sorted(set(re.findall(r"SDPA_API\s+[\w\s\*]*?\b(sdpa_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return sdpa.load_library()
+
+
+def test_header_declares_entry_points():
+    names = _declared_functions()
+    for must in ("sdpa_forward", "sdpa_forward_ws", "sdpa_workspace_bytes", "sdpa_plan",
+                 "sdpa_status_string", "sdpa_last_error_message", "sdpa_version"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared_functions():
+        assert hasattr(lib, name), f"libsdpa.so does not export {name}"
+
+
+def test_version_and_status_strings(lib):
+    assert lib.sdpa_version() >= 100
+    for code, name in sdpa.STATUS.items():
+        assert lib.sdpa_status_string(code).decode() == name
+
+
+def _plan_err(**kw):
+    args = dict(B=1, Hq=8, Hkv=2, L=4, S=64, Dqk=128, Dv=128, causal=True, window_size=0,
+                dtype="bf16", num_sms=148)
+    args.update(kw)
+    with pytest.raises(sdpa.SdpaError) as ei:
+        sdpa.plan(**args)
+    return ei.value
+
+
+@pytest.mark.parametrize("kw,status,words", [
+    (dict(Hq=6, Hkv=4), 1, "multiple of Hkv"),
+    (dict(L=65, S=64), 1, "L <= S"),
+    (dict(window_size=-1), 1, "window_size"),
+    (dict(window_size=8, causal=False), 2, "causal"),
+    (dict(Dqk=512, Dv=512), 2, "head dims"),
+    (dict(Dqk=72, Dv=100), 2, "multiples of 8"),
+    (dict(B=0), 1, ">= 1"),
+    (dict(S=0), 1, ">= 1"),
+])
+def test_invalid_problems_name_the_constraint(kw, status, words):
+    e = _plan_err(**kw)
+    assert e.status == status
+    assert words in e.message
+
+
+def test_non_causal_long_query_is_allowed():
+    info = sdpa.plan(1, 4, 4, 100, 50, 64, 64, causal=False, num_sms=148)
+    assert info["rows"] == 100
+
+
+def test_forward_rejects_null_pointers_before_any_cuda_call(lib):
+    st = lib.sdpa_forward(None, None, None, None, 1, 1, 1, 1, 1, 64, 64, 1.0, 0, 0, 0, None)
+    assert st == 1
+    assert b"non-NULL" in lib.sdpa_last_error_message()
+
+
+def test_forward_rejects_misaligned_pointers(lib):
+    st = lib.sdpa_forward(0x1000, 0x2008, 0x3000, 0x4000, 1, 1, 1, 1, 1, 64, 64, 1.0, 0, 0, 0,
+                          None)
+    assert st == 1
+    assert b"16-byte" in lib.sdpa_last_error_message()
+
+
+def test_forward_rejects_overlapping_output(lib):
+    st = lib.sdpa_forward(0x10000, 0x20000, 0x30000, 0x10000, 1, 1, 1, 4, 4, 64, 64, 1.0, 0, 0,
+                          0, None)
+    assert st == 1
+    assert b"overlap" in lib.sdpa_last_error_message()
+
+
+def test_plan_decode_splits_keys_across_sms():
+    # decode, 64 query heads over 4 KV heads: 16 packed rows per KV head
+    info = sdpa.plan(1, 64, 4, 1, 32768, 192, 128, causal=True, num_sms=148)
+    assert info["rows"] == 16 and info["row_tiles"] == 1
+    assert info["splits"] > 1 and info["launches"] == 2
+    assert info["ctas"] <= 148 and info["ctas"] >= 100
+    assert info["keys_per_split"] * info["splits"] >= 32768
+    assert info["workspace_bytes"] > 0
+
+
+def test_plan_packs_verify_rows_per_kv_head():
+    # verify, GQA 32/8: the 4*L rows of one KV head are packed together
+    for L in (1, 2, 4, 8, 12, 16, 24, 32, 48, 64):
+        info = sdpa.plan(1, 32, 8, L, 16384, 128, 128, causal=False, dtype="f16", num_sms=148)
+        assert info["rows"] == 4 * L
+        assert info["row_tiles"] * info["row_tile"] >= 4 * L
+        assert info["row_tiles"] * info["row_tile"] < 4 * L + info["row_tile"]
+
+
+def test_plan_forced_splits_and_single_split_needs_no_workspace():
+    info = sdpa.plan(1, 8, 2, 3, 1000, 64, 64, causal=True, num_sms=148, force_splits=1)
+    assert info["splits"] == 1 and info["workspace_bytes"] == 0 and info["launches"] == 1
+    info = sdpa.plan(1, 8, 2, 3, 1000, 64, 64, causal=True, num_sms=148, force_splits=7)
+    assert info["splits"] == 7 and info["launches"] == 2
+
+
+def test_plan_head_dim_instances():
+    assert sdpa.plan(1, 16, 16, 1024, 1024, 72, 72, num_sms=148)["dqk_pad"] == 80
+    i = sdpa.plan(1, 64, 4, 1, 256, 192, 128, causal=True, num_sms=148)
+    assert (i["dqk_pad"], i["dv_pad"]) == (192, 128)
+    assert sdpa.plan(1, 16, 8, 2048, 2048, 256, 256, causal=True, window_size=1024,
+                     num_sms=148)["dqk_pad"] == 256
+
+
+def test_workspace_query_without_device_fails_loudly(lib):
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("CPU-only check")
+    n = lib.sdpa_workspace_bytes(1, 64, 4, 1, 32768, 192, 128, 1, 0, 0)
+    assert n == 0
+    assert lib.sdpa_last_error_message() != b""
+
+
+def test_forward_without_device_fails_loudly(lib):
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("CPU-only check")
+    st = lib.sdpa_forward(0x10000, 0x20000, 0x30000, 0x40000, 1, 1, 1, 1, 1, 64, 64, 1.0, 0, 0,
+                          0, None)
+    assert st == 4
+    assert b"CUDA" in lib.sdpa_last_error_message() or b"device" in lib.sdpa_last_error_message()
