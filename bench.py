@@ -160,6 +160,8 @@ def time_cases(sdpa, cases, steps, warmup, flush, sync_all):
         for c in cases:
             flush.zero_()
             e0, e1, m0, m1 = (torch.cuda.Event(enable_timing=True) for _ in range(4))
+            m0.record(stream)  # creates the CUDA handles; the library re-records them
+            m1.record(stream)
             e0.record(stream)
             sdpa.time_next_main_kernel(m0, m1)
             c.call(sdpa)
@@ -256,6 +258,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the prefill / verify / encoder objects")
+    ap.add_argument("--only", default=None,
+                    help="restrict the timed sweep to the named problem (profiling)")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing")
     args = ap.parse_args()
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
@@ -274,6 +280,11 @@ def main():
     torch.cuda.set_device(device)
 
     probs = I.decode_problems()
+    if args.only:
+        probs = [p for p in probs + I.verify_problems() + I.window_problems() +
+                 I.encoder_problems() + [I.tiny_problem()] if p.name == args.only]
+        if not probs:
+            raise SystemExit(f"unknown problem {args.only}")
     peaks, peak_src = load_peaks()
     workload = {"workload": "decode split-KV sweep: B=1, Hq=64, Hkv in {4,8}, L=1, "
                             "S in {256,1024,4096,8192,16384,32768}, Dqk=192, Dv=128, bf16, causal",
@@ -363,7 +374,10 @@ def main():
                        "splits": c.info["splits"], "ctas": c.info["ctas"]})
     launches = sum(c.info["launches"] for c in cases) * args.steps
 
-    e2e_ms, h2d, d2h = time_e2e(sdpa, cases, max(3, args.steps // 4), 2, device)
+    if args.no_e2e:
+        e2e_ms, h2d, d2h = [float("nan")], 0, 0
+    else:
+        e2e_ms, h2d, d2h = time_e2e(sdpa, cases, max(3, args.steps // 4), 2, device)
     e2e_val = step_bytes / (float(np.mean(e2e_ms)) * 1e-3) / 1e9 * world
     del cases
     torch.cuda.empty_cache()
@@ -389,7 +403,7 @@ def main():
                     "ms_per_step": round(float(np.mean(e2e_ms)), 3)},
             "points": points}
     line.update(extra)
-    if rank == 0 and world == 1:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
         host_cases = [HostCase(p) for p in I.decode_problems()]
         val, secs, cores, calls = oracle_sample(host_cases, budget_s=10.0)
         line["cpu_baseline"] = {"value": round(val, 4), "unit": "GB/s (KV, decode)",

@@ -212,7 +212,10 @@ def device_status(clear: bool = True) -> None:
 
 def time_next_main_kernel(start_event, stop_event) -> None:
     """Arm the profiling hook: the next call on this thread records the two
-    torch.cuda.Event objects around its main attention kernel."""
+    torch.cuda.Event objects around its main attention kernel.  The events
+    must already hold a CUDA handle (record them once beforehand)."""
+    if not start_event.cuda_event or not stop_event.cuda_event:
+        raise SdpaError(1, "events have no CUDA handle yet; record them once first")
     load_library().sdpa_time_next_main_kernel(ctypes.c_void_p(start_event.cuda_event),
                                               ctypes.c_void_p(stop_event.cuda_event))
 
