@@ -130,6 +130,13 @@ int pick_pair(int dqk, int dv) {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Upper bound on key splits (the combine keeps one weight per split in
+// shared memory).
+constexpr int kMaxSplits = 4096;
+
+// Packed rows per (batch, KV head) from which the tcgen05 path is taken.
+constexpr int kTcRowThreshold = 128;
+
 sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_splits,
                       Plan *out) {
   Plan pl;
@@ -145,19 +152,28 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
   const int g = pb.Hq / pb.Hkv;
   pl.rows = g * pb.L;
 
-  if (force_path == SDPA_PATH_TC)
-    return fail(SDPA_ERR_UNSUPPORTED, "the tcgen05 tile path is not available in this build");
-  pl.path = SDPA_PATH_SPLITKV;
-  if (pl.rows <= 16) {
-    pl.wr = 1; pl.wk = 4;
-  } else if (pl.rows <= 32) {
-    pl.wr = 2; pl.wk = 2;
+  // Route: packed rows that fill a 128-row tensor-core tile go to the
+  // tcgen05 kernel; fewer rows (decode, short verify windows) go to the
+  // split-KV kernel on 16-row warp tiles.  Both split the keys when the
+  // tiles alone do not fill the GPU.
+  int path = force_path;
+  if (path == SDPA_PATH_AUTO) path = pl.rows >= kTcRowThreshold ? SDPA_PATH_TC : SDPA_PATH_SPLITKV;
+  pl.path = path;
+  if (path == SDPA_PATH_TC) {
+    pl.wr = 0; pl.wk = 0;
+    pl.row_tile = kTcRows;
+    pl.key_block = tc_key_block(kDimPairs[pl.pair].dqk, kDimPairs[pl.pair].dv);
   } else {
-    pl.wr = 4; pl.wk = 1;
+    if (pl.rows <= 16) {
+      pl.wr = 1; pl.wk = 4;
+    } else if (pl.rows <= 32) {
+      pl.wr = 2; pl.wk = 2;
+    } else {
+      pl.wr = 4; pl.wk = 1;
+    }
+    pl.row_tile = 16 * pl.wr;
+    pl.key_block = kSplitKvBN;
   }
-  pl.row_tile = 16 * pl.wr;
-  pl.key_block = kSplitKvBN;
-
   pl.row_tiles = (pl.rows + pl.row_tile - 1) / pl.row_tile;
   // keys visible to at least one row: [kbeg, S); the last row sits at S-1
   const int off = pb.S - pb.L;
@@ -175,6 +191,7 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
     splits = (int)std::max(1LL, num_sms / base);
     splits = std::min(splits, nkb);
   }
+  splits = std::min(splits, kMaxSplits);
   const int bps = (nkb + splits - 1) / splits;
   if (force_splits == 0) splits = (nkb + bps - 1) / bps;
   pl.splits = splits;
@@ -259,12 +276,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+}  // namespace
+
 // ---------------------------------------------------------------------------
 // the call
 // ---------------------------------------------------------------------------
-sdpa_status run(const Problem &pb, const void *q, const void *k, const void *v, void *out,
-                int force_path, int force_splits, void *ws, size_t ws_bytes, bool own_ws,
-                cudaStream_t stream) {
+sdpa_status forward_call(const Problem &pb, const void *q, const void *k, const void *v,
+                         void *out, int force_path, int force_splits, void *ws, size_t ws_bytes,
+                         bool own_ws, cudaStream_t stream) {
   sdpa_status st = validate_shape(pb);
   if (st != SDPA_OK) return st;
   st = validate_pointers(pb, q, k, v, out);
@@ -304,11 +323,10 @@ sdpa_status run(const Problem &pb, const void *q, const void *k, const void *v, 
   ln.stream = stream;
 
   std::string err;
-  cudaEvent_t ev0 = t_ev_start, ev1 = t_ev_stop;
+  ln.ev_start = t_ev_start;
+  ln.ev_stop = t_ev_stop;
   t_ev_start = t_ev_stop = nullptr;
-  if (ev0) cudaEventRecord(ev0, stream);
-  st = launch_splitkv(ln, &err);
-  if (ev1) cudaEventRecord(ev1, stream);
+  st = pl.path == SDPA_PATH_TC ? launch_tc(ln, &err) : launch_splitkv(ln, &err);
   if (st == SDPA_OK && pl.splits > 1) st = launch_combine(ln, &err);
   if (allocated) {
     cudaError_t e = cudaFreeAsync(ws, stream);
@@ -321,7 +339,17 @@ sdpa_status run(const Problem &pb, const void *q, const void *k, const void *v, 
   return SDPA_OK;
 }
 
-}  // namespace
+sdpa_status plan_call(const Problem &pb, int force_path, int force_splits, Plan *plan) {
+  sdpa_status st = validate_shape(pb);
+  if (st != SDPA_OK) return st;
+  int dev, sms;
+  unsigned int *wd;
+  st = device_state(&dev, &sms, &wd);
+  if (st != SDPA_OK) return st;
+  return make_plan(pb, sms, force_path, force_splits, plan);
+}
+
+sdpa_status set_error(sdpa_status st, const std::string &msg) { return fail_str(st, msg); }
 
 // ---------------------------------------------------------------------------
 // shared helpers declared in launch.h
@@ -439,7 +467,7 @@ sdpa_status sdpa_forward(const void *q, const void *k, const void *v, void *out,
                          int Hkv, int L, int S, int Dqk, int Dv, float scale, int causal,
                          int window_size, sdpa_dtype dtype, sdpa_stream_t stream) {
   t_last_error.clear();
-  return run(make_problem(B, Hq, Hkv, L, S, Dqk, Dv, scale, causal, window_size, dtype), q, k, v,
+  return forward_call(make_problem(B, Hq, Hkv, L, S, Dqk, Dv, scale, causal, window_size, dtype), q, k, v,
              out, SDPA_PATH_AUTO, 0, nullptr, 0, true, (cudaStream_t)stream);
 }
 
@@ -461,7 +489,7 @@ sdpa_status sdpa_forward_ws(const void *q, const void *k, const void *v, void *o
                             int causal, int window_size, sdpa_dtype dtype, void *workspace,
                             size_t workspace_bytes, sdpa_stream_t stream) {
   t_last_error.clear();
-  return run(make_problem(B, Hq, Hkv, L, S, Dqk, Dv, scale, causal, window_size, dtype), q, k, v,
+  return forward_call(make_problem(B, Hq, Hkv, L, S, Dqk, Dv, scale, causal, window_size, dtype), q, k, v,
              out, SDPA_PATH_AUTO, 0, workspace, workspace_bytes, false, (cudaStream_t)stream);
 }
 
@@ -486,7 +514,7 @@ sdpa_status sdpa_forward_planned(const void *q, const void *k, const void *v, vo
                                  int force_splits, void *workspace, size_t workspace_bytes,
                                  sdpa_stream_t stream) {
   t_last_error.clear();
-  return run(make_problem(B, Hq, Hkv, L, S, Dqk, Dv, scale, causal, window_size, dtype), q, k, v,
+  return forward_call(make_problem(B, Hq, Hkv, L, S, Dqk, Dv, scale, causal, window_size, dtype), q, k, v,
              out, force_path, force_splits, workspace, workspace_bytes, false,
              (cudaStream_t)stream);
 }

@@ -25,6 +25,13 @@ constexpr int kNumDimPairs = sizeof(kDimPairs) / sizeof(kDimPairs[0]);
 // Key block of the split-KV kernel (keys per pipeline stage).
 constexpr int kSplitKvBN = 64;
 
+// Key block of the tcgen05 kernel: 128 keys while two 128-key score buffers
+// plus O fit TMEM and the slots fit shared memory; 64 for head dims > 128.
+constexpr int tc_key_block(int dqk, int dv) { return (dqk > 128 || dv > 128) ? 64 : 128; }
+
+// Rows of one tcgen05 tile.
+constexpr int kTcRows = 128;
+
 struct Problem {
   int B, Hq, Hkv, L, S, Dqk, Dv;
   float scale;
@@ -59,7 +66,21 @@ struct Launch {
   unsigned int *wd_word;
   uint64_t wd_limit_ns;
   cudaStream_t stream;
+  cudaEvent_t ev_start, ev_stop;  // optional, recorded around the main kernel launch
 };
+
+// Validate, plan for the current device and enqueue one call (the body of
+// every sdpa_forward* entry point).  own_ws: take the split workspace from
+// the stream-ordered pool; otherwise use (ws, ws_bytes).
+sdpa_status forward_call(const Problem &pb, const void *q, const void *k, const void *v,
+                         void *out, int force_path, int force_splits, void *ws, size_t ws_bytes,
+                         bool own_ws, cudaStream_t stream);
+
+// Validate and plan for the current device without enqueuing anything.
+sdpa_status plan_call(const Problem &pb, int force_path, int force_splits, Plan *plan);
+
+// Record `msg` as this thread's last error and return `st`.
+sdpa_status set_error(sdpa_status st, const std::string &msg);
 
 // Encode a tiled TMA descriptor (128-byte swizzle, zero fill out of bounds).
 // rank 2 or 3; dims/strides in elements/bytes as cuTensorMapEncodeTiled wants.
@@ -69,6 +90,7 @@ bool encode_tma(CUtensorMap *map, sdpa_dtype dt, int rank, const void *base,
 
 // Per-path launchers (return SDPA_OK or an error with *err set).
 sdpa_status launch_splitkv(const Launch &ln, std::string *err);
+sdpa_status launch_tc(const Launch &ln, std::string *err);
 sdpa_status launch_combine(const Launch &ln, std::string *err);
 
 // Checks that a kernel fits the device (threads, shared memory) before its

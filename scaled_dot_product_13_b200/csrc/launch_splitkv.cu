@@ -61,7 +61,9 @@ sdpa_status run_splitkv(const Launch &ln, std::string *err) {
   p.part_lse = ln.part_lse;
   p.wd.word = ln.wd_word;
   p.wd.limit_ns = ln.wd_limit_ns;
+  if (ln.ev_start) cudaEventRecord(ln.ev_start, ln.stream);
   kern<<<(unsigned)pl.ctas, Cfg::kThreads, Cfg::kSmemBytes, ln.stream>>>(tq, tk, tv, p);
+  if (ln.ev_stop) cudaEventRecord(ln.ev_stop, ln.stream);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     *err = std::string("splitkv_kernel launch failed: ") + cudaGetErrorString(e);
@@ -101,15 +103,30 @@ sdpa_status launch_splitkv(const Launch &ln, std::string *err) {
 }
 
 sdpa_status launch_combine(const Launch &ln, std::string *err) {
+  // Launched as a programmatic dependent of the attention pass: its CTAs may
+  // be scheduled before that grid finishes and wait (griddepcontrol.wait) for
+  // it, which hides the second launch's latency.
   const long total = (long)ln.pb.B * ln.pb.Hq * ln.pb.L;
-  const unsigned grid = (unsigned)((total + 7) / 8);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)total);
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = (size_t)ln.plan.splits * sizeof(float);
+  cfg.stream = ln.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e;
   if (ln.pb.dtype == SDPA_BF16)
-    combine_kernel<true><<<grid, 256, 0, ln.stream>>>(ln.part_o, ln.part_lse, ln.out, ln.lse_out,
-                                                      total, ln.pb.Dv, ln.plan.splits);
+    e = cudaLaunchKernelEx(&cfg, combine_kernel<true>, (const float *)ln.part_o,
+                           (const float *)ln.part_lse, ln.out, ln.lse_out, total, ln.pb.Dv,
+                           ln.plan.splits);
   else
-    combine_kernel<false><<<grid, 256, 0, ln.stream>>>(ln.part_o, ln.part_lse, ln.out, ln.lse_out,
-                                                       total, ln.pb.Dv, ln.plan.splits);
-  cudaError_t e = cudaGetLastError();
+    e = cudaLaunchKernelEx(&cfg, combine_kernel<false>, (const float *)ln.part_o,
+                           (const float *)ln.part_lse, ln.out, ln.lse_out, total, ln.pb.Dv,
+                           ln.plan.splits);
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) {
     *err = std::string("combine_kernel launch failed: ") + cudaGetErrorString(e);
     return SDPA_ERR_CUDA;

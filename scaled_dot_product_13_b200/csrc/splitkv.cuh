@@ -324,6 +324,7 @@ __global__ void __launch_bounds__(SplitKvCfg<DQK, DV, BN, WR, WK, NST>::kThreads
   }
 
   // ---- epilogue ----
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const float inv_a = l_a > 0.f ? 1.f / l_a : 0.f;
   const float inv_b = l_b > 0.f ? 1.f / l_b : 0.f;
   const bool va = lr_a < tr.nvalid, vb = lr_b < tr.nvalid;
@@ -368,41 +369,66 @@ __global__ void __launch_bounds__(SplitKvCfg<DQK, DV, BN, WR, WK, NST>::kThreads
 // ---------------------------------------------------------------------------
 // Log-sum-exp combine of split partials (mlx issue #3826: split over S, then
 // a log-sum-exp merge; mlx PR #3637: the 2-pass kernel's aggregation).
-// One warp per output row:
+// One CTA of 128 threads per output row:
 //   LSE = max_s LSE_s + ln sum_s exp(LSE_s - max),  O = sum_s exp(LSE_s - LSE) O_s
-// Splits that saw no visible key carry LSE_s = -inf and weight 0.
+// Splits that saw no visible key carry LSE_s = -inf and weight 0.  The
+// weights go to shared memory once; each thread then owns output columns
+// and reads the splits' partials with several loads in flight.
+// Launched as a programmatic dependent of the split pass: it waits for that
+// grid (griddepcontrol.wait) before touching the partials.
 // ---------------------------------------------------------------------------
 template <bool kBF16>
-__global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ part_o,
+__global__ void __launch_bounds__(128) combine_kernel(const float *__restrict__ part_o,
                                                       const float *__restrict__ part_lse,
                                                       void *__restrict__ out, float *lse_out,
                                                       long total_rows, int Dv, int splits) {
-  const long row = (long)blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= total_rows) return;
+  extern __shared__ float s_w[];  // [splits]
+  __shared__ float s_red[4];
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const long row = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   float mx = -INFINITY;
-  for (int s = lane; s < splits; s += 32) mx = fmaxf(mx, part_lse[(long)s * total_rows + row]);
+  for (int s = tid; s < splits; s += 128) mx = fmaxf(mx, part_lse[(long)s * total_rows + row]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if (lane == 0) s_red[wid] = mx;
+  __syncthreads();
+  mx = fmaxf(fmaxf(s_red[0], s_red[1]), fmaxf(s_red[2], s_red[3]));
   const float ref = mx == -INFINITY ? 0.f : mx;
+  __syncthreads();
   float den = 0.f;
-  for (int s = lane; s < splits; s += 32) den += __expf(part_lse[(long)s * total_rows + row] - ref);
+  for (int s = tid; s < splits; s += 128) {
+    const float w = __expf(part_lse[(long)s * total_rows + row] - ref);
+    s_w[s] = w;
+    den += w;
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+  if (lane == 0) s_red[wid] = den;
+  __syncthreads();
+  den = s_red[0] + s_red[1] + s_red[2] + s_red[3];
   const float inv = den > 0.f ? 1.f / den : 0.f;
-  for (int d = lane; d < Dv; d += 32) {
-    float acc = 0.f;
-    for (int s = 0; s < splits; ++s) {
-      const float w = __expf(part_lse[(long)s * total_rows + row] - ref);
-      acc += w * part_o[((long)s * total_rows + row) * Dv + d];
+  const long stride = total_rows * Dv;
+  for (int d = tid; d < Dv; d += 128) {
+    const float *src = part_o + row * Dv + d;
+    float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+    int s = 0;
+    for (; s + 4 <= splits; s += 4) {
+      const float v0 = src[(long)(s + 0) * stride], v1 = src[(long)(s + 1) * stride];
+      const float v2 = src[(long)(s + 2) * stride], v3 = src[(long)(s + 3) * stride];
+      acc0 += s_w[s + 0] * v0;
+      acc1 += s_w[s + 1] * v1;
+      acc2 += s_w[s + 2] * v2;
+      acc3 += s_w[s + 3] * v3;
     }
-    acc *= inv;
+    for (; s < splits; ++s) acc0 += s_w[s] * src[(long)s * stride];
+    const float acc = ((acc0 + acc1) + (acc2 + acc3)) * inv;
     if constexpr (kBF16)
       reinterpret_cast<__nv_bfloat16 *>(out)[row * Dv + d] = __float2bfloat16_rn(acc);
     else
       reinterpret_cast<__half *>(out)[row * Dv + d] = __float2half_rn(acc);
   }
-  if (lse_out != nullptr && lane == 0) lse_out[row] = den > 0.f ? ref + logf(den) : -INFINITY;
+  if (lse_out != nullptr && tid == 0) lse_out[row] = den > 0.f ? ref + logf(den) : -INFINITY;
 }
 
 }  // namespace sdpa
