@@ -140,6 +140,27 @@ class Case:
                         causal=self.p.causal, window_size=self.p.window, out=self.out)
 
 
+def flush_l2(buf):
+    """Evict L2: write a buffer larger than L2, then read it back so that the
+    lines left in L2 are clean (the next kernel pays no write-back)."""
+    buf.zero_()
+    return buf.sum()
+
+
+def max_over_ranks(x: float, dist, device) -> float:
+    """Max of a per-rank float over all ranks (identity without a group)."""
+    if dist is None:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(world: int, bytes_per_rank_step: float, steps: int, max_total_ms: float) -> float:
+    """Whole-job throughput: every rank's bytes over the slowest rank's time."""
+    return world * bytes_per_rank_step * steps / (max_total_ms * 1e-3) / 1e9
+
+
 class HostCase:
     """A problem's seeded inputs on the host (for the CPU oracle)."""
 
@@ -158,7 +179,7 @@ def time_cases(sdpa, cases, steps, warmup, flush, sync_all):
     for it in range(warmup + steps):
         evs = []
         for c in cases:
-            flush.zero_()
+            flush_l2(flush)
             e0, e1, m0, m1 = (torch.cuda.Event(enable_timing=True) for _ in range(4))
             m0.record(stream)  # creates the CUDA handles; the library re-records them
             m1.record(stream)
@@ -288,7 +309,7 @@ def main():
     peaks, peak_src = load_peaks()
     workload = {"workload": "decode split-KV sweep: B=1, Hq=64, Hkv in {4,8}, L=1, "
                             "S in {256,1024,4096,8192,16384,32768}, Dqk=192, Dv=128, bf16, causal",
-                "calls_per_step": len(probs), "l2": "flushed before every call (2x L2 write)",
+                "calls_per_step": len(probs), "l2": "flushed before every call (2x L2 buffer written, then read)",
                 "parallelism": f"replicas x{world} (independent KV-head units, no collective)"}
 
     if args.impl == "reference":
@@ -343,14 +364,9 @@ def main():
     per_step_ms = [sum(cm[s] for cm in call_ms) for s in range(args.steps)]
     local_ms = float(np.mean(per_step_ms))
     local_total = float(sum(per_step_ms))
-    if dist is not None:
-        t = torch.tensor([local_total], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-    else:
-        total_ms = local_total
+    total_ms = max_over_ranks(local_total, dist, device)
     step_bytes = sum(c.kv_bytes for c in cases)
-    value = world * step_bytes * args.steps / (total_ms * 1e-3) / 1e9
+    value = whole_job_gbs(world, step_bytes, args.steps, total_ms)
 
     # roofline of the dominant kernel: the split-KV pass of the largest call
     big = max(range(len(cases)), key=lambda i: cases[i].kv_bytes)
