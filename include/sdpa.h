@@ -137,6 +137,41 @@ SDPA_API sdpa_status sdpa_forward_ws(const void *q, const void *k, const void *v
                             sdpa_dtype dtype, void *workspace, size_t workspace_bytes,
                             sdpa_stream_t stream);
 
+/*
+ * sdpa_forward_noalloc: as sdpa_forward, for callers that cannot allocate
+ * device memory.  (This entry point has no counterpart in the pages; it is
+ * a service of this library.)
+ *
+ * Who needs it: code that must not call cudaMalloc or cudaMallocAsync, for
+ * example a runtime whose device memory is owned by an allocator it cannot
+ * reach at the point of the call, or a latency-critical loop where an
+ * allocation could synchronise the device or grow a memory pool mid-run.
+ * sdpa_forward allocates its split workspace and sdpa_forward_ws needs the
+ * caller to provide one; this call does neither.
+ *
+ * How: when the router splits the keys, the fp32 partial outputs and
+ * log-sum-exp values go to one fixed scratch array of 16 MiB that the library
+ * keeps in each GPU's memory from load until process exit.  The call
+ * allocates nothing (no cudaMalloc, cudaFree or allocating library routine).
+ * The caller still passes q, k, v and out.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - Problems whose split workspace (sdpa_workspace_bytes) exceeds 16 MiB
+ *     are rejected with SDPA_ERR_RESOURCES and a message; use sdpa_forward or
+ *     sdpa_forward_ws for them.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     contents.  Nothing in it needs clearing: each call writes every element
+ *     it later reads.  Calls whose kernels overlap on the GPU (different
+ *     streams, or several host threads) race on the array and may return
+ *     wrong results; order them on one stream or use sdpa_forward_ws.
+ * Other arguments, validation and errors as sdpa_forward.
+ */
+SDPA_API sdpa_status sdpa_forward_noalloc(const void *q, const void *k, const void *v, void *out,
+                                          int B, int Hq, int Hkv, int L, int S, int Dqk, int Dv,
+                                          float scale, int causal, int window_size,
+                                          sdpa_dtype dtype, sdpa_stream_t stream);
+
 /* What the router decides for one problem.  Host-only, no CUDA call. */
 typedef struct {
   int path;          /* sdpa_path actually taken (never AUTO)               */

@@ -18,7 +18,7 @@ from __future__ import annotations
 import ctypes
 import os
 
-__all__ = ["forward", "forward_ws", "workspace_bytes", "plan", "device_status",
+__all__ = ["forward", "forward_ws", "forward_noalloc", "workspace_bytes", "plan", "device_status",
            "set_wait_limit_ns", "watchdog_selftest", "time_next_main_kernel", "load_library", "library_path",
            "SdpaError", "PATH_AUTO", "PATH_SPLITKV", "PATH_TC", "STATUS"]
 
@@ -66,6 +66,7 @@ def load_library() -> ctypes.CDLL:
     common = [vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, i, i]
     lib.sdpa_forward.argtypes = common + [vp]
     lib.sdpa_forward_ws.argtypes = common + [vp, sz, vp]
+    lib.sdpa_forward_noalloc.argtypes = common + [vp]
     lib.sdpa_forward_planned.argtypes = common + [i, i, vp, sz, vp]
     lib.sdpa_workspace_bytes.argtypes = [i] * 10
     lib.sdpa_workspace_bytes.restype = sz
@@ -79,7 +80,7 @@ def load_library() -> ctypes.CDLL:
     lib.sdpa_status_string.restype = ctypes.c_char_p
     lib.sdpa_status_string.argtypes = [i]
     lib.sdpa_last_error_message.restype = ctypes.c_char_p
-    for fn in ("sdpa_forward", "sdpa_forward_ws", "sdpa_forward_planned", "sdpa_plan",
+    for fn in ("sdpa_forward", "sdpa_forward_ws", "sdpa_forward_noalloc", "sdpa_forward_planned", "sdpa_plan",
                "sdpa_device_status", "sdpa_watchdog_selftest"):
         getattr(lib, fn).restype = ctypes.c_int
     _LIB = lib
@@ -151,6 +152,23 @@ def forward(q, k, v, scale: float | None = None, causal: bool = False, window_si
     _check(lib.sdpa_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, Hq,
                             Hkv, L, S, Dqk, Dv, sc, int(bool(causal)), int(window_size),
                             _dtype_code(q), _stream(stream)))
+    return out
+
+
+def forward_noalloc(q, k, v, scale: float | None = None, causal: bool = False,
+                    window_size: int = 0, out=None, stream=None):
+    """As ``forward``, through sdpa_forward_noalloc: no device allocation in
+    the library; split partials go to the library's fixed 16 MiB per-device
+    scratch array.  ``out`` should be preallocated by callers that cannot
+    allocate (when None, this wrapper allocates it with torch).  Calls that
+    overlap on the GPU share that array and race; keep them on one stream."""
+    lib = load_library()
+    B, Hq, Hkv, L, S, Dqk, Dv = _shapes(q, k, v)
+    sc = float(Dqk ** -0.5 if scale is None else scale)
+    out = _out_like(q, L, Dv, out)
+    _check(lib.sdpa_forward_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B,
+                                    Hq, Hkv, L, S, Dqk, Dv, sc, int(bool(causal)),
+                                    int(window_size), _dtype_code(q), _stream(stream)))
     return out
 
 
