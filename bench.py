@@ -170,31 +170,53 @@ class HostCase:
         self.kv_bytes = kv_bytes(p)
 
 
-def time_cases(sdpa, cases, steps, warmup, flush, sync_all):
+def time_cases(sdpa, cases, steps, warmup, flush, sync_all, graphs=True):
     """Per call: flush L2 (untimed), then time the call and its main kernel
-    with CUDA events on the current stream.  Returns per-case lists (ms)."""
+    with CUDA events on the current stream.  With ``graphs`` each call is
+    captured once into a CUDA graph (its split kernel, combine and the two
+    main-kernel events) and replayed, so the device timeline has no host
+    enqueue gaps.  Returns per-case lists (ms)."""
     call_ms = [[] for _ in cases]
     main_ms = [[] for _ in cases]
     stream = torch.cuda.current_stream()
+    hooks = []
+    for c in cases:
+        m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        m0.record(stream)  # creates the CUDA handles; the library re-records them
+        m1.record(stream)
+        c.call(sdpa)  # first call outside any capture (kernel attributes, TMA encode path)
+        hooks.append((m0, m1))
+    torch.cuda.synchronize()
+    runners = []
+    for c, (m0, m1) in zip(cases, hooks):
+        if graphs:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                sdpa.time_next_main_kernel(m0, m1)
+                c.call(sdpa)
+            runners.append(g.replay)
+        else:
+            def eager(c=c, m0=m0, m1=m1):
+                sdpa.time_next_main_kernel(m0, m1)
+                c.call(sdpa)
+            runners.append(eager)
+    torch.cuda.synchronize()
     for it in range(warmup + steps):
         evs = []
-        for c in cases:
+        for run in runners:
             flush_l2(flush)
-            e0, e1, m0, m1 = (torch.cuda.Event(enable_timing=True) for _ in range(4))
-            m0.record(stream)  # creates the CUDA handles; the library re-records them
-            m1.record(stream)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            sdpa.time_next_main_kernel(m0, m1)
-            c.call(sdpa)
+            run()
             e1.record(stream)
-            evs.append((e0, e1, m0, m1))
+            evs.append((e0, e1))
         if it == warmup - 1:
             sync_all()
         if it >= warmup:
             torch.cuda.synchronize()
-            for i, (e0, e1, m0, m1) in enumerate(evs):
+            for i, (e0, e1) in enumerate(evs):
                 call_ms[i].append(e0.elapsed_time(e1))
-                main_ms[i].append(m0.elapsed_time(m1))
+                main_ms[i].append(hooks[i][0].elapsed_time(hooks[i][1]))
     return call_ms, main_ms
 
 
@@ -250,10 +272,10 @@ def oracle_sample(cases, budget_s=12.0):
     return nbytes / dt / 1e9, dt, cores, calls
 
 
-def secondary(sdpa, probs, steps, warmup, flush, sync_all, device, peaks, kind):
+def secondary(sdpa, probs, steps, warmup, flush, sync_all, device, peaks, kind, graphs=True):
     """Time a list of problems (one call each per step); return a summary."""
     cases = [Case(sdpa, p, device) for p in probs]
-    call_ms, main_ms = time_cases(sdpa, cases, steps, warmup, flush, sync_all)
+    call_ms, main_ms = time_cases(sdpa, cases, steps, warmup, flush, sync_all, graphs)
     pts = []
     for c, cm, mm in zip(cases, call_ms, main_ms):
         us = 1e3 * statistics.median(cm)
@@ -283,6 +305,8 @@ def main():
                     help="restrict the timed sweep to the named problem (profiling)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing")
+    ap.add_argument("--eager", action="store_true",
+                    help="time eager calls instead of replaying one CUDA graph per call")
     args = ap.parse_args()
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
@@ -310,6 +334,7 @@ def main():
     workload = {"workload": "decode split-KV sweep: B=1, Hq=64, Hkv in {4,8}, L=1, "
                             "S in {256,1024,4096,8192,16384,32768}, Dqk=192, Dv=128, bf16, causal",
                 "calls_per_step": len(probs), "l2": "flushed before every call (2x L2 buffer written, then read)",
+                "launch": "eager" if args.eager else "one CUDA graph per call (split pass + combine), replayed",
                 "parallelism": f"replicas x{world} (independent KV-head units, no collective)"}
 
     if args.impl == "reference":
@@ -356,7 +381,8 @@ def main():
     sampler = ClockSampler(device.index if device.index is not None else 0)
     # warm-up steps run inside time_cases; the sampler covers the timed steps
     sampler.start()
-    call_ms, main_ms = time_cases(sdpa, cases, args.steps, args.warmup, flush, sync_all)
+    call_ms, main_ms = time_cases(sdpa, cases, args.steps, args.warmup, flush, sync_all,
+                                  graphs=not args.eager)
     sync_all()
     clocks = sampler.stop()
     sdpa.device_status(clear=False)
@@ -401,12 +427,13 @@ def main():
     extra = {}
     if not args.no_secondary:
         sec_steps = max(3, min(args.steps, 10))
+        gr = not args.eager
         extra["prefill"] = secondary(sdpa, I.window_problems() + I.encoder_problems(), sec_steps,
-                                     3, flush, sync_all, device, peaks, "tflops")
+                                     3, flush, sync_all, device, peaks, "tflops", gr)
         extra["verify"] = secondary(sdpa, I.verify_problems(), sec_steps, 3, flush, sync_all,
-                                    device, peaks, "tflops")
+                                    device, peaks, "tflops", gr)
         extra["tiny"] = secondary(sdpa, [I.tiny_problem()], sec_steps, 3, flush, sync_all,
-                                  device, peaks, "tflops")
+                                  device, peaks, "tflops", gr)
 
     line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s (KV, decode)",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
