@@ -45,6 +45,9 @@ def load_oracle(mutant: int = 0) -> ctypes.CDLL:
                   ctypes.c_double, ctypes.c_int, i64, i64, i64,
                   ctypes.POINTER(ctypes.c_int64), i64, ctypes.c_int]
     f.restype = ctypes.c_int
+    g = lib.oracle_sdpa2_f64
+    g.argtypes = f.argtypes + [ctypes.c_int, i64, dp]
+    g.restype = ctypes.c_int
     lib.oracle_mutant_id.restype = ctypes.c_int
     _LIBS[mutant] = lib
     return lib
@@ -63,14 +66,17 @@ def _as_f64(a) -> np.ndarray:
 
 def sdpa_oracle(q, k, v, scale: float, causal: bool = False, window: int = 0,
                 rows=None, key_range=None, nthreads: int | None = None,
-                return_lse: bool = False, mutant: int = 0):
+                return_lse: bool = False, mutant: int = 0, q_offset: int | None = None,
+                sinks=None):
     """Materialised fp64 attention.
 
     q [B,Hq,L,Dqk], k [B,Hkv,S,Dqk], v [B,Hkv,S,Dv] (numpy or torch, any float
     dtype; the values are taken exactly).  ``rows``: optional list of query
     indices; the output then has ``len(rows)`` rows per head.  ``key_range``:
     optional (lo, hi) restricting the keys, as one split of a split-KV pass
-    sees them.  Returns O [B,Hq,rows,Dv] float64 (and LSE [B,Hq,rows]).
+    sees them.  ``q_offset``: key position of query row 0 (default S - L).
+    ``sinks``: optional [Hq] sink logits (natural-log units).
+    Returns O [B,Hq,rows,Dv] float64 (and LSE [B,Hq,rows]).
     """
     qd, kd, vd = _as_f64(q), _as_f64(k), _as_f64(v)
     B, Hq, L, Dqk = qd.shape
@@ -90,13 +96,17 @@ def sdpa_oracle(q, k, v, scale: float, causal: bool = False, window: int = 0,
     lib = load_oracle(mutant)
     dp = ctypes.POINTER(ctypes.c_double)
     nt = nthreads if nthreads is not None else (os.cpu_count() or 1)
-    rc = lib.oracle_sdpa_f64(
+    sk = None if sinks is None else np.ascontiguousarray(_as_f64(sinks).reshape(-1))
+    if sk is not None and sk.size != Hq:
+        raise ValueError("oracle: sinks must have Hq entries")
+    rc = lib.oracle_sdpa2_f64(
         qd.ctypes.data_as(dp), kd.ctypes.data_as(dp), vd.ctypes.data_as(dp),
         out.ctypes.data_as(dp), lse.ctypes.data_as(dp),
         B, Hq, Hkv, L, S, Dqk, Dv, float(scale), int(bool(causal)), int(window),
         lo, hi,
         rows_arr.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)) if rows_arr is not None else None,
-        nrows, int(nt))
+        nrows, int(nt), int(q_offset is not None), int(q_offset or 0),
+        sk.ctypes.data_as(dp) if sk is not None else None)
     if rc != 0:
         raise ValueError(f"oracle_sdpa_f64 returned {rc}")
     return (out, lse) if return_lse else out

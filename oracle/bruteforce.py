@@ -17,8 +17,10 @@ from __future__ import annotations
 import math
 
 
-def sdpa_bruteforce(q, k, v, scale, causal=False, window=0):
-    """q, k, v: nested lists or arrays [B][H][N][D] of Python floats."""
+def sdpa_bruteforce(q, k, v, scale, causal=False, window=0, q_offset=None, sinks=None):
+    """q, k, v: nested lists or arrays [B][H][N][D] of Python floats.
+    ``q_offset``: key position of query 0 (default S - L).  ``sinks``: per
+    query head logit that joins the normalisation without a value row."""
     B = len(q)
     Hq = len(q[0])
     L = len(q[0][0])
@@ -33,14 +35,14 @@ def sdpa_bruteforce(q, k, v, scale, causal=False, window=0):
             hk = hq // g
             oh = []
             for i in range(L):
-                pos = S - L + i
+                pos = (S - L if q_offset is None else q_offset) + i
                 keys = [j for j in range(S)
                         if (not causal or j <= pos) and (window == 0 or j > pos - window)]
                 ws = []
                 for j in keys:
                     s = math.fsum(float(a) * float(c) for a, c in zip(q[b][hq][i], k[b][hk][j]))
                     ws.append(math.exp(scale * s))
-                den = math.fsum(ws)
+                den = math.fsum(ws + ([math.exp(float(sinks[hq]))] if sinks is not None else []))
                 row = [math.fsum(w * float(v[b][hk][j][d]) for w, j in zip(ws, keys)) / den
                        for d in range(Dv)]
                 oh.append(row)

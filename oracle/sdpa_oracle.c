@@ -34,6 +34,19 @@
  *   for) gets O = 0 and LSE = -inf: the weight such a partial result carries
  *   in a log-sum-exp merge is zero.
  *
+ *   Query offset: p = i + q_offset when the caller gives one, for a query
+ *   block that does not end at the last key (chunked prefill, or keys held
+ *   in a rotating window cache, addressed relative to the cache: mlx PR
+ *   #3552, "Implementation", K-relative coordinates).  Without one,
+ *   q_offset = S - L as above.
+ *
+ *   Sinks: when sinks is non-NULL, head hq has a sink logit sigma_hq that
+ *   joins the softmax normalisation as one more score without a value row
+ *   (the `sinks` argument of mlx PR #4185 "API" and mlx PR #3552 "Public
+ *   API"; the pages name it without defining it, this is the plain reading):
+ *     m'  = max(m, sigma),  l = sum_j exp(s_j - m') + exp(sigma - m'),
+ *     O   = sum_j exp(s_j - m') V_j / l,  LSE = m' + log(l).
+ *
  *   The key sub-range [key_lo, key_hi) exists so that a test can check one
  *   split of a split-KV pass (mlx issue #3826: split over S with a
  *   log-sum-exp merge) against the same definition restricted to its keys.
@@ -70,6 +83,8 @@ typedef struct {
   int64_t key_lo, key_hi;
   const int64_t *rows;
   int64_t nrows;
+  int64_t q_offset;
+  const double *sinks;
   int64_t total;      /* B * Hq * nrows work items */
   int64_t next;       /* next unclaimed work item */
   pthread_mutex_t mu;
@@ -109,7 +124,7 @@ static void oracle_row(const oracle_ctx *c, int64_t item, double *scores) {
   /* planted: causal alignment to the start of the keys instead of the end */
   const int64_t p = i;
 #else
-  const int64_t p = i + (c->S - c->L);
+  const int64_t p = i + c->q_offset;
 #endif
   const double *qi = c->q + ((b * c->Hq + hq) * c->L + i) * c->Dqk;
   const double *kh = c->k + (b * c->Hkv + hk) * c->S * c->Dqk;
@@ -133,12 +148,15 @@ static void oracle_row(const oracle_ctx *c, int64_t item, double *scores) {
   }
 
   for (int64_t d = 0; d < c->Dv; ++d) o[d] = 0.0;
+  const int has_sink = c->sinks != NULL;
+  const double sink = has_sink ? c->sinks[hq] : -INFINITY;
   if (!any) {
-    if (c->lse) c->lse[(b * c->Hq + hq) * c->nrows + r] = -INFINITY;
+    if (c->lse) c->lse[(b * c->Hq + hq) * c->nrows + r] = has_sink ? sink : -INFINITY;
     return;
   }
+  if (has_sink && sink > m) m = sink;
 
-  double l = 0.0;
+  double l = has_sink ? exp(sink - m) : 0.0;
   for (int64_t j = 0; j < c->S; ++j) {
     if (!key_visible(c, j, p)) continue;
     const double w = exp(scores[j] - m);
@@ -181,12 +199,13 @@ static void *oracle_worker(void *arg) {
  * Returns 0 on success, a negative number for invalid arguments, -100 if a
  * thread or buffer could not be created.  nthreads <= 0 means one thread.
  */
-int oracle_sdpa_f64(const double *q, const double *k, const double *v,
-                    double *out, double *lse,
-                    int64_t B, int64_t Hq, int64_t Hkv, int64_t L, int64_t S,
-                    int64_t Dqk, int64_t Dv, double scale, int causal,
-                    int64_t window, int64_t key_lo, int64_t key_hi,
-                    const int64_t *rows, int64_t nrows, int nthreads) {
+int oracle_sdpa2_f64(const double *q, const double *k, const double *v,
+                     double *out, double *lse,
+                     int64_t B, int64_t Hq, int64_t Hkv, int64_t L, int64_t S,
+                     int64_t Dqk, int64_t Dv, double scale, int causal,
+                     int64_t window, int64_t key_lo, int64_t key_hi,
+                     const int64_t *rows, int64_t nrows, int nthreads,
+                     int has_q_offset, int64_t q_offset, const double *sinks) {
   if (!q || !k || !v || !out) return -1;
   if (B < 1 || Hq < 1 || Hkv < 1 || L < 1 || S < 1 || Dqk < 1 || Dv < 1) return -2;
   if (Hq % Hkv != 0) return -3;
@@ -205,6 +224,8 @@ int oracle_sdpa_f64(const double *q, const double *k, const double *v,
   c.scale = scale; c.causal = causal; c.window = window;
   c.key_lo = key_lo; c.key_hi = key_hi;
   c.rows = rows; c.nrows = nrows;
+  c.q_offset = has_q_offset ? q_offset : S - L;
+  c.sinks = sinks;
   c.total = B * Hq * nrows;
   c.next = 0;
   pthread_mutex_init(&c.mu, NULL);
@@ -224,6 +245,16 @@ int oracle_sdpa_f64(const double *q, const double *k, const double *v,
   }
   pthread_mutex_destroy(&c.mu);
   return failed ? -100 : 0;
+}
+
+int oracle_sdpa_f64(const double *q, const double *k, const double *v,
+                    double *out, double *lse,
+                    int64_t B, int64_t Hq, int64_t Hkv, int64_t L, int64_t S,
+                    int64_t Dqk, int64_t Dv, double scale, int causal,
+                    int64_t window, int64_t key_lo, int64_t key_hi,
+                    const int64_t *rows, int64_t nrows, int nthreads) {
+  return oracle_sdpa2_f64(q, k, v, out, lse, B, Hq, Hkv, L, S, Dqk, Dv, scale, causal, window,
+                          key_lo, key_hi, rows, nrows, nthreads, 0, 0, NULL);
 }
 
 int oracle_mutant_id(void) { return ORACLE_MUTANT; }

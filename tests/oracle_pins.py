@@ -211,4 +211,88 @@ def pin_lse(mutant=0):
     return fails
 
 
-ALL_PINS = [pin_bruteforce, pin_closed_forms, pin_invariants, pin_torch_library, pin_lse]
+OFFSET_SINK_CASES = [
+    # B, Hq, Hkv, L, S, D, causal, W, q_offset, sinks
+    (1, 2, 1, 5, 9, 8, True, 0, 2, None),
+    (1, 2, 1, 4, 12, 8, True, 3, 6, None),
+    (1, 2, 2, 6, 6, 8, True, 0, None, [0.7, -1.5]),
+    (1, 4, 2, 3, 10, 8, True, 4, 5, [1.0, 2.0, -3.0, 0.0]),
+    (2, 2, 1, 7, 7, 12, False, 0, None, [0.3, 0.9]),
+    (1, 2, 1, 9, 4, 8, True, 0, 0, [0.2, 0.1]),  # more queries than keys, offset 0
+]
+
+
+def pin_offset_and_sinks(mutant=0):
+    """Query offset (chunked prefill, rotating cache) and sinks against the
+    brute force, the chunked-prefill and rotating-cache invariants, and a
+    library cross-check of sinks."""
+    fails = []
+    for n, (B, Hq, Hkv, L, S, D, causal, W, off, sk) in enumerate(OFFSET_SINK_CASES):
+        q, k, v = _qkv(B, Hq, Hkv, L, S, D, D, 500 + n)
+        sc = D ** -0.5
+        ref = np.asarray(sdpa_bruteforce(q.tolist(), k.tolist(), v.tolist(), sc, causal, W,
+                                         q_offset=off, sinks=sk))
+        got = sdpa_oracle(q, k, v, sc, causal, W, q_offset=off, sinks=sk, mutant=mutant)
+        if not np.max(np.abs(got - ref)) <= 1e-12:
+            fails.append(f"offset/sink brute force case {n}")
+    # q_offset = S - L is the default alignment
+    q, k, v = _qkv(1, 2, 1, 5, 11, 8, 8, 531)
+    for c, W in ((True, 0), (True, 4)):
+        a = sdpa_oracle(q, k, v, 0.4, c, W, mutant=mutant)
+        b = sdpa_oracle(q, k, v, 0.4, c, W, q_offset=6, mutant=mutant)
+        if not np.array_equal(a, b):
+            fails.append("q_offset = S - L differs from the default")
+    # chunked prefill: queries [c0, c1) over keys [0, c1) with offset c0 are
+    # rows [c0, c1) of the full causal (and windowed) prefill
+    N = 24
+    q, k, v = _qkv(1, 2, 1, N, N, 8, 8, 532)
+    for W in (0, 5):
+        full = sdpa_oracle(q, k, v, 0.4, True, W, mutant=mutant)
+        for c0, c1 in ((0, 8), (8, 16), (16, 24), (5, 13)):
+            part = sdpa_oracle(q[:, :, c0:c1], k[:, :, :c1], v[:, :, :c1], 0.4, True, W,
+                               q_offset=c0, mutant=mutant)
+            if not np.allclose(part, full[:, :, c0:c1], atol=1e-14):
+                fails.append(f"chunked prefill rows [{c0},{c1}) W={W}")
+    # rotating window cache: only the last W + chunk - 1 keys are held; with
+    # positions relative to the first held key the result is unchanged
+    W, c0, c1 = 6, 14, 20
+    first = c0 - W + 1
+    full = sdpa_oracle(q, k, v, 0.4, True, W, mutant=mutant)
+    part = sdpa_oracle(q[:, :, c0:c1], k[:, :, first:c1], v[:, :, first:c1], 0.4, True, W,
+                       q_offset=c0 - first, mutant=mutant)
+    if not np.allclose(part, full[:, :, c0:c1], atol=1e-14):
+        fails.append("rotating window cache")
+    # sinks: -inf is no sink; weights plus the sink's weight sum to 1
+    q, k, v = _qkv(1, 2, 1, 4, 9, 8, 8, 533)
+    if not np.array_equal(sdpa_oracle(q, k, v, 0.5, True, 0, sinks=[-np.inf, -np.inf], mutant=mutant),
+                          sdpa_oracle(q, k, v, 0.5, True, 0, mutant=mutant)):
+        fails.append("sink -inf differs from no sink")
+    eye = np.eye(9)[None, None]
+    wts, lse = sdpa_oracle(q, k, eye, 0.5, True, 0, sinks=[0.4, 1.7], return_lse=True,
+                           mutant=mutant)
+    w_sink = np.exp(np.array([0.4, 1.7])[None, :, None] - lse)
+    if not np.allclose(wts.sum(-1) + w_sink, 1.0, atol=1e-14):
+        fails.append("weights + sink weight != 1")
+    # library: the sink is one more key with a zero row whose score is set by
+    # an additive float mask; torch's fp64 SDPA then gives the same O
+    q, k, v = _qkv(1, 4, 2, 6, 10, 8, 8, 534)
+    sinks = np.array([0.3, -0.8, 1.2, 2.0])
+    g = 2
+    i = np.arange(6)[:, None] + 4
+    j = np.arange(10)[None, :]
+    bias = np.where(j <= i, 0.0, -np.inf)
+    kk = np.concatenate([np.repeat(k, g, 1), np.zeros((1, 4, 1, 8))], axis=2)
+    vv = np.concatenate([np.repeat(v, g, 1), np.zeros((1, 4, 1, 8))], axis=2)
+    mask = np.concatenate([np.broadcast_to(bias, (1, 4, 6, 10)),
+                           np.broadcast_to(sinks[None, :, None, None], (1, 4, 6, 1))], axis=3)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q), torch.from_numpy(kk), torch.from_numpy(vv),
+        attn_mask=torch.from_numpy(np.ascontiguousarray(mask)), scale=0.35).numpy()
+    got = sdpa_oracle(q, k, v, 0.35, True, 0, sinks=sinks, mutant=mutant)
+    if not np.max(np.abs(got - ref)) <= 1e-12:
+        fails.append("sinks vs torch extra-key construction")
+    return fails
+
+
+ALL_PINS = [pin_bruteforce, pin_closed_forms, pin_invariants, pin_torch_library, pin_lse,
+            pin_offset_and_sinks]
