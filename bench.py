@@ -171,33 +171,37 @@ class HostCase:
 
 
 def time_cases(sdpa, cases, steps, warmup, flush, sync_all, graphs=True):
-    """Per call: flush L2 (untimed), then time the call and its main kernel
-    with CUDA events on the current stream.  With ``graphs`` each call is
-    captured once into a CUDA graph (its split kernel, combine and the two
-    main-kernel events) and replayed, so the device timeline has no host
-    enqueue gaps.  Returns per-case lists (ms)."""
+    """Per call: flush L2 (untimed), then run the call with three CUDA events
+    recorded by the library on its launch stream: before the main kernel,
+    after it, and after the call's last launch (the combine, when split).
+    call time = first to last event (the device time of the library's work);
+    main time = the main kernel alone.  With ``graphs`` each call is captured
+    once into a CUDA graph and replayed, so the device timeline carries no
+    host enqueue gaps.  Returns per-case lists (ms): call, main, outer (the
+    replay including graph-launch edges)."""
     call_ms = [[] for _ in cases]
     main_ms = [[] for _ in cases]
+    outer_ms = [[] for _ in cases]
     stream = torch.cuda.current_stream()
     hooks = []
     for c in cases:
-        m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        m0.record(stream)  # creates the CUDA handles; the library re-records them
-        m1.record(stream)
+        evs = tuple(torch.cuda.Event(enable_timing=True) for _ in range(3))
+        for e in evs:
+            e.record(stream)  # creates the CUDA handles; the library re-records them
         c.call(sdpa)  # first call outside any capture (kernel attributes, TMA encode path)
-        hooks.append((m0, m1))
+        hooks.append(evs)
     torch.cuda.synchronize()
     runners = []
-    for c, (m0, m1) in zip(cases, hooks):
+    for c, (m0, m1, m2) in zip(cases, hooks):
         if graphs:
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g):
-                sdpa.time_next_main_kernel(m0, m1)
+                sdpa.time_next_call(m0, m1, m2)
                 c.call(sdpa)
             runners.append(g.replay)
         else:
-            def eager(c=c, m0=m0, m1=m1):
-                sdpa.time_next_main_kernel(m0, m1)
+            def eager(c=c, m0=m0, m1=m1, m2=m2):
+                sdpa.time_next_call(m0, m1, m2)
                 c.call(sdpa)
             runners.append(eager)
     torch.cuda.synchronize()
@@ -215,9 +219,11 @@ def time_cases(sdpa, cases, steps, warmup, flush, sync_all, graphs=True):
         if it >= warmup:
             torch.cuda.synchronize()
             for i, (e0, e1) in enumerate(evs):
-                call_ms[i].append(e0.elapsed_time(e1))
-                main_ms[i].append(hooks[i][0].elapsed_time(hooks[i][1]))
-    return call_ms, main_ms
+                m0, m1, m2 = hooks[i]
+                call_ms[i].append(m0.elapsed_time(m2))
+                main_ms[i].append(m0.elapsed_time(m1))
+                outer_ms[i].append(e0.elapsed_time(e1))
+    return call_ms, main_ms, outer_ms
 
 
 def time_e2e(sdpa, cases, steps, warmup, device):
@@ -275,7 +281,7 @@ def oracle_sample(cases, budget_s=12.0):
 def secondary(sdpa, probs, steps, warmup, flush, sync_all, device, peaks, kind, graphs=True):
     """Time a list of problems (one call each per step); return a summary."""
     cases = [Case(sdpa, p, device) for p in probs]
-    call_ms, main_ms = time_cases(sdpa, cases, steps, warmup, flush, sync_all, graphs)
+    call_ms, main_ms, _ = time_cases(sdpa, cases, steps, warmup, flush, sync_all, graphs)
     pts = []
     for c, cm, mm in zip(cases, call_ms, main_ms):
         us = 1e3 * statistics.median(cm)
@@ -381,8 +387,8 @@ def main():
     sampler = ClockSampler(device.index if device.index is not None else 0)
     # warm-up steps run inside time_cases; the sampler covers the timed steps
     sampler.start()
-    call_ms, main_ms = time_cases(sdpa, cases, args.steps, args.warmup, flush, sync_all,
-                                  graphs=not args.eager)
+    call_ms, main_ms, outer_ms = time_cases(sdpa, cases, args.steps, args.warmup, flush,
+                                            sync_all, graphs=not args.eager)
     sync_all()
     clocks = sampler.stop()
     sdpa.device_status(clear=False)
@@ -405,12 +411,13 @@ def main():
                 "launch": cases[big].p.name, "peak_source": peak_src,
                 "algorithmic_bytes_per_launch": cases[big].kv_bytes}
     points = []
-    for c, cm, mm in zip(cases, call_ms, main_ms):
+    for c, cm, mm, om in zip(cases, call_ms, main_ms, outer_ms):
         us = 1e3 * statistics.median(cm)
         points.append({"name": c.p.name, "us": round(us, 2),
                        "us_p10": round(1e3 * float(np.percentile(cm, 10)), 2),
                        "us_p90": round(1e3 * float(np.percentile(cm, 90)), 2),
                        "main_kernel_us": round(1e3 * statistics.median(mm), 2),
+                       "outer_us": round(1e3 * statistics.median(om), 2),
                        "kv_gbs": round(c.kv_bytes / (us * 1e-6) / 1e9, 1),
                        "frac_hbm": round(c.kv_bytes / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
                        "splits": c.info["splits"], "ctas": c.info["ctas"]})

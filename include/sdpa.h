@@ -86,8 +86,11 @@ typedef enum {
   SDPA_PATH_SPLITKV = 1, /* split-KV pass over packed (head-in-group, query)
                             rows on warp-level tensor-core tiles, then the
                             log-sum-exp combine when split                   */
-  SDPA_PATH_TC = 2       /* 128-row tiles on tcgen05 with TMEM accumulators,
+  SDPA_PATH_TC = 2,      /* 128-row tiles on tcgen05 with TMEM accumulators,
                             TMA-staged K/V, optional key splits + combine    */
+  SDPA_PATH_TC2 = 3      /* 256-row tiles on a pair of SMs (tcgen05
+                            cta_group::2): each SM loads half of every K/V
+                            block; head dims 256/256 and 192/128             */
 } sdpa_path;
 
 /*
@@ -172,16 +175,56 @@ SDPA_API sdpa_status sdpa_forward_noalloc(const void *q, const void *k, const vo
                                           float scale, int causal, int window_size,
                                           sdpa_dtype dtype, sdpa_stream_t stream);
 
+/*
+ * Options of sdpa_forward_ex (zero-initialise, then set what is needed).
+ *   has_q_offset / q_offset  key position of query row 0.  Without it the
+ *       queries end at the last key (q_offset = S - L).  With it a query block
+ *       can sit anywhere: chunked prefill (queries [c0, c1) over keys [0, c1)
+ *       with q_offset = c0), or keys held in a rotating window cache and
+ *       addressed relative to the first held key (mlx PR #3552,
+ *       "Implementation": K-relative coordinates).  Causal needs q_offset >= 0;
+ *       with a window the last row must still see a held key.
+ *   sinks  optional device array [Hq] of fp32 sink logits (natural-log units):
+ *       one more logit per query head that joins the softmax normalisation
+ *       with no value row (the `sinks` argument of mlx PR #4185 "API" and mlx
+ *       PR #3552 "Public API"):  O = sum_j e^{s_j} V_j / (e^{sink} + sum_j e^{s_j}).
+ *   lse    optional device array [B][Hq][L] of fp32, written with each row's
+ *       natural-log log-sum-exp (sink included), e.g. for a later merge of
+ *       results computed over disjoint key ranges.
+ *   force_path / force_splits  as in sdpa_plan (0 = the router's choice).
+ */
+typedef struct {
+  int has_q_offset;
+  int q_offset;
+  const float *sinks;
+  float *lse;
+  int force_path;
+  int force_splits;
+} sdpa_options;
+
+/*
+ * sdpa_forward_ex: sdpa_forward with sdpa_options (opt may be NULL).
+ * workspace: as sdpa_forward_ws; when workspace is NULL and workspace_bytes
+ * is 0 the call takes it stream-ordered from the pool like sdpa_forward.
+ * Extra errors: SDPA_ERR_INVALID_ARG for a misaligned sinks/lse pointer or a
+ * q_offset that leaves a row without keys.
+ */
+SDPA_API sdpa_status sdpa_forward_ex(const void *q, const void *k, const void *v, void *out,
+                                     int B, int Hq, int Hkv, int L, int S, int Dqk, int Dv,
+                                     float scale, int causal, int window_size, sdpa_dtype dtype,
+                                     const sdpa_options *opt, void *workspace,
+                                     size_t workspace_bytes, sdpa_stream_t stream);
+
 /* What the router decides for one problem.  Host-only, no CUDA call. */
 typedef struct {
   int path;          /* sdpa_path actually taken (never AUTO)               */
   int splits;        /* key splits per row tile (1 = no combine launch)     */
   int rows;          /* packed rows per (batch, KV head): (Hq/Hkv) * L      */
-  int row_tile;      /* rows one CTA owns                                   */
+  int row_tile;      /* rows one CTA (one CTA pair on SDPA_PATH_TC2) owns   */
   int row_tiles;     /* row tiles per (batch, KV head)                      */
   int key_block;     /* keys per pipeline stage                             */
   int keys_per_split;/* keys one split covers (a multiple of key_block)     */
-  int ctas;          /* CTAs of the main launch                             */
+  int ctas;          /* CTAs (CTA pairs on SDPA_PATH_TC2) of the main launch */
   int launches;      /* kernel launches one call makes (1 or 2)             */
   int dqk_pad;       /* head dims the kernel instance is built for          */
   int dv_pad;
@@ -244,6 +287,13 @@ SDPA_API sdpa_status sdpa_watchdog_selftest(uint64_t limit_ns, int *waited_out);
  * Both are cudaEvent_t handles owned by the caller; NULL, NULL disarms.
  */
 SDPA_API void sdpa_time_next_main_kernel(void *start_event, void *stop_event);
+
+/*
+ * As sdpa_time_next_main_kernel, plus `call_event` recorded after the last
+ * launch of the call (after the combine, when there is one).  NULL events
+ * are skipped.
+ */
+SDPA_API void sdpa_time_next_call(void *start_event, void *stop_event, void *call_event);
 
 SDPA_API const char *sdpa_status_string(sdpa_status status);
 /* Message of the last failed call on this thread ("" if none). */

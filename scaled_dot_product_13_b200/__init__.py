@@ -18,14 +18,14 @@ from __future__ import annotations
 import ctypes
 import os
 
-__all__ = ["forward", "forward_ws", "forward_noalloc", "workspace_bytes", "plan", "device_status",
-           "set_wait_limit_ns", "watchdog_selftest", "time_next_main_kernel", "load_library", "library_path",
-           "SdpaError", "PATH_AUTO", "PATH_SPLITKV", "PATH_TC", "STATUS"]
+__all__ = ["forward", "forward_ws", "forward_noalloc", "forward_ex", "Options", "workspace_bytes", "plan", "device_status",
+           "set_wait_limit_ns", "watchdog_selftest", "time_next_main_kernel", "time_next_call", "load_library", "library_path",
+           "SdpaError", "PATH_AUTO", "PATH_SPLITKV", "PATH_TC", "PATH_TC2", "STATUS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB: ctypes.CDLL | None = None
 
-PATH_AUTO, PATH_SPLITKV, PATH_TC = 0, 1, 2
+PATH_AUTO, PATH_SPLITKV, PATH_TC, PATH_TC2 = 0, 1, 2, 3
 STATUS = {0: "SDPA_OK", 1: "SDPA_ERR_INVALID_ARG", 2: "SDPA_ERR_UNSUPPORTED",
           3: "SDPA_ERR_RESOURCES", 4: "SDPA_ERR_CUDA", 5: "SDPA_ERR_TIMEOUT"}
 
@@ -35,6 +35,13 @@ class SdpaError(RuntimeError):
         super().__init__(f"{STATUS.get(status, status)}: {message}")
         self.status = status
         self.message = message
+
+
+class Options(ctypes.Structure):
+    """Mirror of sdpa_options."""
+    _fields_ = [("has_q_offset", ctypes.c_int), ("q_offset", ctypes.c_int),
+                ("sinks", ctypes.c_void_p), ("lse", ctypes.c_void_p),
+                ("force_path", ctypes.c_int), ("force_splits", ctypes.c_int)]
 
 
 class PlanInfo(ctypes.Structure):
@@ -67,6 +74,7 @@ def load_library() -> ctypes.CDLL:
     lib.sdpa_forward.argtypes = common + [vp]
     lib.sdpa_forward_ws.argtypes = common + [vp, sz, vp]
     lib.sdpa_forward_noalloc.argtypes = common + [vp]
+    lib.sdpa_forward_ex.argtypes = common + [ctypes.POINTER(Options), vp, sz, vp]
     lib.sdpa_forward_planned.argtypes = common + [i, i, vp, sz, vp]
     lib.sdpa_workspace_bytes.argtypes = [i] * 10
     lib.sdpa_workspace_bytes.restype = sz
@@ -77,10 +85,13 @@ def load_library() -> ctypes.CDLL:
     lib.sdpa_watchdog_selftest.argtypes = [ctypes.c_uint64, ctypes.POINTER(ctypes.c_int)]
     lib.sdpa_time_next_main_kernel.argtypes = [vp, vp]
     lib.sdpa_time_next_main_kernel.restype = None
+    lib.sdpa_time_next_call.argtypes = [vp, vp, vp]
+    lib.sdpa_time_next_call.restype = None
     lib.sdpa_status_string.restype = ctypes.c_char_p
     lib.sdpa_status_string.argtypes = [i]
     lib.sdpa_last_error_message.restype = ctypes.c_char_p
-    for fn in ("sdpa_forward", "sdpa_forward_ws", "sdpa_forward_noalloc", "sdpa_forward_planned", "sdpa_plan",
+    for fn in ("sdpa_forward", "sdpa_forward_ws", "sdpa_forward_noalloc", "sdpa_forward_ex",
+               "sdpa_forward_planned", "sdpa_plan",
                "sdpa_device_status", "sdpa_watchdog_selftest"):
         getattr(lib, fn).restype = ctypes.c_int
     _LIB = lib
@@ -172,6 +183,40 @@ def forward_noalloc(q, k, v, scale: float | None = None, causal: bool = False,
     return out
 
 
+def forward_ex(q, k, v, scale: float | None = None, causal: bool = False, window_size: int = 0,
+               q_offset: int | None = None, sinks=None, lse=None, out=None, stream=None,
+               workspace=None, force_path: int = 0, force_splits: int = 0):
+    """sdpa_forward_ex: ``q_offset`` = key position of query row 0 (default
+    S - L); ``sinks`` = optional float32 CUDA tensor [Hq] of sink logits;
+    ``lse`` = optional float32 CUDA tensor [B, Hq, L] that receives each row's
+    log-sum-exp.  ``workspace``: as ``forward_ws`` (None = pool allocation)."""
+    import torch
+
+    lib = load_library()
+    B, Hq, Hkv, L, S, Dqk, Dv = _shapes(q, k, v)
+    sc = float(Dqk ** -0.5 if scale is None else scale)
+    out = _out_like(q, L, Dv, out)
+    opt = Options()
+    if q_offset is not None:
+        opt.has_q_offset, opt.q_offset = 1, int(q_offset)
+    for name, t, shape in (("sinks", sinks, (Hq,)), ("lse", lse, (B, Hq, L))):
+        if t is None:
+            continue
+        if not (t.is_cuda and t.dtype == torch.float32 and t.is_contiguous()
+                and tuple(t.shape) == shape):
+            raise SdpaError(1, f"{name} must be a contiguous float32 CUDA tensor of shape {shape}")
+    opt.sinks = sinks.data_ptr() if sinks is not None else None
+    opt.lse = lse.data_ptr() if lse is not None else None
+    opt.force_path, opt.force_splits = int(force_path), int(force_splits)
+    ws_ptr = 0 if workspace is None else workspace.data_ptr()
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.sdpa_forward_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, Hq,
+                               Hkv, L, S, Dqk, Dv, sc, int(bool(causal)), int(window_size),
+                               _dtype_code(q), ctypes.byref(opt), ws_ptr, ws_bytes,
+                               _stream(stream)))
+    return out
+
+
 def forward_ws(q, k, v, workspace, scale: float | None = None, causal: bool = False,
                window_size: int = 0, out=None, stream=None, force_path: int = 0,
                force_splits: int = 0):
@@ -236,6 +281,17 @@ def time_next_main_kernel(start_event, stop_event) -> None:
         raise SdpaError(1, "events have no CUDA handle yet; record them once first")
     load_library().sdpa_time_next_main_kernel(ctypes.c_void_p(start_event.cuda_event),
                                               ctypes.c_void_p(stop_event.cuda_event))
+
+
+def time_next_call(start_event, stop_event, call_event) -> None:
+    """As ``time_next_main_kernel``, plus ``call_event`` recorded after the
+    call's last launch (the combine, when the keys are split)."""
+    for e in (start_event, stop_event, call_event):
+        if not e.cuda_event:
+            raise SdpaError(1, "events have no CUDA handle yet; record them once first")
+    load_library().sdpa_time_next_call(ctypes.c_void_p(start_event.cuda_event),
+                                       ctypes.c_void_p(stop_event.cuda_event),
+                                       ctypes.c_void_p(call_event.cuda_event))
 
 
 def set_wait_limit_ns(ns: int) -> None:

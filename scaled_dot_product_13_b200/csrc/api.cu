@@ -30,7 +30,7 @@ namespace sdpa {
 namespace {
 
 thread_local std::string t_last_error;
-thread_local cudaEvent_t t_ev_start = nullptr, t_ev_stop = nullptr;
+thread_local cudaEvent_t t_ev_start = nullptr, t_ev_stop = nullptr, t_ev_call = nullptr;
 std::atomic<uint64_t> g_wait_limit_ns{0};
 constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;  // 2 s
 
@@ -76,11 +76,19 @@ sdpa_status validate_shape(const Problem &p) {
                 (int)p.dtype);
   if (p.causal != 0 && p.causal != 1)
     return fail(SDPA_ERR_INVALID_ARG, "causal must be 0 or 1 (got %d)", p.causal);
-  if (p.causal && p.L > p.S)
+  if (p.causal && !p.has_q_offset && p.L > p.S)
     return fail(SDPA_ERR_INVALID_ARG,
                 "causal attention needs L <= S (got L=%d > S=%d): queries are aligned to the "
                 "end of the keys, so the first rows would see no key",
                 p.L, p.S);
+  if (p.has_q_offset) {
+    if (p.q_offset < -(1 << 30) || p.q_offset > (1 << 30))
+      return fail(SDPA_ERR_UNSUPPORTED, "q_offset must lie in [-2^30, 2^30] (got %d)", p.q_offset);
+    if (p.causal && p.q_offset < 0)
+      return fail(SDPA_ERR_INVALID_ARG,
+                  "causal attention needs q_offset >= 0 (got %d): query row 0 would see no key",
+                  p.q_offset);
+  }
   if (p.window < 0)
     return fail(SDPA_ERR_INVALID_ARG, "window_size must be >= 0 (got %d)", p.window);
   if (p.window > 0 && !p.causal)
@@ -88,6 +96,11 @@ sdpa_status validate_shape(const Problem &p) {
                 "window_size > 0 is defined only together with causal masking (got causal=0, "
                 "window_size=%d)",
                 p.window);
+  if (p.window > 0 && (long long)p.q_offset + p.L - 1 - (p.window - 1) > (long long)p.S - 1)
+    return fail(SDPA_ERR_INVALID_ARG,
+                "window_size=%d with q_offset=%d: the last query row (position %d) sees no key "
+                "of the %d held",
+                p.window, p.q_offset, p.q_offset + p.L - 1, p.S);
   if (!std::isfinite(p.scale))
     return fail(SDPA_ERR_INVALID_ARG, "scale must be finite");
   for (int d : {p.Dqk, p.Dv}) {
@@ -134,8 +147,17 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 // shared memory).
 constexpr int kMaxSplits = 4096;
 
-// Packed rows per (batch, KV head) from which the tcgen05 path is taken.
-constexpr int kTcRowThreshold = 128;
+// Packed rows per (batch, KV head) from which the tcgen05 path is taken:
+// above four 16-row warp tiles, one 128-row tensor-memory tile costs less.
+constexpr int kTcRowThreshold = 65;
+// ... and from which head dims 256/256 and 192/128 take the two-CTA kernel.
+constexpr int kTc2RowThreshold = 256;
+
+// A split must cover at least this many key blocks, and problems of at most
+// kNoSplitBlocks key blocks are not split: below that the combine launch
+// costs more than the parallelism gains.
+constexpr int kMinBlocksPerSplit = 2;
+constexpr int kNoSplitBlocks = 4;
 
 sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_splits,
                       Plan *out) {
@@ -145,7 +167,7 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
   if (pl.pair < 0)
     return fail(SDPA_ERR_UNSUPPORTED, "no kernel instance covers Dqk=%d, Dv=%d", pb.Dqk, pb.Dv);
   if (force_path != SDPA_PATH_AUTO && force_path != SDPA_PATH_SPLITKV &&
-      force_path != SDPA_PATH_TC)
+      force_path != SDPA_PATH_TC && force_path != SDPA_PATH_TC2)
     return fail(SDPA_ERR_INVALID_ARG, "unknown path %d", force_path);
   if (force_splits < 0) return fail(SDPA_ERR_INVALID_ARG, "force_splits must be >= 0");
   if (num_sms < 1) num_sms = 148;
@@ -157,9 +179,22 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
   // split-KV kernel on 16-row warp tiles.  Both split the keys when the
   // tiles alone do not fill the GPU.
   int path = force_path;
-  if (path == SDPA_PATH_AUTO) path = pl.rows >= kTcRowThreshold ? SDPA_PATH_TC : SDPA_PATH_SPLITKV;
+  if (path == SDPA_PATH_AUTO) {
+    path = pl.rows >= kTcRowThreshold ? SDPA_PATH_TC : SDPA_PATH_SPLITKV;
+    // wide heads with at least one full 256-row pair tile: two SMs per tile
+    if (path == SDPA_PATH_TC && tc2_supports_pair(pl.pair) && pl.rows >= kTc2RowThreshold)
+      path = SDPA_PATH_TC2;
+  }
+  if (path == SDPA_PATH_TC2 && !tc2_supports_pair(pl.pair))
+    return fail(SDPA_ERR_UNSUPPORTED,
+                "the two-CTA path is built for head dims 256/256 and 192/128 (got %d/%d)",
+                pb.Dqk, pb.Dv);
   pl.path = path;
-  if (path == SDPA_PATH_TC) {
+  if (path == SDPA_PATH_TC2) {
+    pl.wr = 0; pl.wk = 0;
+    pl.row_tile = 2 * kTcRows;
+    pl.key_block = 128;
+  } else if (path == SDPA_PATH_TC) {
     pl.wr = 0; pl.wk = 0;
     pl.row_tile = kTcRows;
     pl.key_block = tc_key_block(kDimPairs[pl.pair].dqk, kDimPairs[pl.pair].dv);
@@ -175,28 +210,31 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
     pl.key_block = kSplitKvBN;
   }
   pl.row_tiles = (pl.rows + pl.row_tile - 1) / pl.row_tile;
-  // keys visible to at least one row: [kbeg, S); the last row sits at S-1
-  const int off = pb.S - pb.L;
+  // keys visible to at least one row: [kbeg, kend)
+  const int off = pb.q_offset;
   const int kbeg = pb.window > 0 ? std::max(0, off - pb.window + 1) : 0;
+  const int kend = pb.causal ? (int)std::min<long long>(pb.S, (long long)off + pb.L) : pb.S;
   const int bn = pl.key_block;
   pl.split_base = (kbeg / bn) * bn;
-  const int nkb = (pb.S + bn - 1) / bn - kbeg / bn;
-  const long long base = (long long)pb.B * pb.Hkv * pl.row_tiles;
+  const int nkb = std::max(1, (kend + bn - 1) / bn - kbeg / bn);
+  // CTAs per split: one per row tile, two per pair tile
+  const long long per_tile = pl.path == SDPA_PATH_TC2 ? 2 : 1;
+  const long long base = (long long)pb.B * pb.Hkv * pl.row_tiles * per_tile;
   int splits;
   if (force_splits > 0) {
     splits = std::min(force_splits, nkb);
-  } else if (base >= num_sms) {
+  } else if (base >= num_sms || nkb <= kNoSplitBlocks) {
     splits = 1;
   } else {
     splits = (int)std::max(1LL, num_sms / base);
-    splits = std::min(splits, nkb);
+    splits = std::min(splits, std::max(1, nkb / kMinBlocksPerSplit));
   }
   splits = std::min(splits, kMaxSplits);
   const int bps = (nkb + splits - 1) / splits;
   if (force_splits == 0) splits = (nkb + bps - 1) / bps;
   pl.splits = splits;
   pl.keys_per_split = bps * bn;
-  pl.ctas = base * splits;
+  pl.ctas = (base / per_tile) * splits;
   if (pl.ctas > 0x7fffffffLL)
     return fail(SDPA_ERR_UNSUPPORTED, "problem needs %lld CTAs, above the grid limit", pl.ctas);
   pl.launches = splits > 1 ? 2 : 1;
@@ -283,7 +321,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // ---------------------------------------------------------------------------
 sdpa_status forward_call(const Problem &pb, const void *q, const void *k, const void *v,
                          void *out, int force_path, int force_splits, void *ws, size_t ws_bytes,
-                         bool own_ws, cudaStream_t stream) {
+                         bool own_ws, cudaStream_t stream, const float *sinks, float *lse_out) {
   sdpa_status st = validate_shape(pb);
   if (st != SDPA_OK) return st;
   st = validate_pointers(pb, q, k, v, out);
@@ -317,7 +355,8 @@ sdpa_status forward_call(const Problem &pb, const void *q, const void *k, const 
   ln.q = q; ln.k = k; ln.v = v; ln.out = out;
   ln.part_o = static_cast<float *>(ws);
   ln.part_lse = ws ? reinterpret_cast<float *>(static_cast<char *>(ws) + pl.ws_o_bytes) : nullptr;
-  ln.lse_out = nullptr;
+  ln.lse_out = lse_out;
+  ln.sinks = sinks;
   ln.wd_word = wd;
   ln.wd_limit_ns = wait_limit();
   ln.stream = stream;
@@ -325,9 +364,13 @@ sdpa_status forward_call(const Problem &pb, const void *q, const void *k, const 
   std::string err;
   ln.ev_start = t_ev_start;
   ln.ev_stop = t_ev_stop;
-  t_ev_start = t_ev_stop = nullptr;
-  st = pl.path == SDPA_PATH_TC ? launch_tc(ln, &err) : launch_splitkv(ln, &err);
+  cudaEvent_t ev_call = t_ev_call;
+  t_ev_start = t_ev_stop = t_ev_call = nullptr;
+  st = pl.path == SDPA_PATH_TC2  ? launch_tc2(ln, &err)
+       : pl.path == SDPA_PATH_TC ? launch_tc(ln, &err)
+                                 : launch_splitkv(ln, &err);
   if (st == SDPA_OK && pl.splits > 1) st = launch_combine(ln, &err);
+  if (st == SDPA_OK && ev_call) record_event(ev_call, stream);
   if (allocated) {
     cudaError_t e = cudaFreeAsync(ws, stream);
     if (st == SDPA_OK && e != cudaSuccess) {
@@ -458,6 +501,8 @@ static Problem make_problem(int B, int Hq, int Hkv, int L, int S, int Dqk, int D
   Problem p;
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = L; p.S = S; p.Dqk = Dqk; p.Dv = Dv;
   p.scale = scale; p.causal = causal; p.window = window; p.dtype = dtype;
+  p.q_offset = S - L;
+  p.has_q_offset = 0;
   return p;
 }
 
@@ -519,6 +564,33 @@ sdpa_status sdpa_forward_planned(const void *q, const void *k, const void *v, vo
              (cudaStream_t)stream);
 }
 
+sdpa_status sdpa_forward_ex(const void *q, const void *k, const void *v, void *out, int B, int Hq,
+                            int Hkv, int L, int S, int Dqk, int Dv, float scale, int causal,
+                            int window_size, sdpa_dtype dtype, const sdpa_options *opt,
+                            void *workspace, size_t workspace_bytes, sdpa_stream_t stream) {
+  t_last_error.clear();
+  Problem pb = make_problem(B, Hq, Hkv, L, S, Dqk, Dv, scale, causal, window_size, dtype);
+  int force_path = 0, force_splits = 0;
+  const float *sinks = nullptr;
+  float *lse = nullptr;
+  if (opt != nullptr) {
+    if (opt->has_q_offset) {
+      pb.has_q_offset = 1;
+      pb.q_offset = opt->q_offset;
+    }
+    sinks = opt->sinks;
+    lse = opt->lse;
+    force_path = opt->force_path;
+    force_splits = opt->force_splits;
+    if ((sinks && (reinterpret_cast<uintptr_t>(sinks) & 3u)) ||
+        (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+      return fail(SDPA_ERR_INVALID_ARG, "sinks and lse must be 4-byte aligned");
+  }
+  const bool own = workspace == nullptr && workspace_bytes == 0;
+  return forward_call(pb, q, k, v, out, force_path, force_splits, workspace, workspace_bytes,
+                      own, (cudaStream_t)stream, sinks, lse);
+}
+
 sdpa_status sdpa_device_status(int clear) {
   t_last_error.clear();
   int dev, sms;
@@ -544,8 +616,13 @@ sdpa_status sdpa_device_status(int clear) {
 void sdpa_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns); }
 
 void sdpa_time_next_main_kernel(void *start_event, void *stop_event) {
+  sdpa_time_next_call(start_event, stop_event, nullptr);
+}
+
+void sdpa_time_next_call(void *start_event, void *stop_event, void *call_event) {
   t_ev_start = static_cast<cudaEvent_t>(start_event);
   t_ev_stop = static_cast<cudaEvent_t>(stop_event);
+  t_ev_call = static_cast<cudaEvent_t>(call_event);
 }
 
 sdpa_status sdpa_watchdog_selftest(uint64_t limit_ns, int *waited_out) {

@@ -37,6 +37,8 @@ struct Problem {
   float scale;
   int causal, window;
   sdpa_dtype dtype;
+  int q_offset;      // key position of query row 0 (S - L unless given)
+  int has_q_offset;  // 1 when the caller gave q_offset explicitly
 };
 
 struct Plan {
@@ -63,6 +65,7 @@ struct Launch {
   void *out;
   float *part_o, *part_lse;
   float *lse_out;          // optional final LSE [B*Hq*L] (nullptr = not wanted)
+  const float *sinks;      // optional [Hq] sink logits
   unsigned int *wd_word;
   uint64_t wd_limit_ns;
   cudaStream_t stream;
@@ -74,7 +77,8 @@ struct Launch {
 // the stream-ordered pool; otherwise use (ws, ws_bytes).
 sdpa_status forward_call(const Problem &pb, const void *q, const void *k, const void *v,
                          void *out, int force_path, int force_splits, void *ws, size_t ws_bytes,
-                         bool own_ws, cudaStream_t stream);
+                         bool own_ws, cudaStream_t stream, const float *sinks = nullptr,
+                         float *lse_out = nullptr);
 
 // Validate and plan for the current device without enqueuing anything.
 sdpa_status plan_call(const Problem &pb, int force_path, int force_splits, Plan *plan);
@@ -91,7 +95,22 @@ bool encode_tma(CUtensorMap *map, sdpa_dtype dt, int rank, const void *base,
 // Per-path launchers (return SDPA_OK or an error with *err set).
 sdpa_status launch_splitkv(const Launch &ln, std::string *err);
 sdpa_status launch_tc(const Launch &ln, std::string *err);
+sdpa_status launch_tc2(const Launch &ln, std::string *err);
+
+// Head-dim pairs the two-CTA kernel is built for (index into kDimPairs).
+constexpr bool tc2_supports_pair(int pair) { return pair == 3 || pair == 5; }
 sdpa_status launch_combine(const Launch &ln, std::string *err);
+
+// Record a timing event on `stream`.  Inside stream capture a plain
+// cudaEventRecord only orders work within the graph; an external record node
+// is needed for the event to carry a timestamp when the graph is replayed.
+inline void record_event(cudaEvent_t ev, cudaStream_t stream) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(ev, stream, cudaEventRecordExternal);
+  else
+    cudaEventRecord(ev, stream);
+}
 
 // Checks that a kernel fits the device (threads, shared memory) before its
 // first launch, and raises its dynamic shared-memory limit.  Cached per

@@ -48,7 +48,7 @@ sdpa_status run_splitkv(const Launch &ln, std::string *err) {
   AttnParams p;
   p.B = pb.B; p.Hq = pb.Hq; p.Hkv = pb.Hkv; p.L = pb.L; p.S = pb.S; p.Dqk = pb.Dqk; p.Dv = pb.Dv;
   p.R = pl.rows;
-  p.off = pb.S - pb.L;
+  p.off = pb.q_offset;
   p.causal = pb.causal;
   p.window = pb.window;
   p.scale_log2 = pb.scale * 1.4426950408889634f;
@@ -59,11 +59,13 @@ sdpa_status run_splitkv(const Launch &ln, std::string *err) {
   p.out = ln.out;
   p.part_o = ln.part_o;
   p.part_lse = ln.part_lse;
+  p.sinks = ln.sinks;
+  p.lse_out = ln.lse_out;
   p.wd.word = ln.wd_word;
   p.wd.limit_ns = ln.wd_limit_ns;
-  if (ln.ev_start) cudaEventRecord(ln.ev_start, ln.stream);
+  if (ln.ev_start) record_event(ln.ev_start, ln.stream);
   kern<<<(unsigned)pl.ctas, Cfg::kThreads, Cfg::kSmemBytes, ln.stream>>>(tq, tk, tv, p);
-  if (ln.ev_stop) cudaEventRecord(ln.ev_stop, ln.stream);
+  if (ln.ev_stop) record_event(ln.ev_stop, ln.stream);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     *err = std::string("splitkv_kernel launch failed: ") + cudaGetErrorString(e);
@@ -120,12 +122,12 @@ sdpa_status launch_combine(const Launch &ln, std::string *err) {
   cudaError_t e;
   if (ln.pb.dtype == SDPA_BF16)
     e = cudaLaunchKernelEx(&cfg, combine_kernel<true>, (const float *)ln.part_o,
-                           (const float *)ln.part_lse, ln.out, ln.lse_out, total, ln.pb.Dv,
-                           ln.plan.splits);
+                           (const float *)ln.part_lse, ln.out, ln.lse_out, ln.sinks, total,
+                           ln.pb.Dv, ln.plan.splits, ln.pb.L, ln.pb.Hq);
   else
     e = cudaLaunchKernelEx(&cfg, combine_kernel<false>, (const float *)ln.part_o,
-                           (const float *)ln.part_lse, ln.out, ln.lse_out, total, ln.pb.Dv,
-                           ln.plan.splits);
+                           (const float *)ln.part_lse, ln.out, ln.lse_out, ln.sinks, total,
+                           ln.pb.Dv, ln.plan.splits, ln.pb.L, ln.pb.Hq);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) {
     *err = std::string("combine_kernel launch failed: ") + cudaGetErrorString(e);

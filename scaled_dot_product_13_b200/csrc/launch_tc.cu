@@ -13,9 +13,9 @@ sdpa_status run_tc(const Launch &ln, std::string *err) {
   constexpr uint32_t kK = ((DQK + 63) / 64) * kBN * 128;
   constexpr uint32_t kV = ((DV + 63) / 64) * kBN * 128;
   constexpr uint32_t kSlot = kK > kV ? kK : kV;
-  constexpr uint32_t kP = 2 * 128 * kBN * 2;
-  constexpr uint32_t kBudget = 232448u - 2048u;
-  constexpr int kFit = (int)((kBudget - kQ - kP) / kSlot);
+  // everything but Q and the slots: row-max exchange (2 KB) and the barriers
+  constexpr uint32_t kBudget = 232448u - 4u * 128u * 4u - 40u * 8u - 16u;
+  constexpr int kFit = (int)((kBudget - kQ) / kSlot);
   constexpr int kNSlot = kFit > 8 ? 8 : kFit;
   static_assert(kNSlot >= 2, "at least two K/V slots");
   using Cfg = TcCfg<DQK, DV, kBN, kNSlot>;
@@ -48,7 +48,7 @@ sdpa_status run_tc(const Launch &ln, std::string *err) {
   AttnParams p;
   p.B = pb.B; p.Hq = pb.Hq; p.Hkv = pb.Hkv; p.L = pb.L; p.S = pb.S; p.Dqk = pb.Dqk; p.Dv = pb.Dv;
   p.R = pl.rows;
-  p.off = pb.S - pb.L;
+  p.off = pb.q_offset;
   p.causal = pb.causal;
   p.window = pb.window;
   p.scale_log2 = pb.scale * 1.4426950408889634f;
@@ -59,11 +59,13 @@ sdpa_status run_tc(const Launch &ln, std::string *err) {
   p.out = ln.out;
   p.part_o = ln.part_o;
   p.part_lse = ln.part_lse;
+  p.sinks = ln.sinks;
+  p.lse_out = ln.lse_out;
   p.wd.word = ln.wd_word;
   p.wd.limit_ns = ln.wd_limit_ns;
-  if (ln.ev_start) cudaEventRecord(ln.ev_start, ln.stream);
+  if (ln.ev_start) record_event(ln.ev_start, ln.stream);
   kern<<<(unsigned)pl.ctas, Cfg::kThreads, Cfg::kSmemBytes, ln.stream>>>(tq, tk, tv, p);
-  if (ln.ev_stop) cudaEventRecord(ln.ev_stop, ln.stream);
+  if (ln.ev_stop) record_event(ln.ev_stop, ln.stream);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     *err = std::string("tc_attn_kernel launch failed: ") + cudaGetErrorString(e);

@@ -1,0 +1,105 @@
+// Launch unit of the two-CTA (cta_group::2) attention kernel.
+#include "launch.h"
+#include "tc2.cuh"
+
+namespace sdpa {
+
+namespace {
+
+template <bool kBF16, int DQK, int DV>
+sdpa_status run_tc2(const Launch &ln, std::string *err) {
+  constexpr int kBN = 128;
+  constexpr uint32_t kQ = (DQK / 64) * 128 * 128;
+  constexpr uint32_t kK = (DQK / 64) * (kBN / 2) * 128;
+  constexpr uint32_t kV = (DV / 128) * kBN * 128;
+  constexpr uint32_t kSlot = kK > kV ? kK : kV;
+  constexpr uint32_t kBudget = 232448u - 4u * 128u * 4u - 48u * 8u - 16u;
+  constexpr int kFit = (int)((kBudget - kQ) / kSlot);
+  constexpr int kNSlot = kFit > 8 ? 8 : kFit;
+  static_assert(kNSlot >= 2, "at least two K/V slots");
+  using Cfg = Tc2Cfg<DQK, DV, kBN, kNSlot>;
+  auto kern = tc2_attn_kernel<kBF16, DQK, DV, kBN, kNSlot>;
+  sdpa_status st =
+      prepare_kernel((const void *)kern, Cfg::kThreads, Cfg::kSmemBytes, "tc2_attn_kernel", err);
+  if (st != SDPA_OK) return st;
+
+  const Problem &pb = ln.pb;
+  const Plan &pl = ln.plan;
+  CUtensorMap tq, tk, tv;
+  {
+    const uint64_t dims[2] = {(uint64_t)pb.Dqk, (uint64_t)pb.B * pb.Hq * pb.L};
+    const uint64_t strides[1] = {(uint64_t)pb.Dqk * 2};
+    const uint32_t box[2] = {64, 128};
+    if (!encode_tma(&tq, pb.dtype, 2, ln.q, dims, strides, box, err)) return SDPA_ERR_CUDA;
+  }
+  {  // each CTA loads half of a key block: BN/2 keys
+    const uint64_t dims[3] = {(uint64_t)pb.Dqk, (uint64_t)pb.S, (uint64_t)pb.B * pb.Hkv};
+    const uint64_t strides[2] = {(uint64_t)pb.Dqk * 2, (uint64_t)pb.S * pb.Dqk * 2};
+    const uint32_t box[3] = {64, (uint32_t)(kBN / 2), 1};
+    if (!encode_tma(&tk, pb.dtype, 3, ln.k, dims, strides, box, err)) return SDPA_ERR_CUDA;
+  }
+  {  // and half of a value block's columns, all BN keys
+    const uint64_t dims[3] = {(uint64_t)pb.Dv, (uint64_t)pb.S, (uint64_t)pb.B * pb.Hkv};
+    const uint64_t strides[2] = {(uint64_t)pb.Dv * 2, (uint64_t)pb.S * pb.Dv * 2};
+    const uint32_t box[3] = {64, (uint32_t)kBN, 1};
+    if (!encode_tma(&tv, pb.dtype, 3, ln.v, dims, strides, box, err)) return SDPA_ERR_CUDA;
+  }
+  AttnParams p;
+  p.B = pb.B; p.Hq = pb.Hq; p.Hkv = pb.Hkv; p.L = pb.L; p.S = pb.S; p.Dqk = pb.Dqk; p.Dv = pb.Dv;
+  p.R = pl.rows;
+  p.off = pb.q_offset;
+  p.causal = pb.causal;
+  p.window = pb.window;
+  p.scale_log2 = pb.scale * 1.4426950408889634f;
+  p.row_tiles = pl.row_tiles;
+  p.splits = pl.splits;
+  p.split_base = pl.split_base;
+  p.keys_per_split = pl.keys_per_split;
+  p.out = ln.out;
+  p.part_o = ln.part_o;
+  p.part_lse = ln.part_lse;
+  p.sinks = ln.sinks;
+  p.lse_out = ln.lse_out;
+  p.wd.word = ln.wd_word;
+  p.wd.limit_ns = ln.wd_limit_ns;
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * pl.ctas));
+  cfg.blockDim = dim3(Cfg::kThreads);
+  cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+  cfg.stream = ln.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (ln.ev_start) record_event(ln.ev_start, ln.stream);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, p);
+  if (ln.ev_stop) record_event(ln.ev_stop, ln.stream);
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    *err = std::string("tc2_attn_kernel launch failed: ") + cudaGetErrorString(e);
+    return SDPA_ERR_CUDA;
+  }
+  return SDPA_OK;
+}
+
+template <bool kBF16>
+sdpa_status run_dtype(const Launch &ln, std::string *err) {
+  switch (ln.plan.pair) {
+    case 3: return run_tc2<kBF16, 192, 128>(ln, err);
+    case 5: return run_tc2<kBF16, 256, 256>(ln, err);
+  }
+  *err = "internal: no two-CTA instance for this head-dim pair";
+  return SDPA_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+
+sdpa_status launch_tc2(const Launch &ln, std::string *err) {
+  return ln.pb.dtype == SDPA_BF16 ? run_dtype<true>(ln, err) : run_dtype<false>(ln, err);
+}
+
+}  // namespace sdpa

@@ -73,6 +73,8 @@ extern "C" SDPA_API sdpa_status sdpa_forward_noalloc(const void *q, const void *
   Problem pb;
   pb.B = B; pb.Hq = Hq; pb.Hkv = Hkv; pb.L = L; pb.S = S; pb.Dqk = Dqk; pb.Dv = Dv;
   pb.scale = scale; pb.causal = causal; pb.window = window_size; pb.dtype = dtype;
+  pb.q_offset = S - L;  // queries end at the last key
+  pb.has_q_offset = 0;
   Plan pl;
   sdpa_status st = plan_call(pb, SDPA_PATH_AUTO, 0, &pl);
   if (st != SDPA_OK) return st;

@@ -28,8 +28,31 @@ struct AttnParams {
   void *out;          // [B*Hq*L][Dv] in the I/O type (written when splits == 1)
   float *part_o;      // [splits][B*Hq*L][Dv] fp32, normalised per split
   float *part_lse;    // [splits][B*Hq*L] fp32 natural-log LSE, -inf if empty
+  const float *sinks; // optional [Hq] sink logits (natural-log units), applied when splits == 1
+  float *lse_out;     // optional [B*Hq*L] natural-log LSE output, written when splits == 1
   Watchdog wd;
 };
+
+// Finish one row: fold in the head's sink (one more logit with no value row)
+// and return the factor O must be multiplied by; m (log2 units) and l are
+// updated to include the sink.  Without a sink the factor is 1/l.
+__device__ __forceinline__ float finish_row(const AttnParams &p, long grow, float &m, float &l) {
+  if (p.sinks != nullptr) {
+    const int hq = (int)((grow / p.L) % p.Hq);
+    const float sg = p.sinks[hq] * 1.4426950408889634f;
+    const float mf = fmaxf(m, sg);
+    const float so = m == -INFINITY ? 0.f : exp2f(m - mf);
+    l = l * so + exp2f(sg - mf);
+    m = mf;
+    return l > 0.f ? so / l : 0.f;
+  }
+  return l > 0.f ? 1.f / l : 0.f;
+}
+
+// Natural-log LSE of a finished row (m in log2 units).
+__device__ __forceinline__ float row_lse(float m, float l) {
+  return l > 0.f ? (m + log2f(l)) * 0.693147180559945309f : -INFINITY;
+}
 
 // Range of positions covered by the valid rows of a tile.
 struct TileRows {

@@ -84,6 +84,9 @@ __global__ void __launch_bounds__(SplitKvCfg<DQK, DV, BN, WR, WK, NST>::kThreads
     fence_barrier_init();
   }
   __syncthreads();
+  // Let the dependent combine launch now: its CTAs wait in griddepcontrol.wait
+  // until this grid has finished, so its launch latency overlaps this pass.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (warp == Cfg::kConsumers) {
     // ===================== producer warp =====================
@@ -324,14 +327,19 @@ __global__ void __launch_bounds__(SplitKvCfg<DQK, DV, BN, WR, WK, NST>::kThreads
   }
 
   // ---- epilogue ----
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const float inv_a = l_a > 0.f ? 1.f / l_a : 0.f;
-  const float inv_b = l_b > 0.f ? 1.f / l_b : 0.f;
+  float inv_a = l_a > 0.f ? 1.f / l_a : 0.f;
+  float inv_b = l_b > 0.f ? 1.f / l_b : 0.f;
   const bool va = lr_a < tr.nvalid, vb = lr_b < tr.nvalid;
   const long grow_a = (long)bh * p.R + tr.row0 + lr_a;
   const long grow_b = grow_a + 8;
   const int c0 = (lane & 3) * 2;
   if (p.splits == 1) {
+    inv_a = finish_row(p, grow_a, m_a, l_a);
+    inv_b = finish_row(p, grow_b, m_b, l_b);
+    if (p.lse_out != nullptr && (lane & 3) == 0) {
+      if (va) p.lse_out[grow_a] = row_lse(m_a, l_a);
+      if (vb) p.lse_out[grow_b] = row_lse(m_b, l_b);
+    }
     uint32_t *out32 = reinterpret_cast<uint32_t *>(p.out);
 #pragma unroll
     for (int i = 0; i < kOT; ++i) {
@@ -357,10 +365,9 @@ __global__ void __launch_bounds__(SplitKvCfg<DQK, DV, BN, WR, WK, NST>::kThreads
       }
     }
     if ((lane & 3) == 0) {
-      constexpr float kLn2 = 0.693147180559945309f;
       float *pl = p.part_lse + (long)split * total_rows;
-      if (va) pl[grow_a] = l_a > 0.f ? (m_a + log2f(l_a)) * kLn2 : -INFINITY;
-      if (vb) pl[grow_b] = l_b > 0.f ? (m_b + log2f(l_b)) * kLn2 : -INFINITY;
+      if (va) pl[grow_a] = row_lse(m_a, l_a);
+      if (vb) pl[grow_b] = row_lse(m_b, l_b);
     }
   }
   (void)ok;
@@ -371,7 +378,9 @@ __global__ void __launch_bounds__(SplitKvCfg<DQK, DV, BN, WR, WK, NST>::kThreads
 // a log-sum-exp merge; mlx PR #3637: the 2-pass kernel's aggregation).
 // One CTA of 128 threads per output row:
 //   LSE = max_s LSE_s + ln sum_s exp(LSE_s - max),  O = sum_s exp(LSE_s - LSE) O_s
-// Splits that saw no visible key carry LSE_s = -inf and weight 0.  The
+// Splits that saw no visible key carry LSE_s = -inf and weight 0.  A head's
+// sink (when given) joins as one more term with weight exp(sink - LSE) and
+// no value row.  The
 // weights go to shared memory once; each thread then owns output columns
 // and reads the splits' partials with several loads in flight.
 // Launched as a programmatic dependent of the split pass: it waits for that
@@ -381,24 +390,28 @@ template <bool kBF16>
 __global__ void __launch_bounds__(128) combine_kernel(const float *__restrict__ part_o,
                                                       const float *__restrict__ part_lse,
                                                       void *__restrict__ out, float *lse_out,
-                                                      long total_rows, int Dv, int splits) {
+                                                      const float *__restrict__ sinks,
+                                                      long total_rows, int Dv, int splits, int L,
+                                                      int Hq) {
   extern __shared__ float s_w[];  // [splits]
   __shared__ float s_red[4];
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const long row = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   float mx = -INFINITY;
-  for (int s = tid; s < splits; s += 128) mx = fmaxf(mx, part_lse[(long)s * total_rows + row]);
+  for (int s = tid; s < splits; s += 128) mx = fmaxf(mx, __ldcg(part_lse + (long)s * total_rows + row));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   if (lane == 0) s_red[wid] = mx;
   __syncthreads();
   mx = fmaxf(fmaxf(s_red[0], s_red[1]), fmaxf(s_red[2], s_red[3]));
+  const float sink = sinks != nullptr ? sinks[(int)((row / L) % Hq)] : -INFINITY;
+  mx = fmaxf(mx, sink);
   const float ref = mx == -INFINITY ? 0.f : mx;
   __syncthreads();
   float den = 0.f;
   for (int s = tid; s < splits; s += 128) {
-    const float w = __expf(part_lse[(long)s * total_rows + row] - ref);
+    const float w = __expf(__ldcg(part_lse + (long)s * total_rows + row) - ref);
     s_w[s] = w;
     den += w;
   }
@@ -406,27 +419,29 @@ __global__ void __launch_bounds__(128) combine_kernel(const float *__restrict__ 
   for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
   if (lane == 0) s_red[wid] = den;
   __syncthreads();
-  den = s_red[0] + s_red[1] + s_red[2] + s_red[3];
+  den = s_red[0] + s_red[1] + s_red[2] + s_red[3] + (sinks != nullptr ? __expf(sink - ref) : 0.f);
   const float inv = den > 0.f ? 1.f / den : 0.f;
   const long stride = total_rows * Dv;
   for (int d = tid; d < Dv; d += 128) {
     const float *src = part_o + row * Dv + d;
-    float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+    float acc[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) acc[t] = 0.f;
     int s = 0;
-    for (; s + 4 <= splits; s += 4) {
-      const float v0 = src[(long)(s + 0) * stride], v1 = src[(long)(s + 1) * stride];
-      const float v2 = src[(long)(s + 2) * stride], v3 = src[(long)(s + 3) * stride];
-      acc0 += s_w[s + 0] * v0;
-      acc1 += s_w[s + 1] * v1;
-      acc2 += s_w[s + 2] * v2;
-      acc3 += s_w[s + 3] * v3;
+    for (; s + 8 <= splits; s += 8) {
+      float v[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) v[t] = __ldcg(src + (long)(s + t) * stride);
+#pragma unroll
+      for (int t = 0; t < 8; ++t) acc[t] += s_w[s + t] * v[t];
     }
-    for (; s < splits; ++s) acc0 += s_w[s] * src[(long)s * stride];
-    const float acc = ((acc0 + acc1) + (acc2 + acc3)) * inv;
+    for (; s < splits; ++s) acc[s & 7] += s_w[s] * __ldcg(src + (long)s * stride);
+    const float res =
+        (((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]))) * inv;
     if constexpr (kBF16)
-      reinterpret_cast<__nv_bfloat16 *>(out)[row * Dv + d] = __float2bfloat16_rn(acc);
+      reinterpret_cast<__nv_bfloat16 *>(out)[row * Dv + d] = __float2bfloat16_rn(res);
     else
-      reinterpret_cast<__half *>(out)[row * Dv + d] = __float2half_rn(acc);
+      reinterpret_cast<__half *>(out)[row * Dv + d] = __float2half_rn(res);
   }
   if (lse_out != nullptr && tid == 0) lse_out[row] = den > 0.f ? ref + logf(den) : -INFINITY;
 }

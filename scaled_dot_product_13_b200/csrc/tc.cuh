@@ -7,23 +7,29 @@
 //   per-element masks run only on the diagonal, window-edge and tail blocks
 //   (mlx PR #3552, "Implementation").
 //
-// Warp roles (192 threads):
-//   warps 0-3  softmax: thread t owns query row t of the tile (TMEM lane t);
-//              fp32 online softmax with a lazily updated running max, P
-//              written to shared memory as the 16-bit input type; at the end
-//              the epilogue (O / l, rounded, stored).
-//   warp 4     TMA producer: Q once, then K and V blocks, in the order the
-//              MMA consumes them (K0, K1, V0, K2, V1, ...), through a FIFO
-//              ring of NSLOT shared-memory slots (128-byte swizzle, zero fill
-//              past S and past the head dim).
-//   warp 5     allocates TMEM and issues tcgen05.mma from one thread:
-//              S_j = Q K_j^T into one of two TMEM score buffers, then
-//              O += P_{j-1} V_{j-1} into the TMEM output accumulator, so the
-//              tensor core computes the next scores while the softmax warps
-//              work on the current ones.
+// Warp roles (320 threads):
+//   warps 0-7  softmax: warps w and w+4 share query rows 32(w%4) .. +31
+//              (TMEM lanes), each taking one half of every key block's
+//              columns; the pair exchanges its row maxima through shared
+//              memory behind a bounded mbarrier.  fp32 online softmax with a
+//              lazily updated running max.  P is rounded to the 16-bit input
+//              type and written back into tensor memory over the scores it
+//              came from.  At the end the epilogue (O / l, rounded, stored),
+//              each warp of a pair writing half of O's columns.
+//   warp 8     TMA producer: Q once, then K and V blocks in the order the MMA
+//              consumes them (K0, K1, then V_j, K_{j+2} for j = 0, 1, ...)
+//              through a FIFO ring of NSLOT shared-memory slots (128-byte
+//              swizzle, zero fill past S and past the head dim), and L2
+//              prefetches of the blocks further ahead.
+//   warp 9     allocates TMEM and issues tcgen05.mma from one thread:
+//              S_j = Q K_j^T (A = Q from shared memory) into score buffer
+//              j % 3, and O += P_j V_j with A = P_j read from tensor memory,
+//              then S_{j+2}; the tensor core computes the next scores while
+//              the softmax warps work on the current ones.
 //
-// TMEM (512 columns x 128 lanes x 32 bit): S buffers at columns [0, BN) and
-// [BN, 2BN), O at [2BN, 2BN + DV).
+// TMEM (512 columns x 128 lanes x 32 bit): three score buffers of BN
+// columns (P_j overwrites the first BN/2 columns of its buffer as packed
+// 16-bit pairs), O at [3 BN, 3 BN + DV).
 //
 // Running max: the row max m used as the exponent reference is only moved
 // when a block's max exceeds it by more than 8 (log2 units), so O in TMEM is
@@ -39,6 +45,7 @@ namespace sdpa {
 template <int DQK, int DV, int BN, int NSLOT>
 struct TcCfg {
   static constexpr int kBM = 128;
+  static constexpr int kBufs = 3;        // score / P buffers in TMEM
   static constexpr int kQBoxes = (DQK + 63) / 64;
   static constexpr int kVBoxes = (DV + 63) / 64;
   static constexpr int kKS = DQK / 16;   // k16 steps of S = Q K^T
@@ -47,44 +54,54 @@ struct TcCfg {
   static constexpr uint32_t kKBytes = kQBoxes * BN * 128;
   static constexpr uint32_t kVBytes = kVBoxes * BN * 128;
   static constexpr uint32_t kSlotBytes = kKBytes > kVBytes ? kKBytes : kVBytes;
-  static constexpr uint32_t kPBytes = kBM * BN * 2;
-  static constexpr uint32_t kPOff = kQBytes;
-  static constexpr uint32_t kSlotOff = kPOff + 2 * kPBytes;
-  static constexpr uint32_t kBarOff = kSlotOff + NSLOT * kSlotBytes;
-  static constexpr int kNumBars = 2 * NSLOT + 13;
-  static constexpr uint32_t kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;
-  static constexpr int kThreads = 192;
+  static constexpr uint32_t kSlotOff = kQBytes;
+  static constexpr uint32_t kXOff = kSlotOff + NSLOT * kSlotBytes;  // row-max exchange
+  static constexpr uint32_t kXBytes = 4 * kBM * 4;  // [2 bufs][2 halves][128] row maxima
+  static constexpr uint32_t kBarOff = kXOff + kXBytes;
+  static constexpr int kNumBars = 2 * NSLOT + 17;
+  // exact: the dynamic shared-memory base is 1024-byte aligned (checked at run time)
+  static constexpr uint32_t kSmemBytes = kBarOff + kNumBars * 8 + 16;
+  static constexpr int kThreads = 320;
+  static constexpr int kHalf = BN / 2;  // key columns per softmax thread
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr int kOCol = 2 * BN;
+  static constexpr int kOCol = kBufs * BN;
+  static constexpr int kPrefetch = 4;   // blocks prefetched to L2 beyond the one loaded
   static_assert(DQK % 16 == 0 && DV % 16 == 0 && DV >= 16 && DV <= 256, "head dims");
   static_assert(BN == 64 || BN == 128, "key block");
-  static_assert(2 * BN + DV <= 512, "TMEM columns");
+  static_assert(kBufs * BN + DV <= 512, "TMEM columns");
   static_assert(kSmemBytes <= 232448, "shared memory");
 };
 
 template <bool kBF16, int DQK, int DV, int BN, int NSLOT>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     tc_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   using Cfg = TcCfg<DQK, DV, BN, NSLOT>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                              ~uintptr_t(1023));
+  constexpr int NB = Cfg::kBufs;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // The 128-byte swizzle atoms need 1024-byte aligned tiles.  The layout has no
+  // slack for realignment, so a misaligned base is reported and the CTA exits
+  // before touching barriers or tensor memory.
+  if ((smem_u32(smem_raw) & 1023u) != 0u) {
+    if (threadIdx.x == 0) wd_record(p.wd, kWdSmemAlign);
+    return;
+  }
+  uint8_t *smem = smem_raw;
   uint8_t *sQ = smem;
-  uint8_t *sP = smem + Cfg::kPOff;
   uint8_t *sSlots = smem + Cfg::kSlotOff;
+  float *xmax = reinterpret_cast<float *>(smem + Cfg::kXOff);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kBarOff);
   uint64_t *slot_full = bars;
   uint64_t *slot_empty = bars + NSLOT;
   uint64_t *q_full = bars + 2 * NSLOT;
-  uint64_t *s_full = q_full + 1;   // [2]
-  uint64_t *s_free = s_full + 2;   // [2]
-  uint64_t *p_full = s_free + 2;   // [2]
-  uint64_t *p_free = p_full + 2;   // [2]
-  uint64_t *o_bar = p_free + 2;
-  uint64_t *fin_bar = o_bar + 1;
-  uint64_t *o_final = fin_bar + 1;  // one phase: every P V of the tile has completed
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(o_final + 1);
+  uint64_t *s_full = q_full + 1;      // [3] S_j complete (MMA -> softmax)
+  uint64_t *p_full = s_full + NB;     // [3] P_j in TMEM, O rescaled (softmax -> MMA)
+  uint64_t *buf_free = p_full + NB;   // [3] P_j V complete: buffer reusable (MMA -> MMA)
+  uint64_t *o_bar = buf_free + NB;    // one phase per P V
+  uint64_t *o_final = o_bar + 1;      // one phase: every P V of the tile has completed
+  uint64_t *fin_bar = o_final + 1;    // teardown drain of the MMA warp
+  uint64_t *pair_bar = fin_bar + 1;   // [4] softmax warp pairs (row-max exchange)
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(pair_bar + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -108,18 +125,18 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&slot_empty[s], 1);
     }
     mbar_init(q_full, 1);
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NB; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&s_free[b], 4);
-      mbar_init(&p_full[b], 4);
-      mbar_init(&p_free[b], 1);
+      mbar_init(&p_full[b], 8);
+      mbar_init(&buf_free[b], 1);
     }
     mbar_init(o_bar, 1);
-    mbar_init(fin_bar, 1);
     mbar_init(o_final, 1);
+    mbar_init(fin_bar, 1);
+    for (int q = 0; q < 4; ++q) mbar_init(&pair_bar[q], 64);
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(tmem_slot, Cfg::kTmemCols);
     tmem_relinquish();
   }
@@ -127,8 +144,10 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Let a dependent combine launch now (it waits for this grid to finish).
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ============================ TMA producer ============================
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
@@ -141,24 +160,13 @@ __global__ void __launch_bounds__(192, 1)
         tma_load_2d(sQ + bx * (Cfg::kBM * 128), &tm_q, q_full, bx * 64, grow0);
       int u = 0;
       bool ok = true;
-      // load order = MMA consumption order: K0, (K_j, V_{j-1}) for j >= 1, V_last
-      const int nloads = nblk > 0 ? 2 * nblk : 0;
-      for (int t = 0; t < nloads && ok; ++t) {
-        bool is_k;
-        int blk;
-        if (t == 0) {
-          is_k = true; blk = 0;
-        } else if (t == nloads - 1) {
-          is_k = false; blk = nblk - 1;
-        } else {
-          is_k = (t & 1) != 0;
-          blk = is_k ? (t + 1) / 2 : t / 2 - 1;
-        }
+      // one load into the next ring slot, plus an L2 prefetch further ahead
+      auto emit = [&](bool is_k, int blk) {
         const int slot = u % NSLOT;
         const uint32_t ph = (uint32_t)(u / NSLOT) & 1u;
         if (!mbar_wait(&slot_empty[slot], ph ^ 1u, p.wd, kWdTmaEmpty)) {
           ok = false;
-          break;
+          return;
         }
         uint8_t *dst = sSlots + slot * Cfg::kSlotBytes;
         const int k0 = k_lo + blk * BN;
@@ -167,6 +175,15 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int bx = 0; bx < Cfg::kQBoxes; ++bx)
             tma_load_3d(dst + bx * (BN * 128), &tm_k, &slot_full[slot], bx * 64, k0, bh);
+          const int pf = blk + Cfg::kPrefetch;
+          if (pf < nblk) {
+#pragma unroll
+            for (int bx = 0; bx < Cfg::kQBoxes; ++bx)
+              tma_prefetch_l2_3d(&tm_k, bx * 64, k_lo + pf * BN, bh);
+#pragma unroll
+            for (int bx = 0; bx < Cfg::kVBoxes; ++bx)
+              tma_prefetch_l2_3d(&tm_v, bx * 64, k_lo + pf * BN, bh);
+          }
         } else {
           mbar_arrive_expect_tx(&slot_full[slot], Cfg::kVBytes);
 #pragma unroll
@@ -174,72 +191,73 @@ __global__ void __launch_bounds__(192, 1)
             tma_load_3d(dst + bx * (BN * 128), &tm_v, &slot_full[slot], bx * 64, k0, bh);
         }
         ++u;
+      };
+      if (nblk > 0) emit(true, 0);
+      if (ok && nblk > 1) emit(true, 1);
+      for (int j = 0; ok && j < nblk; ++j) {
+        emit(false, j);
+        if (ok && j + 2 < nblk) emit(true, j + 2);
       }
       // drain copies still landing (only ever waits after an abort)
       mbar_wait_drain(q_full, 0, p.wd);
       for (int v = u - NSLOT > 0 ? u - NSLOT : 0; v < u; ++v)
         mbar_wait_drain(&slot_full[v % NSLOT], (uint32_t)(v / NSLOT) & 1u, p.wd);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ============================ MMA issuer ============================
     if (lane == 0) {
       constexpr uint32_t kIdescS = umma_idesc_f16(kBF16, 128, BN, false, false);
       constexpr uint32_t kIdescPV = umma_idesc_f16(kBF16, 128, DV, false, true);
       const uint32_t q_addr = smem_u32(sQ);
-      const uint32_t p_addr = smem_u32(sP);
       const uint32_t slot_addr = smem_u32(sSlots);
       bool ok = mbar_wait(q_full, 0, p.wd, kWdTmaFull);
       int u = 0;
-      auto pv = [&](int i) -> bool {
+      // S_n = Q K_n^T into buffer n % 3 (free once P_{n-3} V has completed)
+      auto issue_s = [&](int n) -> bool {
         const int slot = u % NSLOT;
         if (!mbar_wait(&slot_full[slot], (uint32_t)(u / NSLOT) & 1u, p.wd, kWdTmaFull)) return false;
         ++u;
-        const int pb = i & 1;
-        if (!mbar_wait(&p_full[pb], (uint32_t)(i >> 1) & 1u, p.wd, kWdSoftmax)) return false;
-        tc_fence_after();
-        const uint32_t vb = slot_addr + slot * Cfg::kSlotBytes;
-        const uint32_t pbase = p_addr + pb * Cfg::kPBytes;
-#pragma unroll
-        for (int ks = 0; ks < Cfg::kPVK; ++ks) {
-          const uint64_t a = umma_desc_sw128(pbase + (ks >> 2) * (Cfg::kBM * 128) + (ks & 3) * 32,
-                                             16, 1024);
-          const uint64_t b = umma_desc_sw128_mn(vb + ks * 2048, BN * 128, 1024);
-          tc_mma_ss(tmem + Cfg::kOCol, a, b, kIdescPV, (i > 0 || ks > 0) ? 1u : 0u);
-        }
-        tc_commit(o_bar);
-        tc_commit(&p_free[pb]);
-        tc_commit(&slot_empty[slot]);
-        return true;
-      };
-      for (int j = 0; ok && j < nblk; ++j) {
-        const int slot = u % NSLOT;
-        if (!mbar_wait(&slot_full[slot], (uint32_t)(u / NSLOT) & 1u, p.wd, kWdTmaFull)) {
-          ok = false;
-          break;
-        }
-        ++u;
-        const int sb = j & 1;
-        if (!mbar_wait(&s_free[sb], ((uint32_t)(j >> 1) & 1u) ^ 1u, p.wd, kWdSoftmax)) {
-          ok = false;
-          break;
-        }
+        const int b = n % NB;
+        if (!mbar_wait(&buf_free[b], ((uint32_t)(n / NB) & 1u) ^ 1u, p.wd, kWdMma)) return false;
         tc_fence_after();
         const uint32_t kb = slot_addr + slot * Cfg::kSlotBytes;
 #pragma unroll
         for (int ks = 0; ks < Cfg::kKS; ++ks) {
           const uint64_t a =
               umma_desc_sw128(q_addr + (ks >> 2) * (Cfg::kBM * 128) + (ks & 3) * 32, 16, 1024);
-          const uint64_t b = umma_desc_sw128(kb + (ks >> 2) * (BN * 128) + (ks & 3) * 32, 16, 1024);
-          tc_mma_ss(tmem + sb * BN, a, b, kIdescS, ks > 0 ? 1u : 0u);
+          const uint64_t bd = umma_desc_sw128(kb + (ks >> 2) * (BN * 128) + (ks & 3) * 32, 16, 1024);
+          tc_mma_ss(tmem + b * BN, a, bd, kIdescS, ks > 0 ? 1u : 0u);
         }
-        tc_commit(&s_full[sb]);
+        tc_commit(&s_full[b]);
         tc_commit(&slot_empty[slot]);
-        if (j >= 1 && !pv(j - 1)) {
-          ok = false;
-          break;
+        return true;
+      };
+      // O += P_j V_j with P_j in TMEM (first BN/2 columns of buffer j % 3)
+      auto issue_pv = [&](int j) -> bool {
+        const int slot = u % NSLOT;
+        if (!mbar_wait(&slot_full[slot], (uint32_t)(u / NSLOT) & 1u, p.wd, kWdTmaFull)) return false;
+        ++u;
+        const int b = j % NB;
+        if (!mbar_wait(&p_full[b], (uint32_t)(j / NB) & 1u, p.wd, kWdSoftmax)) return false;
+        tc_fence_after();
+        const uint32_t vb = slot_addr + slot * Cfg::kSlotBytes;
+#pragma unroll
+        for (int ks = 0; ks < Cfg::kPVK; ++ks) {
+          const uint64_t bd = umma_desc_sw128_mn(vb + ks * 2048, BN * 128, 1024);
+          tc_mma_ts(tmem + Cfg::kOCol, tmem + b * BN + ks * 8, bd, kIdescPV,
+                    (j > 0 || ks > 0) ? 1u : 0u);
         }
+        tc_commit(o_bar);
+        tc_commit(&buf_free[b]);
+        tc_commit(&slot_empty[slot]);
+        return true;
+      };
+      if (ok && nblk > 0) ok = issue_s(0);
+      if (ok && nblk > 1) ok = issue_s(1);
+      for (int j = 0; ok && j < nblk; ++j) {
+        ok = issue_pv(j);
+        if (ok && j + 2 < nblk) ok = issue_s(j + 2);
       }
-      if (ok && nblk > 0) ok = pv(nblk - 1);
       // o_bar tells one P V from the next only while at most one is pending;
       // the epilogue needs "all of them", so it gets its own one-shot barrier
       if (ok && nblk > 0) tc_commit(o_final);
@@ -248,44 +266,92 @@ __global__ void __launch_bounds__(192, 1)
       mbar_wait_drain(fin_bar, 0, p.wd);
     }
   } else {
-    // ====================== softmax warps (rows 0..127) ======================
-    const int r = warp * 32 + lane;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    // ============ softmax warps: rows 32*(w%4) .. +31, column half w/4 ============
+    const int quarter = warp & 3;
+    const int half = warp >> 2;
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const int pos = ((tr.row0 + r) % p.L) + p.off;
     const float c = p.scale_log2;
+    const bool c_pos = c >= 0.f;
+    const float neutral = c_pos ? -INFINITY : INFINITY;  // never wins the row reduction
+    constexpr int kH = Cfg::kHalf;
+    constexpr int kOChunks = DV / 16;
+    constexpr int kOC0 = (kOChunks + 1) / 2;
+    const int oc_begin = half == 0 ? 0 : kOC0;
+    const int oc_end = half == 0 ? kOC0 : kOChunks;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    const uint32_t p_row = smem_u32(sP) + r * 128;
+    uint32_t pair_phase = 0;
     for (int j = 0; j < nblk; ++j) {
-      const int sb = j & 1;
+      const int b = j % NB;
       bool w = true;
-      if (lane == 0) w = mbar_wait(&s_full[sb], (uint32_t)(j >> 1) & 1u, p.wd, kWdMma);
+      if (lane == 0) w = mbar_wait(&s_full[b], (uint32_t)(j / NB) & 1u, p.wd, kWdMma);
       if (!__shfl_sync(0xffffffffu, (int)w, 0)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      float s[BN];
+      float s[kH];
 #pragma unroll
-      for (int c32 = 0; c32 < BN / 32; ++c32)
-        tmem_ld32(tmem + lane_base + sb * BN + c32 * 32, s + c32 * 32);
+      for (int c32 = 0; c32 < kH / 32; ++c32)
+        tmem_ld32(tmem + lane_base + b * BN + half * kH + c32 * 32, s + c32 * 32);
       tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[sb]);
 
-      const int k0 = k_lo + j * BN;
+      // ---- this half's raw row max (masked keys excluded) ----
+      const int kbase = k_lo + j * BN;
+      const bool masked = block_needs_mask(p, tr, kbase, BN);
+      uint64_t vis = ~0ull;
+      if (masked) {
+        vis = 0ull;
 #pragma unroll
-      for (int i = 0; i < BN; ++i) s[i] *= c;
-      if (block_needs_mask(p, tr, k0, BN)) {
-#pragma unroll
-        for (int i = 0; i < BN; ++i)
-          if (!key_visible(p, pos, k0 + i)) s[i] = -INFINITY;
+        for (int i = 0; i < kH; ++i) {
+          if (key_visible(p, pos, kbase + half * kH + i)) vis |= 1ull << i;
+          else s[i] = neutral;
+        }
       }
-      float mx = -INFINITY;
+      float mr[4];
 #pragma unroll
-      for (int i = 0; i < BN; ++i) mx = fmaxf(mx, s[i]);
-      const float m_new = fmaxf(m_used, mx);
+      for (int t = 0; t < 4; ++t) mr[t] = s[t];
+      if (c_pos) {
+#pragma unroll
+        for (int i = 4; i < kH; i += 8) {
+          mr[0] = fmax3f(mr[0], s[i], s[i + 1]);
+          mr[1] = fmax3f(mr[1], s[i + 2], s[i + 3]);
+          if (i + 4 < kH) {
+            mr[2] = fmax3f(mr[2], s[i + 4], s[i + 5]);
+            mr[3] = fmax3f(mr[3], s[i + 6], s[i + 7]);
+          }
+        }
+        mr[0] = fmax3f(mr[0], mr[1], fmaxf(mr[2], mr[3]));
+      } else {
+#pragma unroll
+        for (int i = 4; i < kH; i += 8) {
+          mr[0] = fmin3f(mr[0], s[i], s[i + 1]);
+          mr[1] = fmin3f(mr[1], s[i + 2], s[i + 3]);
+          if (i + 4 < kH) {
+            mr[2] = fmin3f(mr[2], s[i + 4], s[i + 5]);
+            mr[3] = fmin3f(mr[3], s[i + 6], s[i + 7]);
+          }
+        }
+        mr[0] = fmin3f(mr[0], mr[1], fminf(mr[2], mr[3]));
+      }
+      // ---- combine with the other half of the row (bounded pair barrier).
+      // The barrier also orders this warp's score reads before the partner
+      // overwrites them with P. ----
+      xmax[((j & 1) * 2 + half) * Cfg::kBM + r] = mr[0];
+      tc_fence_before();
+      mbar_arrive(&pair_bar[quarter]);
+      if (!mbar_wait(&pair_bar[quarter], pair_phase & 1u, p.wd, kWdSoftmax)) {
+        ok = false;
+        break;
+      }
+      ++pair_phase;
+      tc_fence_after();
+      const float other = xmax[((j & 1) * 2 + (half ^ 1)) * Cfg::kBM + r];
+      const float mraw = c_pos ? fmaxf(mr[0], other) : fminf(mr[0], other);
+      const float mblk = isinf(mraw) ? -INFINITY : mraw * c;
+      const float m_new = fmaxf(m_used, mblk);
       const bool need = m_new > m_used + 8.0f;
       float alpha = 1.f;
       if (need) {
@@ -294,11 +360,11 @@ __global__ void __launch_bounds__(192, 1)
         l *= alpha;
       }
       if (j > 0 && __any_sync(0xffffffffu, need)) {
-        // O holds P_0..P_{j-1} V: wait for the last P V, then rescale in TMEM.
-        // Parity is unambiguous here: S_j's completion implies P_{j-2} V
-        // completed (one thread issues both, in order), and P_j V is not
-        // issued before this warp signals p_full, so o_bar is in phase j-1
-        // or j.
+        // O holds P_0..P_{j-1} V: wait for the last P V, then rescale this
+        // warp's columns in TMEM.  Parity is unambiguous here: S_j was issued
+        // after P_{j-2} V by the same thread, so S_j's completion implies that
+        // P V completed; P_j V is not issued before p_full: o_bar is in phase
+        // j-1 or j.
         if (lane == 0) w = mbar_wait(o_bar, (uint32_t)(j - 1) & 1u, p.wd, kWdMma);
         if (!__shfl_sync(0xffffffffu, (int)w, 0)) {
           ok = false;
@@ -306,7 +372,7 @@ __global__ void __launch_bounds__(192, 1)
         }
         tc_fence_after();
 #pragma unroll 1
-        for (int c16 = 0; c16 < DV / 16; ++c16) {
+        for (int c16 = oc_begin; c16 < oc_end; ++c16) {
           float o[16];
           tmem_ld16(tmem + lane_base + Cfg::kOCol + c16 * 16, o);
           tmem_wait_ld();
@@ -316,37 +382,46 @@ __global__ void __launch_bounds__(192, 1)
         }
         tmem_wait_st();
       }
+      // ---- P = exp2(s * c - m) (two lanes per FMA), row sums ----
       const float mref = m_used == -INFINITY ? 0.f : m_used;
-      float rs = 0.f;
+      const float2 c2 = make_float2(c, c), nm2 = make_float2(-mref, -mref);
+      float2 acc[4];
 #pragma unroll
-      for (int i = 0; i < BN; ++i) {
-        s[i] = fast_exp2(s[i] - mref);
-        rs += s[i];
-      }
-      l += rs;
-      // P buffer sb is free once the P V that last read it has completed
-      if (lane == 0) w = mbar_wait(&p_free[sb], ((uint32_t)(j >> 1) & 1u) ^ 1u, p.wd, kWdMma);
-      if (!__shfl_sync(0xffffffffu, (int)w, 0)) {
-        ok = false;
-        break;
-      }
-      const uint32_t pb = p_row + sb * Cfg::kPBytes;
+      for (int t = 0; t < 4; ++t) acc[t] = make_float2(0.f, 0.f);
+      uint32_t pk[kH / 2];
 #pragma unroll
-      for (int ch = 0; ch < BN / 8; ++ch) {
-        const uint32_t addr = pb + (ch >> 3) * (Cfg::kBM * 128) + ((((uint32_t)ch & 7u) ^ ((uint32_t)r & 7u)) << 4);
-        st_shared_v4(addr, pack2<kBF16>(s[ch * 8 + 0], s[ch * 8 + 1]),
-                     pack2<kBF16>(s[ch * 8 + 2], s[ch * 8 + 3]),
-                     pack2<kBF16>(s[ch * 8 + 4], s[ch * 8 + 5]),
-                     pack2<kBF16>(s[ch * 8 + 6], s[ch * 8 + 7]));
+      for (int i = 0; i < kH; i += 2) {
+        float2 t = fma2(make_float2(s[i], s[i + 1]), c2, nm2);
+        t.x = fast_exp2(t.x);
+        t.y = fast_exp2(t.y);
+        if (masked) {
+          t.x = ((vis >> i) & 1ull) ? t.x : 0.f;
+          t.y = ((vis >> (i + 1)) & 1ull) ? t.y : 0.f;
+        }
+        acc[(i >> 1) & 3] = add2(acc[(i >> 1) & 3], t);
+        pk[i >> 1] = pack2<kBF16>(t.x, t.y);
       }
-      fence_proxy_async_smem();
+      const float2 a01 = add2(acc[0], acc[1]), a23 = add2(acc[2], acc[3]);
+      const float2 at = add2(a01, a23);
+      l += at.x + at.y;
+      // P_j into this warp's columns of buffer b (over the scores of half 0)
+#pragma unroll
+      for (int c16 = 0; c16 < kH / 32; ++c16)
+        tmem_st_u16x(tmem + lane_base + b * BN + half * (kH / 2) + c16 * 16, pk + c16 * 16);
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[sb]);
+      if (lane == 0) mbar_arrive(&p_full[b]);
     }
 
     // ------------------------------ epilogue ------------------------------
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    // row sum = both halves' partial sums, exchanged through the max buffer the
+    // last block did not use (its last reader passed the last pair barrier)
+    float *xl = xmax + (nblk & 1) * 2 * Cfg::kBM;
+    xl[half * Cfg::kBM + r] = l;
+    mbar_arrive(&pair_bar[quarter]);
+    if (!mbar_wait(&pair_bar[quarter], pair_phase & 1u, p.wd, kWdSoftmax)) ok = false;
+    l += xl[(half ^ 1) * Cfg::kBM + r];
     if (ok && nblk > 0) {
       bool w = true;
       if (lane == 0) w = mbar_wait(o_final, 0, p.wd, kWdMma);
@@ -355,12 +430,14 @@ __global__ void __launch_bounds__(192, 1)
     }
     const bool valid = r < tr.nvalid;
     const long grow = (long)bh * p.R + tr.row0 + r;
-    const float inv = l > 0.f ? 1.f / l : 0.f;
     const bool have_o = ok && nblk > 0;
+    float inv = l > 0.f ? 1.f / l : 0.f;
     if (p.splits == 1) {
+      inv = finish_row(p, grow, m_used, l);
+      if (p.lse_out != nullptr && valid && half == 0) p.lse_out[grow] = row_lse(m_used, l);
       uint8_t *orow = reinterpret_cast<uint8_t *>(p.out) + grow * p.Dv * 2;
 #pragma unroll 1
-      for (int c16 = 0; c16 < DV / 16; ++c16) {
+      for (int c16 = oc_begin; c16 < oc_end; ++c16) {
         float o[16];
         if (have_o) {
           tmem_ld16(tmem + lane_base + Cfg::kOCol + c16 * 16, o);
@@ -382,7 +459,7 @@ __global__ void __launch_bounds__(192, 1)
       const long total_rows = (long)p.B * p.Hq * p.L;
       float *po = p.part_o + ((long)split * total_rows + grow) * p.Dv;
 #pragma unroll 1
-      for (int c16 = 0; c16 < DV / 16; ++c16) {
+      for (int c16 = oc_begin; c16 < oc_end; ++c16) {
         float o[16];
         if (have_o) {
           tmem_ld16(tmem + lane_base + Cfg::kOCol + c16 * 16, o);
@@ -400,18 +477,15 @@ __global__ void __launch_bounds__(192, 1)
                             o[q4 * 4 + 3] * inv);
         }
       }
-      if (valid) {
-        constexpr float kLn2 = 0.693147180559945309f;
-        p.part_lse[(long)split * total_rows + grow] =
-            (have_o && l > 0.f) ? (m_used + log2f(l)) * kLn2 : -INFINITY;
-      }
+      if (valid && half == 0)
+        p.part_lse[(long)split * total_rows + grow] = have_o ? row_lse(m_used, l) : -INFINITY;
     }
   }
 
   // ------------------------------ teardown ------------------------------
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, Cfg::kTmemCols);
   }

@@ -1,0 +1,501 @@
+// Attention on a pair of SMs: tcgen05 cta_group::2 MMAs over 256-row tiles.
+//
+// The same method as tc.cuh (key-block range from kb_start / kb_lim, edge
+// masks, fp32 online softmax with a lazily moved running max, P in tensor
+// memory), but two CTAs of a cluster own one 256-row tile together: CTA r
+// holds rows [128 r, 128 r + 128) of Q, of S and of O, while each K block is
+// split by keys (CTA r loads keys [r BN/2, (r+1) BN/2) of it) and each V block
+// by columns (CTA r loads columns [r DV/2, (r+1) DV/2)).  The even CTA issues
+// M=256 MMAs that read both CTAs' shared and tensor memory.  Every K/V byte a
+// CTA loads therefore feeds 256 query rows instead of 128, which halves the
+// load traffic per FLOP: with 128-row tiles and head dim 256 the kernel is
+// limited by how fast K/V reach shared memory, not by the tensor cores.
+//
+// Loads stay plain TMA into the loading CTA's own shared memory (no
+// multicast).  A forwarder warp of the odd CTA relays the completion of each
+// of its loads to the even CTA's barriers; the even CTA's MMA thread commits
+// to barriers in both CTAs with two plain commits.
+//
+// Warp roles per CTA (352 threads):
+//   warps 0-7  softmax on this CTA's 128 rows, as in tc.cuh; P_j is written
+//              to this CTA's TMEM and signalled to the even CTA's p_full.
+//   warp 8     TMA producer for this CTA's halves.
+//   warp 9     TMEM allocation (pair); the MMA issuer in the even CTA.
+//   warp 10    odd CTA: forwards its load completions to the even CTA.
+//
+// TMEM per CTA: two score buffers of BN columns (P_j over the first BN/2
+// columns of buffer j % 2), O at [2 BN, 2 BN + DV).  A score buffer is reused
+// two blocks later: the MMA for S_{j+2} is issued after P_j V by the same
+// thread, and one thread's tcgen05 MMAs execute in order.
+#pragma once
+
+#include "params.cuh"
+
+namespace sdpa {
+
+template <int DQK, int DV, int BN, int NSLOT>
+struct Tc2Cfg {
+  static constexpr int kBM = 128;              // rows per CTA (256 per pair)
+  static constexpr int kQBoxes = DQK / 64;
+  static constexpr int kVHalf = DV / 2;         // V columns per CTA
+  static constexpr int kVBoxes = kVHalf / 64;
+  static constexpr int kKS = DQK / 16;
+  static constexpr int kPVK = BN / 16;
+  static constexpr uint32_t kQBytes = kQBoxes * kBM * 128;
+  static constexpr uint32_t kKBytes = kQBoxes * (BN / 2) * 128;  // this CTA's K half
+  static constexpr uint32_t kVBytes = kVBoxes * BN * 128;        // this CTA's V half
+  static constexpr uint32_t kSlotBytes = kKBytes > kVBytes ? kKBytes : kVBytes;
+  static constexpr uint32_t kSlotOff = kQBytes;
+  static constexpr uint32_t kXOff = kSlotOff + NSLOT * kSlotBytes;
+  static constexpr uint32_t kXBytes = 4 * kBM * 4;
+  static constexpr uint32_t kBarOff = kXOff + kXBytes;
+  static constexpr int kNumBars = 3 * NSLOT + 20;
+  static constexpr uint32_t kSmemBytes = kBarOff + kNumBars * 8 + 16;
+  static constexpr int kThreads = 352;
+  static constexpr int kHalf = BN / 2;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr int kOCol = 2 * BN;
+  static_assert(DQK % 64 == 0 && (DV == 128 || DV == 256), "pair split needs 64-column halves");
+  static_assert(BN == 128, "key block");
+  static_assert(2 * BN + DV <= 512, "TMEM columns");
+  static_assert(kSmemBytes <= 232448, "shared memory");
+};
+
+template <bool kBF16, int DQK, int DV, int BN, int NSLOT>
+__global__ void __launch_bounds__(352, 1)
+    tc2_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+  using Cfg = Tc2Cfg<DQK, DV, BN, NSLOT>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // same layout in both CTAs, so both take this exit together
+  if ((smem_u32(smem_raw) & 1023u) != 0u) {
+    if (threadIdx.x == 0) wd_record(p.wd, kWdSmemAlign);
+    return;
+  }
+  uint8_t *smem = smem_raw;
+  uint8_t *sQ = smem;
+  uint8_t *sSlots = smem + Cfg::kSlotOff;
+  float *xmax = reinterpret_cast<float *>(smem + Cfg::kXOff);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kBarOff);
+  uint64_t *slot_full = bars;                // [NSLOT] this CTA's loads landed
+  uint64_t *slot_empty = slot_full + NSLOT;  // [NSLOT] the pair's MMA is done with the slot
+  uint64_t *peer_full = slot_empty + NSLOT;  // [NSLOT] even CTA: the odd CTA's loads landed
+  uint64_t *q_full = peer_full + NSLOT;
+  uint64_t *peer_q = q_full + 1;             // even CTA: the odd CTA's Q landed
+  uint64_t *s_full = peer_q + 1;             // [2]
+  uint64_t *p_full = s_full + 2;             // [2] even CTA: P_j of both CTAs written
+  uint64_t *o_bar = p_full + 2;
+  uint64_t *o_final = o_bar + 1;
+  uint64_t *fin_bar = o_final + 1;           // all MMAs of the pair complete
+  uint64_t *bye_bar = fin_bar + 1;           // teardown: the other CTA is done with us
+  uint64_t *pair_bar = bye_bar + 1;          // [4] softmax warp pairs
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(pair_bar + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+
+  // --- work item of the pair: (batch*KV head) fastest, then split, then the
+  // 256-row tile, heaviest first ---
+  int bid = blockIdx.x >> 1;
+  const int BH = p.B * p.Hkv;
+  const int bh = bid % BH;
+  bid /= BH;
+  const int split = bid % p.splits;
+  const int pair_tile = p.row_tiles - 1 - bid / p.splits;
+  const TileRows tpair = tile_rows(p, pair_tile, 2 * Cfg::kBM);
+  int k_lo, k_hi;
+  tile_key_range(p, tpair, BN, split, k_lo, k_hi);  // identical in both CTAs
+  const int nblk = (k_hi - k_lo) / BN;
+  TileRows tr = tile_rows(p, pair_tile * 2 + (int)rank, Cfg::kBM);  // this CTA's rows
+  if (tr.nvalid <= 0) {
+    tr.nvalid = 0;
+    tr.pos_min = tpair.pos_min;
+    tr.pos_max = tpair.pos_max;
+  }
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NSLOT; ++s) {
+      mbar_init(&slot_full[s], 1);
+      mbar_init(&slot_empty[s], 1);
+      mbar_init(&peer_full[s], 1);
+    }
+    mbar_init(q_full, 1);
+    mbar_init(peer_q, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&p_full[b], 16);
+    }
+    mbar_init(o_bar, 1);
+    mbar_init(o_final, 1);
+    mbar_init(fin_bar, 1);
+    mbar_init(bye_bar, 1);
+    for (int q = 0; q < 4; ++q) mbar_init(&pair_bar[q], 64);
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    tmem_alloc_pair(tmem_slot, Cfg::kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  // barriers of both CTAs are initialised before any remote arrive
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+  if (warp == 8) {
+    // ====================== TMA producer (this CTA's halves) ======================
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      const int grow0 = bh * p.R + tpair.row0 + (int)rank * Cfg::kBM;
+      mbar_arrive_expect_tx(q_full, Cfg::kQBytes);
+#pragma unroll
+      for (int bx = 0; bx < Cfg::kQBoxes; ++bx)
+        tma_load_2d(sQ + bx * (Cfg::kBM * 128), &tm_q, q_full, bx * 64, grow0);
+      int u = 0;
+      bool ok = true;
+      auto emit = [&](bool is_k, int blk) {
+        const int slot = u % NSLOT;
+        if (!mbar_wait_cluster(&slot_empty[slot], ((uint32_t)(u / NSLOT) & 1u) ^ 1u, p.wd,
+                               kWdTmaEmpty)) {
+          ok = false;
+          return;
+        }
+        uint8_t *dst = sSlots + slot * Cfg::kSlotBytes;
+        const int k0 = k_lo + blk * BN;
+        if (is_k) {
+          mbar_arrive_expect_tx(&slot_full[slot], Cfg::kKBytes);
+#pragma unroll
+          for (int bx = 0; bx < Cfg::kQBoxes; ++bx)
+            tma_load_3d(dst + bx * ((BN / 2) * 128), &tm_k, &slot_full[slot], bx * 64,
+                        k0 + (int)rank * (BN / 2), bh);
+        } else {
+          mbar_arrive_expect_tx(&slot_full[slot], Cfg::kVBytes);
+#pragma unroll
+          for (int bx = 0; bx < Cfg::kVBoxes; ++bx)
+            tma_load_3d(dst + bx * (BN * 128), &tm_v, &slot_full[slot],
+                        (int)rank * Cfg::kVHalf + bx * 64, k0, bh);
+        }
+        ++u;
+      };
+      if (nblk > 0) emit(true, 0);
+      if (ok && nblk > 1) emit(true, 1);
+      for (int j = 0; ok && j < nblk; ++j) {
+        emit(false, j);
+        if (ok && j + 2 < nblk) emit(true, j + 2);
+      }
+      mbar_wait_drain(q_full, 0, p.wd);
+      for (int v = u - NSLOT > 0 ? u - NSLOT : 0; v < u; ++v)
+        mbar_wait_drain(&slot_full[v % NSLOT], (uint32_t)(v / NSLOT) & 1u, p.wd);
+    }
+  } else if (warp == 10) {
+    // ============ odd CTA: relay its load completions to the even CTA ============
+    if (!leader && lane == 0) {
+      const int nloads = nblk > 0 ? 2 * nblk : 0;
+      const uint32_t leader_peer_q = mapa_shared(smem_u32(peer_q), 0);
+      bool ok = mbar_wait(q_full, 0, p.wd, kWdTmaFull);
+      if (ok) mbar_arrive_cluster(leader_peer_q);
+      for (int u = 0; ok && u < nloads; ++u) {
+        const int slot = u % NSLOT;
+        if (!mbar_wait(&slot_full[slot], (uint32_t)(u / NSLOT) & 1u, p.wd, kWdTmaFull)) break;
+        mbar_arrive_cluster(mapa_shared(smem_u32(&peer_full[slot]), 0));
+      }
+    }
+  } else if (warp == 9) {
+    // ====================== MMA issuer (even CTA only) ======================
+    if (leader && lane == 0) {
+      constexpr uint32_t kIdescS = umma_idesc_f16(kBF16, 256, BN, false, false);
+      constexpr uint32_t kIdescPV = umma_idesc_f16(kBF16, 256, DV, false, true);
+      const uint32_t q_addr = smem_u32(sQ);
+      const uint32_t slot_addr = smem_u32(sSlots);
+      // commit targets in both CTAs
+      auto both = [&](uint64_t *bar) {
+        const uint32_t a = smem_u32(bar);
+        tc_commit_pair(mapa_shared(a, 0));
+        tc_commit_pair(mapa_shared(a, 1));
+      };
+      bool ok = mbar_wait(q_full, 0, p.wd, kWdTmaFull) &&
+                mbar_wait_cluster(peer_q, 0, p.wd, kWdTmaFull);
+      int u = 0;
+      auto take_slot = [&](int &slot) -> bool {
+        slot = u % NSLOT;
+        const uint32_t ph = (uint32_t)(u / NSLOT) & 1u;
+        if (!mbar_wait(&slot_full[slot], ph, p.wd, kWdTmaFull)) return false;
+        if (!mbar_wait_cluster(&peer_full[slot], ph, p.wd, kWdTmaFull)) return false;
+        ++u;
+        return true;
+      };
+      auto issue_s = [&](int n) -> bool {
+        int slot;
+        if (!take_slot(slot)) return false;
+        const int b = n & 1;
+        tc_fence_after();
+        const uint32_t kb = slot_addr + slot * Cfg::kSlotBytes;
+#pragma unroll
+        for (int ks = 0; ks < Cfg::kKS; ++ks) {
+          const uint64_t a =
+              umma_desc_sw128(q_addr + (ks >> 2) * (Cfg::kBM * 128) + (ks & 3) * 32, 16, 1024);
+          const uint64_t bd =
+              umma_desc_sw128(kb + (ks >> 2) * ((BN / 2) * 128) + (ks & 3) * 32, 16, 1024);
+          tc_mma_ss_pair(tmem + b * BN, a, bd, kIdescS, ks > 0 ? 1u : 0u);
+        }
+        both(&s_full[b]);
+        both(&slot_empty[slot]);
+        return true;
+      };
+      auto issue_pv = [&](int j) -> bool {
+        int slot;
+        if (!take_slot(slot)) return false;
+        const int b = j & 1;
+        if (!mbar_wait_cluster(&p_full[b], (uint32_t)(j >> 1) & 1u, p.wd, kWdSoftmax)) return false;
+        tc_fence_after();
+        const uint32_t vb = slot_addr + slot * Cfg::kSlotBytes;
+#pragma unroll
+        for (int ks = 0; ks < Cfg::kPVK; ++ks) {
+          const uint64_t bd = umma_desc_sw128_mn(vb + ks * 2048, BN * 128, 1024);
+          tc_mma_ts_pair(tmem + Cfg::kOCol, tmem + b * BN + ks * 8, bd, kIdescPV,
+                         (j > 0 || ks > 0) ? 1u : 0u);
+        }
+        both(o_bar);
+        both(&slot_empty[slot]);
+        return true;
+      };
+      if (ok && nblk > 0) ok = issue_s(0);
+      if (ok && nblk > 1) ok = issue_s(1);
+      for (int j = 0; ok && j < nblk; ++j) {
+        ok = issue_pv(j);
+        if (ok && j + 2 < nblk) ok = issue_s(j + 2);
+      }
+      if (ok && nblk > 0) both(o_final);
+      both(fin_bar);
+    }
+  } else {
+    // ============ softmax warps on this CTA's 128 rows ============
+    const int quarter = warp & 3;
+    const int half = warp >> 2;
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const int pos = ((tr.row0 + r) % p.L) + p.off;
+    const float c = p.scale_log2;
+    const bool c_pos = c >= 0.f;
+    const float neutral = c_pos ? -INFINITY : INFINITY;
+    constexpr int kH = Cfg::kHalf;
+    constexpr int kOChunks = DV / 16;
+    constexpr int kOC0 = (kOChunks + 1) / 2;
+    const int oc_begin = half == 0 ? 0 : kOC0;
+    const int oc_end = half == 0 ? kOC0 : kOChunks;
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    uint32_t pair_phase = 0;
+    for (int j = 0; j < nblk; ++j) {
+      const int b = j & 1;
+      bool w = true;
+      if (lane == 0) w = mbar_wait_cluster(&s_full[b], (uint32_t)(j >> 1) & 1u, p.wd, kWdMma);
+      if (!__shfl_sync(0xffffffffu, (int)w, 0)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float s[kH];
+#pragma unroll
+      for (int c32 = 0; c32 < kH / 32; ++c32)
+        tmem_ld32(tmem + lane_base + b * BN + half * kH + c32 * 32, s + c32 * 32);
+      tmem_wait_ld();
+
+      const int kbase = k_lo + j * BN;
+      const bool masked = block_needs_mask(p, tr, kbase, BN);
+      uint64_t vis = ~0ull;
+      if (masked) {
+        vis = 0ull;
+#pragma unroll
+        for (int i = 0; i < kH; ++i) {
+          if (key_visible(p, pos, kbase + half * kH + i)) vis |= 1ull << i;
+          else s[i] = neutral;
+        }
+      }
+      float mr[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) mr[t] = s[t];
+      if (c_pos) {
+#pragma unroll
+        for (int i = 4; i < kH; i += 8) {
+          mr[0] = fmax3f(mr[0], s[i], s[i + 1]);
+          mr[1] = fmax3f(mr[1], s[i + 2], s[i + 3]);
+          if (i + 4 < kH) {
+            mr[2] = fmax3f(mr[2], s[i + 4], s[i + 5]);
+            mr[3] = fmax3f(mr[3], s[i + 6], s[i + 7]);
+          }
+        }
+        mr[0] = fmax3f(mr[0], mr[1], fmaxf(mr[2], mr[3]));
+      } else {
+#pragma unroll
+        for (int i = 4; i < kH; i += 8) {
+          mr[0] = fmin3f(mr[0], s[i], s[i + 1]);
+          mr[1] = fmin3f(mr[1], s[i + 2], s[i + 3]);
+          if (i + 4 < kH) {
+            mr[2] = fmin3f(mr[2], s[i + 4], s[i + 5]);
+            mr[3] = fmin3f(mr[3], s[i + 6], s[i + 7]);
+          }
+        }
+        mr[0] = fmin3f(mr[0], mr[1], fminf(mr[2], mr[3]));
+      }
+      xmax[((j & 1) * 2 + half) * Cfg::kBM + r] = mr[0];
+      tc_fence_before();
+      mbar_arrive(&pair_bar[quarter]);
+      if (!mbar_wait(&pair_bar[quarter], pair_phase & 1u, p.wd, kWdSoftmax)) {
+        ok = false;
+        break;
+      }
+      ++pair_phase;
+      tc_fence_after();
+      const float other = xmax[((j & 1) * 2 + (half ^ 1)) * Cfg::kBM + r];
+      const float mraw = c_pos ? fmaxf(mr[0], other) : fminf(mr[0], other);
+      const float mblk = isinf(mraw) ? -INFINITY : mraw * c;
+      const float m_new = fmaxf(m_used, mblk);
+      const bool need = m_new > m_used + 8.0f;
+      float alpha = 1.f;
+      if (need) {
+        alpha = fast_exp2(m_used - m_new);
+        m_used = m_new;
+        l *= alpha;
+      }
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+        // as in tc.cuh: S_j was issued after P_{j-2} V, and P_j V waits for
+        // p_full, so o_bar is in phase j-1 or j here
+        if (lane == 0) w = mbar_wait_cluster(o_bar, (uint32_t)(j - 1) & 1u, p.wd, kWdMma);
+        if (!__shfl_sync(0xffffffffu, (int)w, 0)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll 1
+        for (int c16 = oc_begin; c16 < oc_end; ++c16) {
+          float o[16];
+          tmem_ld16(tmem + lane_base + Cfg::kOCol + c16 * 16, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) o[e] *= alpha;
+          tmem_st16(tmem + lane_base + Cfg::kOCol + c16 * 16, o);
+        }
+        tmem_wait_st();
+      }
+      const float mref = m_used == -INFINITY ? 0.f : m_used;
+      const float2 c2 = make_float2(c, c), nm2 = make_float2(-mref, -mref);
+      float2 acc[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) acc[t] = make_float2(0.f, 0.f);
+      uint32_t pk[kH / 2];
+#pragma unroll
+      for (int i = 0; i < kH; i += 2) {
+        float2 t = fma2(make_float2(s[i], s[i + 1]), c2, nm2);
+        t.x = fast_exp2(t.x);
+        t.y = fast_exp2(t.y);
+        if (masked) {
+          t.x = ((vis >> i) & 1ull) ? t.x : 0.f;
+          t.y = ((vis >> (i + 1)) & 1ull) ? t.y : 0.f;
+        }
+        acc[(i >> 1) & 3] = add2(acc[(i >> 1) & 3], t);
+        pk[i >> 1] = pack2<kBF16>(t.x, t.y);
+      }
+      const float2 a01 = add2(acc[0], acc[1]), a23 = add2(acc[2], acc[3]);
+      const float2 at = add2(a01, a23);
+      l += at.x + at.y;
+#pragma unroll
+      for (int c16 = 0; c16 < kH / 32; ++c16)
+        tmem_st_u16x(tmem + lane_base + b * BN + half * (kH / 2) + c16 * 16, pk + c16 * 16);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&p_full[b]), 0));
+    }
+
+    // ------------------------------ epilogue ------------------------------
+    float *xl = xmax + (nblk & 1) * 2 * Cfg::kBM;
+    xl[half * Cfg::kBM + r] = l;
+    mbar_arrive(&pair_bar[quarter]);
+    if (!mbar_wait(&pair_bar[quarter], pair_phase & 1u, p.wd, kWdSoftmax)) ok = false;
+    l += xl[(half ^ 1) * Cfg::kBM + r];
+    if (ok && nblk > 0) {
+      bool w = true;
+      if (lane == 0) w = mbar_wait_cluster(o_final, 0, p.wd, kWdMma);
+      ok = __shfl_sync(0xffffffffu, (int)w, 0) != 0;
+      tc_fence_after();
+    }
+    const bool valid = r < tr.nvalid;
+    const long grow = (long)bh * p.R + tr.row0 + r;
+    const bool have_o = ok && nblk > 0;
+    float inv = l > 0.f ? 1.f / l : 0.f;
+    if (p.splits == 1) {
+      inv = finish_row(p, grow, m_used, l);
+      if (p.lse_out != nullptr && valid && half == 0) p.lse_out[grow] = row_lse(m_used, l);
+      uint8_t *orow = reinterpret_cast<uint8_t *>(p.out) + grow * p.Dv * 2;
+#pragma unroll 1
+      for (int c16 = oc_begin; c16 < oc_end; ++c16) {
+        float o[16];
+        if (have_o) {
+          tmem_ld16(tmem + lane_base + Cfg::kOCol + c16 * 16, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) o[e] = 0.f;
+        }
+        uint32_t w8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w8[e] = pack2<kBF16>(o[2 * e] * inv, o[2 * e + 1] * inv);
+        const int col = c16 * 16;
+        if (valid && col + 8 <= p.Dv)
+          *reinterpret_cast<uint4 *>(orow + col * 2) = make_uint4(w8[0], w8[1], w8[2], w8[3]);
+        if (valid && col + 16 <= p.Dv)
+          *reinterpret_cast<uint4 *>(orow + col * 2 + 16) = make_uint4(w8[4], w8[5], w8[6], w8[7]);
+      }
+    } else {
+      const long total_rows = (long)p.B * p.Hq * p.L;
+      float *po = p.part_o + ((long)split * total_rows + grow) * p.Dv;
+#pragma unroll 1
+      for (int c16 = oc_begin; c16 < oc_end; ++c16) {
+        float o[16];
+        if (have_o) {
+          tmem_ld16(tmem + lane_base + Cfg::kOCol + c16 * 16, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) o[e] = 0.f;
+        }
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const int col = c16 * 16 + q4 * 4;
+          if (valid && col + 4 <= p.Dv)
+            *reinterpret_cast<float4 *>(po + col) =
+                make_float4(o[q4 * 4] * inv, o[q4 * 4 + 1] * inv, o[q4 * 4 + 2] * inv,
+                            o[q4 * 4 + 3] * inv);
+        }
+      }
+      if (valid && half == 0)
+        p.part_lse[(long)split * total_rows + grow] = have_o ? row_lse(m_used, l) : -INFINITY;
+    }
+  }
+
+  // ------------------------------ teardown ------------------------------
+  // Neither CTA may exit while the other can still reach its shared memory:
+  // the even CTA's MMAs read the odd CTA's tiles (done once fin_bar fires in
+  // both), and the odd CTA arrives on the even CTA's barriers.  Each CTA
+  // signals the other's bye_bar after that and waits for its own, bounded.
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_wait_cluster_drain(fin_bar, 0, p.wd);
+    mbar_arrive_cluster(mapa_shared(smem_u32(bye_bar), rank ^ 1u));
+    mbar_wait_cluster_drain(bye_bar, 0, p.wd);
+  }
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, Cfg::kTmemCols);
+  }
+}
+
+}  // namespace sdpa

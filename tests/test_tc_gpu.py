@@ -35,6 +35,15 @@ def test_tc_vs_oracle(cuda_lib, case):
     assert info["path"] == S.PATH_TC
 
 
+@pytest.mark.parametrize("scale", [-0.09, 0.0, 0.5])
+@pytest.mark.parametrize("path", [S.PATH_TC, S.PATH_SPLITKV])
+def test_unusual_scales(cuda_lib, scale, path):
+    # a negative scale flips which score is the row max; zero gives uniform
+    # weights over the visible keys
+    p = I.Problem(1, 4, 2, 150, 260, 128, 128, "bf16", True, 30, scale, 24, "scales")
+    check_problem(cuda_lib, p, force_path=path)
+
+
 @pytest.mark.parametrize("splits", [2, 5, 0])
 def test_tc_with_key_splits(cuda_lib, splits):
     p = I.Problem(1, 8, 2, 64, 3000, 128, 128, "bf16", True, 0, None, 22, "tc_split")
