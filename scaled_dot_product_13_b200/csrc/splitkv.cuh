@@ -395,11 +395,27 @@ __global__ void __launch_bounds__(128) combine_kernel(const float *__restrict__ 
                                                       int Hq) {
   extern __shared__ float s_w[];  // [splits]
   __shared__ float s_red[4];
+  constexpr int kPre = 16;        // splits whose partials are loaded before the weights exist
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const long row = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const long stride = total_rows * Dv;
+  const int d0 = tid, d1 = tid + 128;  // this thread's output columns (Dv <= 256)
+  const float *src0 = part_o + row * Dv + d0;
+  const float *src1 = part_o + row * Dv + d1;
+  // issue the partial loads first so they are in flight with the LSE loads
+  float v0[kPre], v1[kPre];
+#pragma unroll
+  for (int t = 0; t < kPre; ++t) {
+    v0[t] = (t < splits && d0 < Dv) ? __ldcg(src0 + (long)t * stride) : 0.f;
+    v1[t] = (t < splits && d1 < Dv) ? __ldcg(src1 + (long)t * stride) : 0.f;
+  }
   float mx = -INFINITY;
-  for (int s = tid; s < splits; s += 128) mx = fmaxf(mx, __ldcg(part_lse + (long)s * total_rows + row));
+  for (int s = tid; s < splits; s += 128) {
+    const float x = __ldcg(part_lse + (long)s * total_rows + row);
+    s_w[s] = x;
+    mx = fmaxf(mx, x);
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   if (lane == 0) s_red[wid] = mx;
@@ -411,37 +427,38 @@ __global__ void __launch_bounds__(128) combine_kernel(const float *__restrict__ 
   __syncthreads();
   float den = 0.f;
   for (int s = tid; s < splits; s += 128) {
-    const float w = __expf(__ldcg(part_lse + (long)s * total_rows + row) - ref);
+    const float w = __expf(s_w[s] - ref);
     s_w[s] = w;
     den += w;
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+  __syncthreads();  // s_red reuse and the weights in s_w
   if (lane == 0) s_red[wid] = den;
   __syncthreads();
   den = s_red[0] + s_red[1] + s_red[2] + s_red[3] + (sinks != nullptr ? __expf(sink - ref) : 0.f);
   const float inv = den > 0.f ? 1.f / den : 0.f;
-  const long stride = total_rows * Dv;
-  for (int d = tid; d < Dv; d += 128) {
-    const float *src = part_o + row * Dv + d;
-    float acc[8];
+  float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-    for (int t = 0; t < 8; ++t) acc[t] = 0.f;
-    int s = 0;
-    for (; s + 8 <= splits; s += 8) {
-      float v[8];
-#pragma unroll
-      for (int t = 0; t < 8; ++t) v[t] = __ldcg(src + (long)(s + t) * stride);
-#pragma unroll
-      for (int t = 0; t < 8; ++t) acc[t] += s_w[s + t] * v[t];
+  for (int t = 0; t < kPre; ++t) {
+    if (t < splits) {
+      a0 += s_w[t] * v0[t];
+      a1 += s_w[t] * v1[t];
     }
-    for (; s < splits; ++s) acc[s & 7] += s_w[s] * __ldcg(src + (long)s * stride);
-    const float res =
-        (((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]))) * inv;
-    if constexpr (kBF16)
-      reinterpret_cast<__nv_bfloat16 *>(out)[row * Dv + d] = __float2bfloat16_rn(res);
-    else
-      reinterpret_cast<__half *>(out)[row * Dv + d] = __float2half_rn(res);
+  }
+  for (int s = kPre; s < splits; ++s) {
+    const float w = s_w[s];
+    if (d0 < Dv) a0 += w * __ldcg(src0 + (long)s * stride);
+    if (d1 < Dv) a1 += w * __ldcg(src1 + (long)s * stride);
+  }
+  if constexpr (kBF16) {
+    __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(out) + row * Dv;
+    if (d0 < Dv) o[d0] = __float2bfloat16_rn(a0 * inv);
+    if (d1 < Dv) o[d1] = __float2bfloat16_rn(a1 * inv);
+  } else {
+    __half *o = reinterpret_cast<__half *>(out) + row * Dv;
+    if (d0 < Dv) o[d0] = __float2half_rn(a0 * inv);
+    if (d1 < Dv) o[d1] = __float2half_rn(a1 * inv);
   }
   if (lse_out != nullptr && tid == 0) lse_out[row] = den > 0.f ? ref + logf(den) : -INFINITY;
 }
