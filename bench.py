@@ -171,57 +171,67 @@ class HostCase:
 
 
 def time_cases(sdpa, cases, steps, warmup, flush, sync_all, graphs=True):
-    """Per call: flush L2 (untimed), then run the call with three CUDA events
-    recorded by the library on its launch stream: before the main kernel,
-    after it, and after the call's last launch (the combine, when split).
-    call time = first to last event (the device time of the library's work);
-    main time = the main kernel alone.  With ``graphs`` each call is captured
-    once into a CUDA graph and replayed, so the device timeline carries no
-    host enqueue gaps.  Returns per-case lists (ms): call, main, outer (the
-    replay including graph-launch edges)."""
+    """Per call: flush L2 (untimed), then run the call with CUDA events
+    recorded by the library on its launch stream.
+
+    Two interleaved runners per call.  The timed one records an event before
+    the main kernel and one after the call's last launch (the combine, when
+    split): call time = the device time of the library's work.  Nothing sits
+    between the split pass and the combine there, so the combine keeps its
+    programmatic (early) launch.  The second runner adds an event right after
+    the main kernel, which serialises the combine behind it; it only gives the
+    main kernel's own time for the roofline.  With ``graphs`` each runner is
+    captured once into a CUDA graph and replayed, so the device timeline
+    carries no host enqueue gaps.  Returns per-case lists (ms): call, main,
+    outer (the timed replay including graph-launch edges)."""
     call_ms = [[] for _ in cases]
     main_ms = [[] for _ in cases]
     outer_ms = [[] for _ in cases]
     stream = torch.cuda.current_stream()
     hooks = []
     for c in cases:
-        evs = tuple(torch.cuda.Event(enable_timing=True) for _ in range(3))
+        evs = tuple(torch.cuda.Event(enable_timing=True) for _ in range(5))
         for e in evs:
             e.record(stream)  # creates the CUDA handles; the library re-records them
         c.call(sdpa)  # first call outside any capture (kernel attributes, TMA encode path)
         hooks.append(evs)
     torch.cuda.synchronize()
-    runners = []
-    for c, (m0, m1, m2) in zip(cases, hooks):
+
+    def runner(c, a, b, d):
         if graphs:
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g):
-                sdpa.time_next_call(m0, m1, m2)
+                sdpa.time_next_call(a, b, d)
                 c.call(sdpa)
-            runners.append(g.replay)
-        else:
-            def eager(c=c, m0=m0, m1=m1, m2=m2):
-                sdpa.time_next_call(m0, m1, m2)
-                c.call(sdpa)
-            runners.append(eager)
+            return g.replay
+
+        def eager():
+            sdpa.time_next_call(a, b, d)
+            c.call(sdpa)
+        return eager
+
+    timed = [runner(c, h[0], None, h[1]) for c, h in zip(cases, hooks)]
+    probes = [runner(c, h[2], h[3], h[4]) for c, h in zip(cases, hooks)]
     torch.cuda.synchronize()
     for it in range(warmup + steps):
         evs = []
-        for run in runners:
+        for run, probe in zip(timed, probes):
             flush_l2(flush)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             run()
             e1.record(stream)
             evs.append((e0, e1))
+            flush_l2(flush)
+            probe()
         if it == warmup - 1:
             sync_all()
         if it >= warmup:
             torch.cuda.synchronize()
             for i, (e0, e1) in enumerate(evs):
-                m0, m1, m2 = hooks[i]
-                call_ms[i].append(m0.elapsed_time(m2))
-                main_ms[i].append(m0.elapsed_time(m1))
+                h = hooks[i]
+                call_ms[i].append(h[0].elapsed_time(h[1]))
+                main_ms[i].append(h[2].elapsed_time(h[3]))
                 outer_ms[i].append(e0.elapsed_time(e1))
     return call_ms, main_ms, outer_ms
 
@@ -333,7 +343,8 @@ def main():
     probs = I.decode_problems()
     if args.only:
         probs = [p for p in probs + I.verify_problems() + I.window_problems() +
-                 I.encoder_problems() + [I.tiny_problem()] if p.name == args.only]
+                 I.encoder_problems() + [I.tiny_problem()] + I.wide_problems()
+                 if p.name == args.only]
         if not probs:
             raise SystemExit(f"unknown problem {args.only}")
     peaks, peak_src = load_peaks()
@@ -341,6 +352,8 @@ def main():
                             "S in {256,1024,4096,8192,16384,32768}, Dqk=192, Dv=128, bf16, causal",
                 "calls_per_step": len(probs), "l2": "flushed before every call (2x L2 buffer written, then read)",
                 "launch": "eager" if args.eager else "one CUDA graph per call (split pass + combine), replayed",
+                "timing": "call = library events before the split pass and after the combine; "
+                          "main-kernel time from separate probe replays with an event after the split pass",
                 "parallelism": f"replicas x{world} (independent KV-head units, no collective)"}
 
     if args.impl == "reference":
@@ -440,6 +453,8 @@ def main():
         extra["verify"] = secondary(sdpa, I.verify_problems(), sec_steps, 3, flush, sync_all,
                                     device, peaks, "tflops", gr)
         extra["tiny"] = secondary(sdpa, [I.tiny_problem()], sec_steps, 3, flush, sync_all,
+                                  device, peaks, "tflops", gr)
+        extra["wide"] = secondary(sdpa, I.wide_problems(), sec_steps, 3, flush, sync_all,
                                   device, peaks, "tflops", gr)
 
     line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s (KV, decode)",

@@ -15,7 +15,8 @@
  *     kb_start / kb_lim, left-edge rule row - col >= W masked);
  *   - asymmetric head dims Dqk != Dv, e.g. 192/128 (mlx PR #3637);
  *   - head dims outside the usual fused sets: 72, 192, 256 (mlx-rs issue
- *     #339 finding 1; mlx PR #4185 "Kernel support");
+ *     #339 finding 1; mlx PR #4185 "Kernel support"), and 512, where the
+ *     pages' kernels stop (mlx PR #4185, "Kernel support");
  *   - decode and short "verify" queries processed as a split over the keys
  *     with a log-sum-exp merge, so the work stays parallel over S
  *     (mlx issue #3826, routing analysis and the 2-pass extension);
@@ -88,9 +89,14 @@ typedef enum {
                             log-sum-exp combine when split                   */
   SDPA_PATH_TC = 2,      /* 128-row tiles on tcgen05 with TMEM accumulators,
                             TMA-staged K/V, optional key splits + combine    */
-  SDPA_PATH_TC2 = 3      /* 256-row tiles on a pair of SMs (tcgen05
+  SDPA_PATH_TC2 = 3,     /* 256-row tiles on a pair of SMs (tcgen05
                             cta_group::2): each SM loads half of every K/V
-                            block; head dims 256/256 and 192/128             */
+                            block; head dims 256/256, 192/128 (routed) and
+                            128/128 (on request)                             */
+  SDPA_PATH_WIDE = 4     /* head dims above 256 (up to 512): 16-row groups
+                            whose four warps split the output columns, key
+                            splits + combine as on SDPA_PATH_SPLITKV; the
+                            only path for those head dims                    */
 } sdpa_path;
 
 /*
@@ -108,8 +114,8 @@ typedef enum {
  *                         Hq not a multiple of Hkv; causal with L > S (no key
  *                         would be visible to the first rows); window_size <
  *                         0; a non-finite scale; out overlapping an input.
- *   SDPA_ERR_UNSUPPORTED  Dqk or Dv not a multiple of 8 or above 256 (for
- *                         example 512); an unknown dtype; window_size > 0
+ *   SDPA_ERR_UNSUPPORTED  Dqk or Dv not a multiple of 8 or above 512 (for
+ *                         example 576); an unknown dtype; window_size > 0
  *                         with causal = 0; sizes whose element offsets
  *                         exceed 2^31 rows of 2^31 bytes.
  *   SDPA_ERR_CUDA         no usable CUDA device, or a launch failed.

@@ -20,12 +20,13 @@ import os
 
 __all__ = ["forward", "forward_ws", "forward_noalloc", "forward_ex", "Options", "workspace_bytes", "plan", "device_status",
            "set_wait_limit_ns", "watchdog_selftest", "time_next_main_kernel", "time_next_call", "load_library", "library_path",
-           "SdpaError", "PATH_AUTO", "PATH_SPLITKV", "PATH_TC", "PATH_TC2", "STATUS"]
+           "SdpaError", "PATH_AUTO", "PATH_SPLITKV", "PATH_TC", "PATH_TC2", "PATH_WIDE",
+           "STATUS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB: ctypes.CDLL | None = None
 
-PATH_AUTO, PATH_SPLITKV, PATH_TC, PATH_TC2 = 0, 1, 2, 3
+PATH_AUTO, PATH_SPLITKV, PATH_TC, PATH_TC2, PATH_WIDE = 0, 1, 2, 3, 4
 STATUS = {0: "SDPA_OK", 1: "SDPA_ERR_INVALID_ARG", 2: "SDPA_ERR_UNSUPPORTED",
           3: "SDPA_ERR_RESOURCES", 4: "SDPA_ERR_CUDA", 5: "SDPA_ERR_TIMEOUT"}
 
@@ -285,13 +286,14 @@ def time_next_main_kernel(start_event, stop_event) -> None:
 
 def time_next_call(start_event, stop_event, call_event) -> None:
     """As ``time_next_main_kernel``, plus ``call_event`` recorded after the
-    call's last launch (the combine, when the keys are split)."""
+    call's last launch (the combine, when the keys are split).  Any of the
+    three may be None (not recorded)."""
+    handles = []
     for e in (start_event, stop_event, call_event):
-        if not e.cuda_event:
+        if e is not None and not e.cuda_event:
             raise SdpaError(1, "events have no CUDA handle yet; record them once first")
-    load_library().sdpa_time_next_call(ctypes.c_void_p(start_event.cuda_event),
-                                       ctypes.c_void_p(stop_event.cuda_event),
-                                       ctypes.c_void_p(call_event.cuda_event))
+        handles.append(ctypes.c_void_p(e.cuda_event if e is not None else None))
+    load_library().sdpa_time_next_call(*handles)
 
 
 def set_wait_limit_ns(ns: int) -> None:

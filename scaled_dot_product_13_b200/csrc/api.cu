@@ -104,9 +104,9 @@ sdpa_status validate_shape(const Problem &p) {
   if (!std::isfinite(p.scale))
     return fail(SDPA_ERR_INVALID_ARG, "scale must be finite");
   for (int d : {p.Dqk, p.Dv}) {
-    if (d < 8 || d > 256 || d % 8 != 0)
+    if (d < 8 || d > 512 || d % 8 != 0)
       return fail(SDPA_ERR_UNSUPPORTED,
-                  "head dims must be multiples of 8 in [8, 256] (got Dqk=%d, Dv=%d)", p.Dqk,
+                  "head dims must be multiples of 8 in [8, 512] (got Dqk=%d, Dv=%d)", p.Dqk,
                   p.Dv);
   }
   const long long rows = (long long)p.B * p.Hq * p.L;
@@ -157,6 +157,7 @@ constexpr int kTc2RowThreshold = 256;
 // kNoSplitBlocks key blocks are not split: below that the combine launch
 // costs more than the parallelism gains.
 constexpr int kMinBlocksPerSplit = 2;
+constexpr int kMinBlocksPerSplitWide = 8;
 constexpr int kNoSplitBlocks = 4;
 
 sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_splits,
@@ -167,8 +168,15 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
   if (pl.pair < 0)
     return fail(SDPA_ERR_UNSUPPORTED, "no kernel instance covers Dqk=%d, Dv=%d", pb.Dqk, pb.Dv);
   if (force_path != SDPA_PATH_AUTO && force_path != SDPA_PATH_SPLITKV &&
-      force_path != SDPA_PATH_TC && force_path != SDPA_PATH_TC2)
+      force_path != SDPA_PATH_TC && force_path != SDPA_PATH_TC2 && force_path != SDPA_PATH_WIDE)
     return fail(SDPA_ERR_INVALID_ARG, "unknown path %d", force_path);
+  // head dims above 256 run only on the column-split kernel, and it only on them
+  const bool wide = pl.pair == kWidePair;
+  if (force_path != SDPA_PATH_AUTO && (force_path == SDPA_PATH_WIDE) != wide)
+    return fail(SDPA_ERR_UNSUPPORTED,
+                wide ? "head dims above 256 (got Dqk=%d, Dv=%d) run only on the wide path"
+                     : "the wide path is built for head dims above 256 (got Dqk=%d, Dv=%d)",
+                pb.Dqk, pb.Dv);
   if (force_splits < 0) return fail(SDPA_ERR_INVALID_ARG, "force_splits must be >= 0");
   if (num_sms < 1) num_sms = 148;
   const int g = pb.Hq / pb.Hkv;
@@ -179,18 +187,33 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
   // split-KV kernel on 16-row warp tiles.  Both split the keys when the
   // tiles alone do not fill the GPU.
   int path = force_path;
+  if (path == SDPA_PATH_AUTO && wide) path = SDPA_PATH_WIDE;
   if (path == SDPA_PATH_AUTO) {
     path = pl.rows >= kTcRowThreshold ? SDPA_PATH_TC : SDPA_PATH_SPLITKV;
     // wide heads with at least one full 256-row pair tile: two SMs per tile
-    if (path == SDPA_PATH_TC && tc2_supports_pair(pl.pair) && pl.rows >= kTc2RowThreshold)
+    if (path == SDPA_PATH_TC && tc2_preferred_pair(pl.pair) && pl.rows >= kTc2RowThreshold)
       path = SDPA_PATH_TC2;
+  }
+  if (path == SDPA_PATH_TC2 && !tc2_supports_pair(pl.pair)) {
+    // the smallest two-CTA instance that covers the head dims (zero filled)
+    for (int i = pl.pair + 1; i < kNumDimPairs; ++i)
+      if (tc2_supports_pair(i) && kDimPairs[i].dqk >= pb.Dqk && kDimPairs[i].dv >= pb.Dv) {
+        pl.pair = i;
+        break;
+      }
   }
   if (path == SDPA_PATH_TC2 && !tc2_supports_pair(pl.pair))
     return fail(SDPA_ERR_UNSUPPORTED,
-                "the two-CTA path is built for head dims 256/256 and 192/128 (got %d/%d)",
+                "the two-CTA path is built for head dims 256/256, 192/128 and 128/128 (got %d/%d)",
                 pb.Dqk, pb.Dv);
   pl.path = path;
-  if (path == SDPA_PATH_TC2) {
+  if (path == SDPA_PATH_WIDE) {
+    // one 16-row group (four warps) for decode-sized problems, two otherwise
+    pl.wr = pl.rows <= 16 ? 1 : 2;
+    pl.wk = 0;
+    pl.row_tile = 16 * pl.wr;
+    pl.key_block = kWideBN;
+  } else if (path == SDPA_PATH_TC2) {
     pl.wr = 0; pl.wk = 0;
     pl.row_tile = 2 * kTcRows;
     pl.key_block = 128;
@@ -226,8 +249,11 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
   } else if (base >= num_sms || nkb <= kNoSplitBlocks) {
     splits = 1;
   } else {
+    // the wide kernel's 32-key blocks are small and its partials wide
+    // (Dv up to 512 floats per row and split): give each split more keys
+    const int min_blocks = path == SDPA_PATH_WIDE ? kMinBlocksPerSplitWide : kMinBlocksPerSplit;
     splits = (int)std::max(1LL, num_sms / base);
-    splits = std::min(splits, std::max(1, nkb / kMinBlocksPerSplit));
+    splits = std::min(splits, std::max(1, nkb / min_blocks));
   }
   splits = std::min(splits, kMaxSplits);
   const int bps = (nkb + splits - 1) / splits;
@@ -366,9 +392,10 @@ sdpa_status forward_call(const Problem &pb, const void *q, const void *k, const 
   ln.ev_stop = t_ev_stop;
   cudaEvent_t ev_call = t_ev_call;
   t_ev_start = t_ev_stop = t_ev_call = nullptr;
-  st = pl.path == SDPA_PATH_TC2  ? launch_tc2(ln, &err)
-       : pl.path == SDPA_PATH_TC ? launch_tc(ln, &err)
-                                 : launch_splitkv(ln, &err);
+  st = pl.path == SDPA_PATH_TC2    ? launch_tc2(ln, &err)
+       : pl.path == SDPA_PATH_TC   ? launch_tc(ln, &err)
+       : pl.path == SDPA_PATH_WIDE ? launch_wide(ln, &err)
+                                   : launch_splitkv(ln, &err);
   if (st == SDPA_OK && pl.splits > 1) st = launch_combine(ln, &err);
   if (st == SDPA_OK && ev_call) record_event(ev_call, stream);
   if (allocated) {

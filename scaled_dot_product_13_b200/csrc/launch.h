@@ -18,9 +18,14 @@ namespace sdpa {
 struct DimPair {
   int dqk, dv;
 };
-constexpr DimPair kDimPairs[] = {{64, 64},   {80, 80},   {128, 128},
-                                 {192, 128}, {192, 192}, {256, 256}};
+constexpr DimPair kDimPairs[] = {{64, 64},   {80, 80},   {128, 128}, {192, 128},
+                                 {192, 192}, {256, 256}, {512, 512}};
 constexpr int kNumDimPairs = sizeof(kDimPairs) / sizeof(kDimPairs[0]);
+// The 512/512 pair is built only for the wide (column-split) kernel.
+constexpr int kWidePair = 6;
+
+// Key block of the wide kernel.
+constexpr int kWideBN = 32;
 
 // Key block of the split-KV kernel (keys per pipeline stage).
 constexpr int kSplitKvBN = 64;
@@ -42,10 +47,10 @@ struct Problem {
 };
 
 struct Plan {
-  int path;            // SDPA_PATH_SPLITKV or SDPA_PATH_TC
+  int path;            // SDPA_PATH_SPLITKV, _TC, _TC2 or _WIDE
   int pair;            // index into kDimPairs
   int rows;            // g * L
-  int wr, wk;          // split-KV warp layout (rows x key slices)
+  int wr, wk;          // split-KV warp layout (rows x key slices); wide: row groups
   int row_tile;
   int row_tiles;
   int key_block;
@@ -96,9 +101,13 @@ bool encode_tma(CUtensorMap *map, sdpa_dtype dt, int rank, const void *base,
 sdpa_status launch_splitkv(const Launch &ln, std::string *err);
 sdpa_status launch_tc(const Launch &ln, std::string *err);
 sdpa_status launch_tc2(const Launch &ln, std::string *err);
+sdpa_status launch_wide(const Launch &ln, std::string *err);
 
-// Head-dim pairs the two-CTA kernel is built for (index into kDimPairs).
-constexpr bool tc2_supports_pair(int pair) { return pair == 3 || pair == 5; }
+// Head-dim pairs the two-CTA kernel is built for (index into kDimPairs), and
+// those the router sends to it by itself (where it measured faster than one
+// SM per 128-row tile).
+constexpr bool tc2_supports_pair(int pair) { return pair == 2 || pair == 3 || pair == 5; }
+constexpr bool tc2_preferred_pair(int pair) { return pair == 3 || pair == 5; }
 sdpa_status launch_combine(const Launch &ln, std::string *err);
 
 // Record a timing event on `stream`.  Inside stream capture a plain

@@ -119,15 +119,12 @@ sdpa_status launch_combine(const Launch &ln, std::string *err) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e;
-  if (ln.pb.dtype == SDPA_BF16)
-    e = cudaLaunchKernelEx(&cfg, combine_kernel<true>, (const float *)ln.part_o,
-                           (const float *)ln.part_lse, ln.out, ln.lse_out, ln.sinks, total,
-                           ln.pb.Dv, ln.plan.splits, ln.pb.L, ln.pb.Hq);
-  else
-    e = cudaLaunchKernelEx(&cfg, combine_kernel<false>, (const float *)ln.part_o,
-                           (const float *)ln.part_lse, ln.out, ln.lse_out, ln.sinks, total,
-                           ln.pb.Dv, ln.plan.splits, ln.pb.L, ln.pb.Hq);
+  const bool bf16 = ln.pb.dtype == SDPA_BF16, four = ln.pb.Dv > 256;
+  auto kern = bf16 ? (four ? combine_kernel<true, 4> : combine_kernel<true, 2>)
+                   : (four ? combine_kernel<false, 4> : combine_kernel<false, 2>);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, (const float *)ln.part_o,
+                                     (const float *)ln.part_lse, ln.out, ln.lse_out, ln.sinks,
+                                     total, ln.pb.Dv, ln.plan.splits, ln.pb.L, ln.pb.Hq);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) {
     *err = std::string("combine_kernel launch failed: ") + cudaGetErrorString(e);

@@ -89,6 +89,7 @@ sdpa_status run_tc2(const Launch &ln, std::string *err) {
 template <bool kBF16>
 sdpa_status run_dtype(const Launch &ln, std::string *err) {
   switch (ln.plan.pair) {
+    case 2: return run_tc2<kBF16, 128, 128>(ln, err);
     case 3: return run_tc2<kBF16, 192, 128>(ln, err);
     case 5: return run_tc2<kBF16, 256, 256>(ln, err);
   }

@@ -376,7 +376,7 @@ __global__ void __launch_bounds__(SplitKvCfg<DQK, DV, BN, WR, WK, NST>::kThreads
 // ---------------------------------------------------------------------------
 // Log-sum-exp combine of split partials (mlx issue #3826: split over S, then
 // a log-sum-exp merge; mlx PR #3637: the 2-pass kernel's aggregation).
-// One CTA of 128 threads per output row:
+// One CTA of 128 threads per output row (NC output columns per thread):
 //   LSE = max_s LSE_s + ln sum_s exp(LSE_s - max),  O = sum_s exp(LSE_s - LSE) O_s
 // Splits that saw no visible key carry LSE_s = -inf and weight 0.  A head's
 // sink (when given) joins as one more term with weight exp(sink - LSE) and
@@ -386,7 +386,7 @@ __global__ void __launch_bounds__(SplitKvCfg<DQK, DV, BN, WR, WK, NST>::kThreads
 // Launched as a programmatic dependent of the split pass: it waits for that
 // grid (griddepcontrol.wait) before touching the partials.
 // ---------------------------------------------------------------------------
-template <bool kBF16>
+template <bool kBF16, int NC>
 __global__ void __launch_bounds__(128) combine_kernel(const float *__restrict__ part_o,
                                                       const float *__restrict__ part_lse,
                                                       void *__restrict__ out, float *lse_out,
@@ -400,16 +400,15 @@ __global__ void __launch_bounds__(128) combine_kernel(const float *__restrict__ 
   const long row = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const long stride = total_rows * Dv;
-  const int d0 = tid, d1 = tid + 128;  // this thread's output columns (Dv <= 256)
-  const float *src0 = part_o + row * Dv + d0;
-  const float *src1 = part_o + row * Dv + d1;
+  // this thread's output columns: tid + 128 c for c < NC (Dv <= 128 NC)
+  const float *src = part_o + row * Dv + tid;
   // issue the partial loads first so they are in flight with the LSE loads
-  float v0[kPre], v1[kPre];
+  float v[kPre][NC];
 #pragma unroll
-  for (int t = 0; t < kPre; ++t) {
-    v0[t] = (t < splits && d0 < Dv) ? __ldcg(src0 + (long)t * stride) : 0.f;
-    v1[t] = (t < splits && d1 < Dv) ? __ldcg(src1 + (long)t * stride) : 0.f;
-  }
+  for (int t = 0; t < kPre; ++t)
+#pragma unroll
+    for (int c = 0; c < NC; ++c)
+      v[t][c] = (t < splits && tid + 128 * c < Dv) ? __ldcg(src + (long)t * stride + 128 * c) : 0.f;
   float mx = -INFINITY;
   for (int s = tid; s < splits; s += 128) {
     const float x = __ldcg(part_lse + (long)s * total_rows + row);
@@ -438,27 +437,42 @@ __global__ void __launch_bounds__(128) combine_kernel(const float *__restrict__ 
   __syncthreads();
   den = s_red[0] + s_red[1] + s_red[2] + s_red[3] + (sinks != nullptr ? __expf(sink - ref) : 0.f);
   const float inv = den > 0.f ? 1.f / den : 0.f;
-  float a0 = 0.f, a1 = 0.f;
+  float acc[NC];
+#pragma unroll
+  for (int c = 0; c < NC; ++c) acc[c] = 0.f;
 #pragma unroll
   for (int t = 0; t < kPre; ++t) {
     if (t < splits) {
-      a0 += s_w[t] * v0[t];
-      a1 += s_w[t] * v1[t];
+#pragma unroll
+      for (int c = 0; c < NC; ++c) acc[c] += s_w[t] * v[t][c];
     }
   }
-  for (int s = kPre; s < splits; ++s) {
-    const float w = s_w[s];
-    if (d0 < Dv) a0 += w * __ldcg(src0 + (long)s * stride);
-    if (d1 < Dv) a1 += w * __ldcg(src1 + (long)s * stride);
+  // the remaining splits, kBatch per round trip to L2
+  constexpr int kBatch = 8;
+  for (int s0 = kPre; s0 < splits; s0 += kBatch) {
+    float x[kBatch][NC];
+#pragma unroll
+    for (int t = 0; t < kBatch; ++t)
+#pragma unroll
+      for (int c = 0; c < NC; ++c)
+        x[t][c] = (s0 + t < splits && tid + 128 * c < Dv)
+                      ? __ldcg(src + (long)(s0 + t) * stride + 128 * c)
+                      : 0.f;
+#pragma unroll
+    for (int t = 0; t < kBatch; ++t) {
+      const float w = s0 + t < splits ? s_w[s0 + t] : 0.f;
+#pragma unroll
+      for (int c = 0; c < NC; ++c) acc[c] += w * x[t][c];
+    }
   }
-  if constexpr (kBF16) {
-    __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(out) + row * Dv;
-    if (d0 < Dv) o[d0] = __float2bfloat16_rn(a0 * inv);
-    if (d1 < Dv) o[d1] = __float2bfloat16_rn(a1 * inv);
-  } else {
-    __half *o = reinterpret_cast<__half *>(out) + row * Dv;
-    if (d0 < Dv) o[d0] = __float2half_rn(a0 * inv);
-    if (d1 < Dv) o[d1] = __float2half_rn(a1 * inv);
+#pragma unroll
+  for (int c = 0; c < NC; ++c) {
+    const int d = tid + 128 * c;
+    if (d >= Dv) continue;
+    if constexpr (kBF16)
+      reinterpret_cast<__nv_bfloat16 *>(out)[row * Dv + d] = __float2bfloat16_rn(acc[c] * inv);
+    else
+      reinterpret_cast<__half *>(out)[row * Dv + d] = __float2half_rn(acc[c] * inv);
   }
   if (lse_out != nullptr && tid == 0) lse_out[row] = den > 0.f ? ref + logf(den) : -INFINITY;
 }

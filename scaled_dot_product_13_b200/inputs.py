@@ -132,5 +132,18 @@ def window_problems(include_32k: bool = True):
     return out
 
 
+def wide_problems():
+    """Head dim 512: decode (16 query heads on one KV head) at 8K and 32K keys,
+    and a causal prefill of 4096 tokens over 8 heads.  The pages name head dim
+    512 as the case their fused kernels do not cover; no page measures it, so
+    these shapes extend the decode and prefill workloads above."""
+    out = [Problem(1, 16, 1, 1, s, 512, 512, "bf16", True, 0, None, 5, f"wide_decode_d512_s{s}")
+           for s in (8192, 32768)]
+    out.append(Problem(1, 8, 8, 4096, 4096, 512, 512, "bf16", True, 0, None, 5,
+                       "wide_prefill_d512_l4096"))
+    return out
+
+
 __all__ = ["Problem", "make_qkv", "sample_rows", "tiny_problem", "decode_problems",
-           "verify_problems", "encoder_problems", "window_problems", "DECODE_S", "VERIFY_L"]
+           "verify_problems", "encoder_problems", "window_problems", "wide_problems",
+           "DECODE_S", "VERIFY_L"]

@@ -53,7 +53,8 @@ def _plan_err(**kw):
     (dict(L=65, S=64), 1, "L <= S"),
     (dict(window_size=-1), 1, "window_size"),
     (dict(window_size=8, causal=False), 2, "causal"),
-    (dict(Dqk=512, Dv=512), 2, "head dims"),
+    (dict(Dqk=576, Dv=512), 2, "head dims"),
+    (dict(Dqk=512, Dv=520), 2, "[8, 512]"),
     (dict(Dqk=72, Dv=100), 2, "multiples of 8"),
     (dict(B=0), 1, ">= 1"),
     (dict(S=0), 1, ">= 1"),
@@ -142,3 +143,24 @@ def test_forward_without_device_fails_loudly(lib):
                           0, None)
     assert st == 4
     assert b"CUDA" in lib.sdpa_last_error_message() or b"device" in lib.sdpa_last_error_message()
+
+
+def test_plan_head_dims_above_256_take_the_wide_path():
+    # decode at head dim 512: one 16-row group, keys split over the SMs
+    info = sdpa.plan(1, 16, 1, 1, 8192, 512, 512, causal=True, num_sms=148)
+    assert info["path"] == sdpa.PATH_WIDE and (info["dqk_pad"], info["dv_pad"]) == (512, 512)
+    assert info["row_tile"] == 16 and info["key_block"] == 32 and info["splits"] > 1
+    # prefill: two 16-row groups per CTA
+    info = sdpa.plan(1, 8, 8, 1024, 1024, 512, 512, causal=True, num_sms=148)
+    assert info["path"] == sdpa.PATH_WIDE and info["row_tile"] == 32
+    # mixed dims above 256 run on the 512/512 instance
+    assert sdpa.plan(1, 4, 4, 64, 64, 320, 128, num_sms=148)["path"] == sdpa.PATH_WIDE
+    assert sdpa.plan(1, 4, 4, 64, 64, 128, 384, num_sms=148)["path"] == sdpa.PATH_WIDE
+    # no other path takes them, and the wide path takes nothing else
+    for path in (sdpa.PATH_SPLITKV, sdpa.PATH_TC, sdpa.PATH_TC2):
+        with pytest.raises(sdpa.SdpaError) as ei:
+            sdpa.plan(1, 4, 4, 64, 64, 512, 512, num_sms=148, force_path=path)
+        assert ei.value.status == 2 and "wide" in ei.value.message
+    with pytest.raises(sdpa.SdpaError) as ei:
+        sdpa.plan(1, 4, 4, 64, 64, 256, 256, num_sms=148, force_path=sdpa.PATH_WIDE)
+    assert ei.value.status == 2

@@ -100,7 +100,7 @@ def test_errors_raise_before_launch(cuda_lib):
     with pytest.raises(cuda_lib.SdpaError) as ei:
         cuda_lib.forward(q, k, k, causal=True)
     assert "L <= S" in ei.value.message
-    big = torch.zeros(1, 4, 8, 512, dtype=torch.bfloat16, device="cuda")
+    big = torch.zeros(1, 4, 8, 576, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(cuda_lib.SdpaError) as ei:
         cuda_lib.forward(big, big, big)
     assert ei.value.status == 2

@@ -24,6 +24,10 @@ CASES = [
     ("d192_128_f16", 2, 2, 2, 400, 400, 192, 128, "f16", False, 0),
     ("d256_small_pair_rows", 1, 1, 1, 64, 64, 256, 256, "bf16", True, 0),
     ("d256_window_1", 1, 2, 1, 260, 260, 256, 256, "bf16", True, 1),
+    ("d128_causal", 1, 4, 2, 600, 600, 128, 128, "bf16", True, 0),
+    ("d128_f16_window", 2, 4, 4, 300, 450, 128, 128, "f16", True, 77),
+    ("d64_padded", 1, 4, 4, 512, 512, 64, 64, "bf16", False, 0),
+    ("d72_padded", 1, 2, 2, 700, 700, 72, 72, "bf16", False, 0),
 ]
 
 
@@ -68,3 +72,25 @@ def test_tc2_agrees_with_tc(cuda_lib, case):
     b = run_gpu(cuda_lib, p, q, k, v, force_path=S.PATH_TC)[0].float()
     tol = 4e-3 if dt == "bf16" else 1e-3
     assert (a - b).abs().max().item() <= tol
+
+
+# More 256-row tiles than SM pairs (several waves of CTA pairs), mixed tile
+# weights; with causal masking and forced key splits some (tile, split) units
+# see no key block at all.
+WALK = [
+    # name, B, Hq, Hkv, L, S, causal, window, force_splits
+    ("walk_causal", 2, 16, 16, 1024, 1024, True, 0, 0),
+    ("walk_gqa_noncausal", 3, 32, 8, 512, 640, False, 0, 0),
+    ("walk_window", 2, 16, 8, 1536, 1536, True, 200, 0),
+    ("walk_split_empty_items", 2, 16, 16, 1024, 1024, True, 0, 3),
+]
+
+
+@pytest.mark.parametrize("case", WALK, ids=[c[0] for c in WALK])
+def test_tc2_many_waves(cuda_lib, case):
+    name, B, Hq, Hkv, L, Sk, causal, W, fs = case
+    p = I.Problem(B, Hq, Hkv, L, Sk, 256, 256, "bf16", causal, W, None, 45, name)
+    rows = sorted(set([0, 1, 127, 128, 255, 256, L // 2, L - 129, L - 2, L - 1]))
+    _, _, info = check_problem(cuda_lib, p, rows=rows, force_path=S.PATH_TC2, force_splits=fs)
+    assert info["path"] == S.PATH_TC2
+    assert info["ctas"] > 74
