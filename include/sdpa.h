@@ -301,6 +301,16 @@ SDPA_API void sdpa_time_next_main_kernel(void *start_event, void *stop_event);
  */
 SDPA_API void sdpa_time_next_call(void *start_event, void *stop_event, void *call_event);
 
+/*
+ * Self-test of the kernels' FMA-pipe exp2 (a Cody-Waite range reduction with
+ * a fitted minimax polynomial, used for part of the softmax exponentials):
+ * writes that function's value and exp2f's for n points spread evenly over
+ * [lo, hi] into the device arrays poly[n] and ref[n] (caller-owned, fp32),
+ * asynchronously on the legacy default stream.  For tests; no counterpart in
+ * the pages.
+ */
+SDPA_API sdpa_status sdpa_exp2_selftest(float lo, float hi, int n, float *poly, float *ref);
+
 SDPA_API const char *sdpa_status_string(sdpa_status status);
 /* Message of the last failed call on this thread ("" if none). */
 SDPA_API const char *sdpa_last_error_message(void);

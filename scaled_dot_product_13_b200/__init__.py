@@ -19,7 +19,7 @@ import ctypes
 import os
 
 __all__ = ["forward", "forward_ws", "forward_noalloc", "forward_ex", "Options", "workspace_bytes", "plan", "device_status",
-           "set_wait_limit_ns", "watchdog_selftest", "time_next_main_kernel", "time_next_call", "load_library", "library_path",
+           "set_wait_limit_ns", "watchdog_selftest", "exp2_selftest", "time_next_main_kernel", "time_next_call", "load_library", "library_path",
            "SdpaError", "PATH_AUTO", "PATH_SPLITKV", "PATH_TC", "PATH_TC2", "PATH_WIDE",
            "STATUS"]
 
@@ -84,6 +84,7 @@ def load_library() -> ctypes.CDLL:
     lib.sdpa_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
     lib.sdpa_set_wait_limit_ns.restype = None
     lib.sdpa_watchdog_selftest.argtypes = [ctypes.c_uint64, ctypes.POINTER(ctypes.c_int)]
+    lib.sdpa_exp2_selftest.argtypes = [ctypes.c_float, ctypes.c_float, i, vp, vp]
     lib.sdpa_time_next_main_kernel.argtypes = [vp, vp]
     lib.sdpa_time_next_main_kernel.restype = None
     lib.sdpa_time_next_call.argtypes = [vp, vp, vp]
@@ -93,7 +94,7 @@ def load_library() -> ctypes.CDLL:
     lib.sdpa_last_error_message.restype = ctypes.c_char_p
     for fn in ("sdpa_forward", "sdpa_forward_ws", "sdpa_forward_noalloc", "sdpa_forward_ex",
                "sdpa_forward_planned", "sdpa_plan",
-               "sdpa_device_status", "sdpa_watchdog_selftest"):
+               "sdpa_device_status", "sdpa_watchdog_selftest", "sdpa_exp2_selftest"):
         getattr(lib, fn).restype = ctypes.c_int
     _LIB = lib
     return lib
@@ -294,6 +295,20 @@ def time_next_call(start_event, stop_event, call_event) -> None:
             raise SdpaError(1, "events have no CUDA handle yet; record them once first")
         handles.append(ctypes.c_void_p(e.cuda_event if e is not None else None))
     load_library().sdpa_time_next_call(*handles)
+
+
+def exp2_selftest(lo: float, hi: float, n: int, device="cuda"):
+    """(poly, ref): the kernels' FMA-pipe exp2 and exp2f on n points over
+    [lo, hi], as fp32 CUDA tensors."""
+    import torch
+
+    poly = torch.empty(n, dtype=torch.float32, device=device)
+    ref = torch.empty(n, dtype=torch.float32, device=device)
+    _check(load_library().sdpa_exp2_selftest(ctypes.c_float(lo), ctypes.c_float(hi), int(n),
+                                             ctypes.c_void_p(poly.data_ptr()),
+                                             ctypes.c_void_p(ref.data_ptr())))
+    torch.cuda.synchronize()
+    return poly, ref
 
 
 def set_wait_limit_ns(ns: int) -> None:

@@ -516,6 +516,24 @@ __global__ void watchdog_selftest_kernel(Watchdog wd, int *result) {
   if (threadIdx.x == 0) *result = ok ? 1 : 0;
 }
 
+// Self-test of the FMA-pipe exp2: evaluates exp2_poly2 and exp2f on n
+// points spread evenly over [lo, hi] and writes both results.
+__global__ void exp2_selftest_kernel(float lo, float hi, int n, float *poly, float *ref) {
+  for (int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x); i < n;
+       i += 2 * gridDim.x * blockDim.x) {
+    const float step = n > 1 ? (hi - lo) / (float)(n - 1) : 0.f;
+    const float x0 = lo + step * (float)i;
+    const float x1 = i + 1 < n ? lo + step * (float)(i + 1) : x0;
+    const float2 y = exp2_poly2(make_float2(x0, x1));
+    poly[i] = y.x;
+    ref[i] = exp2f(x0);
+    if (i + 1 < n) {
+      poly[i + 1] = y.y;
+      ref[i + 1] = exp2f(x1);
+    }
+  }
+}
+
 }  // namespace sdpa
 
 // ===========================================================================
@@ -671,6 +689,20 @@ sdpa_status sdpa_watchdog_selftest(uint64_t limit_ns, int *waited_out) {
   cudaFree(d_res);
   if (e != cudaSuccess) return fail(SDPA_ERR_CUDA, "selftest: %s", cudaGetErrorString(e));
   if (waited_out) *waited_out = res;
+  return SDPA_OK;
+}
+
+sdpa_status sdpa_exp2_selftest(float lo, float hi, int n, float *poly, float *ref) {
+  t_last_error.clear();
+  if (n < 1 || !poly || !ref || !(lo <= hi))
+    return fail(SDPA_ERR_INVALID_ARG, "exp2 self-test needs n >= 1, lo <= hi and two buffers");
+  int dev, sms;
+  unsigned int *wd;
+  sdpa_status st = device_state(&dev, &sms, &wd);
+  if (st != SDPA_OK) return st;
+  exp2_selftest_kernel<<<(n + 511) / 512, 256>>>(lo, hi, n, poly, ref);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(SDPA_ERR_CUDA, "exp2 self-test: %s", cudaGetErrorString(e));
   return SDPA_OK;
 }
 

@@ -2,6 +2,11 @@
 #include "launch.h"
 #include "tc.cuh"
 
+// upper bound on K/V ring slots (shared memory allowing)
+#ifndef SDPA_TC_MAX_SLOTS
+#define SDPA_TC_MAX_SLOTS 8
+#endif
+
 namespace sdpa {
 
 namespace {
@@ -13,10 +18,11 @@ sdpa_status run_tc(const Launch &ln, std::string *err) {
   constexpr uint32_t kK = ((DQK + 63) / 64) * kBN * 128;
   constexpr uint32_t kV = ((DV + 63) / 64) * kBN * 128;
   constexpr uint32_t kSlot = kK > kV ? kK : kV;
-  // everything but Q and the slots: row-max exchange (2 KB) and the barriers
-  constexpr uint32_t kBudget = 232448u - 4u * 128u * 4u - 40u * 8u - 16u;
+  // everything but Q and the slots: row-max exchange and the barriers
+  constexpr uint32_t kBudget =
+      232448u - 2u * SDPA_TC_PARTS * 128u * 4u - (2u * SDPA_TC_MAX_SLOTS + 17u) * 8u - 16u;
   constexpr int kFit = (int)((kBudget - kQ) / kSlot);
-  constexpr int kNSlot = kFit > 8 ? 8 : kFit;
+  constexpr int kNSlot = kFit > SDPA_TC_MAX_SLOTS ? SDPA_TC_MAX_SLOTS : kFit;
   static_assert(kNSlot >= 2, "at least two K/V slots");
   using Cfg = TcCfg<DQK, DV, kBN, kNSlot>;
   auto kern = tc_attn_kernel<kBF16, DQK, DV, kBN, kNSlot>;

@@ -10,6 +10,8 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+
+#include "exp2_poly.h"
 #include <stdint.h>
 
 namespace sdpa {
@@ -335,6 +337,15 @@ __device__ __forceinline__ void tmem_st_u16x(uint32_t taddr, const uint32_t *v) 
       : "memory");
 }
 
+// 8 consecutive 32-bit columns per thread (e.g. 16 packed 16-bit values).
+__device__ __forceinline__ void tmem_st_u8x(uint32_t taddr, const uint32_t *v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(
+                   taddr),
+               "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
+               "r"(v[7])
+               : "memory");
+}
+
 // Prefetch one box of a tiled tensor into L2 (no shared memory, no barrier).
 __device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap *map, int x, int y, int z) {
   asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global [%0, {%1, %2, %3}];" ::"l"(
@@ -358,6 +369,34 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b) {
       : "=l"(d)
       : "l"(*reinterpret_cast<uint64_t *>(&a)), "l"(*reinterpret_cast<uint64_t *>(&b)));
   return *reinterpret_cast<float2 *>(&d);
+}
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  uint64_t d;
+  asm("sub.f32x2 %0, %1, %2;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<uint64_t *>(&a)), "l"(*reinterpret_cast<uint64_t *>(&b)));
+  return *reinterpret_cast<float2 *>(&d);
+}
+
+// 2^x on the FMA and integer pipes, for two values at once (x <= 126).
+// Range reduction in the Cody-Waite style: n = round(x) with the 1.5 * 2^23
+// shifter (the integer lands in the low mantissa bits of x + shifter),
+// f = x - n in [-1/2, 1/2], 2^f by the degree-3 minimax polynomial of
+// exp2_poly.h, and n added to the exponent field.  x is clamped at -126 so
+// the exponent cannot wrap; results below 2^-126 come out as tiny normals or
+// denormals instead of zero.  Maximum relative error kExp2PolyMaxRelErr.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  const float2 shifter = make_float2(12582912.f, 12582912.f);
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 t = add2(x, shifter);
+  const float2 f = sub2(x, sub2(t, shifter));
+  float2 q = fma2(make_float2(kExp2C3, kExp2C3), f, make_float2(kExp2C2, kExp2C2));
+  q = fma2(q, f, make_float2(kExp2C1, kExp2C1));
+  q = fma2(q, f, make_float2(kExp2C0, kExp2C0));
+  const int nx = __float_as_int(t.x) << 23, ny = __float_as_int(t.y) << 23;
+  return make_float2(__int_as_float(__float_as_int(q.x) + nx),
+                     __int_as_float(__float_as_int(q.y) + ny));
 }
 __device__ __forceinline__ float fmax3f(float a, float b, float c) {
   float d;

@@ -7,21 +7,24 @@
 //   per-element masks run only on the diagonal, window-edge and tail blocks
 //   (mlx PR #3552, "Implementation").
 //
-// Warp roles (320 threads):
-//   warps 0-7  softmax: warps w and w+4 share query rows 32(w%4) .. +31
-//              (TMEM lanes), each taking one half of every key block's
-//              columns; the pair exchanges its row maxima through shared
-//              memory behind a bounded mbarrier.  fp32 online softmax with a
-//              lazily updated running max.  P is rounded to the 16-bit input
-//              type and written back into tensor memory over the scores it
-//              came from.  At the end the epilogue (O / l, rounded, stored),
-//              each warp of a pair writing half of O's columns.
-//   warp 8     TMA producer: Q once, then K and V blocks in the order the MMA
+// Warp roles (576 threads):
+//   warps 0-15 softmax: warps w, w+4, w+8 and w+12 share query rows
+//              32(w%4) .. +31 (TMEM lanes), each taking one quarter of every
+//              key block's columns; the four exchange their row maxima
+//              through shared memory behind a bounded mbarrier.  Four warps
+//              per scheduler keep the exp / convert chains of one block
+//              overlapped with those of the others.  fp32 online softmax
+//              with a lazily updated running max.  P is rounded to the
+//              16-bit input type and written back into tensor memory over the
+//              scores it came from.  At the end the epilogue (O / l, rounded,
+//              stored), each warp of a row group writing a quarter of O's
+//              columns.
+//   warp 16    TMA producer: Q once, then K and V blocks in the order the MMA
 //              consumes them (K0, K1, then V_j, K_{j+2} for j = 0, 1, ...)
 //              through a FIFO ring of NSLOT shared-memory slots (128-byte
 //              swizzle, zero fill past S and past the head dim), and L2
 //              prefetches of the blocks further ahead.
-//   warp 9     allocates TMEM and issues tcgen05.mma from one thread:
+//   warp 17    allocates TMEM and issues tcgen05.mma from one thread:
 //              S_j = Q K_j^T (A = Q from shared memory) into score buffer
 //              j % 3, and O += P_j V_j with A = P_j read from tensor memory,
 //              then S_{j+2}; the tensor core computes the next scores while
@@ -40,6 +43,20 @@
 
 #include "params.cuh"
 
+// Softmax warps sharing one row of the tile (2 or 4), and how many of every
+// four exponential pairs go to the FMA-pipe polynomial instead of the
+// MUFU ex2 unit (0-4).  Build-time knobs for measurement.
+#ifndef SDPA_TC_PARTS
+#define SDPA_TC_PARTS 2
+#endif
+#ifndef SDPA_TC_POLY_OF4
+#define SDPA_TC_POLY_OF4 0
+#endif
+// blocks prefetched into L2 beyond the one being loaded
+#ifndef SDPA_TC_PREFETCH
+#define SDPA_TC_PREFETCH 4
+#endif
+
 namespace sdpa {
 
 template <int DQK, int DV, int BN, int NSLOT>
@@ -56,24 +73,29 @@ struct TcCfg {
   static constexpr uint32_t kSlotBytes = kKBytes > kVBytes ? kKBytes : kVBytes;
   static constexpr uint32_t kSlotOff = kQBytes;
   static constexpr uint32_t kXOff = kSlotOff + NSLOT * kSlotBytes;  // row-max exchange
-  static constexpr uint32_t kXBytes = 4 * kBM * 4;  // [2 bufs][2 halves][128] row maxima
+  static constexpr int kParts = SDPA_TC_PARTS;      // softmax warps sharing one row
+  static constexpr int kSoftmaxWarps = 4 * kParts;
+  static constexpr int kProducerWarp = kSoftmaxWarps;
+  static constexpr int kMmaWarp = kSoftmaxWarps + 1;
+  static constexpr uint32_t kXBytes = 2 * kParts * kBM * 4;  // [2 bufs][parts][128] row maxima
   static constexpr uint32_t kBarOff = kXOff + kXBytes;
   static constexpr int kNumBars = 2 * NSLOT + 17;
   // exact: the dynamic shared-memory base is 1024-byte aligned (checked at run time)
   static constexpr uint32_t kSmemBytes = kBarOff + kNumBars * 8 + 16;
-  static constexpr int kThreads = 320;
-  static constexpr int kHalf = BN / 2;  // key columns per softmax thread
+  static constexpr int kThreads = (kSoftmaxWarps + 2) * 32;
+  static constexpr int kCols = BN / kParts;  // key columns per softmax thread
   static constexpr uint32_t kTmemCols = 512;
   static constexpr int kOCol = kBufs * BN;
-  static constexpr int kPrefetch = 4;   // blocks prefetched to L2 beyond the one loaded
+  static constexpr int kPrefetch = SDPA_TC_PREFETCH;
   static_assert(DQK % 16 == 0 && DV % 16 == 0 && DV >= 16 && DV <= 256, "head dims");
   static_assert(BN == 64 || BN == 128, "key block");
+  static_assert(kCols == 16 || kCols % 32 == 0, "TMEM load / store widths");
   static_assert(kBufs * BN + DV <= 512, "TMEM columns");
   static_assert(kSmemBytes <= 232448, "shared memory");
 };
 
 template <bool kBF16, int DQK, int DV, int BN, int NSLOT>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(TcCfg<DQK, DV, BN, NSLOT>::kThreads, 1)
     tc_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   using Cfg = TcCfg<DQK, DV, BN, NSLOT>;
@@ -100,8 +122,8 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t *o_bar = buf_free + NB;    // one phase per P V
   uint64_t *o_final = o_bar + 1;      // one phase: every P V of the tile has completed
   uint64_t *fin_bar = o_final + 1;    // teardown drain of the MMA warp
-  uint64_t *pair_bar = fin_bar + 1;   // [4] softmax warp pairs (row-max exchange)
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(pair_bar + 4);
+  uint64_t *part_bar = fin_bar + 1;   // [4] softmax warps of one row group (row-max exchange)
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(part_bar + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -127,16 +149,16 @@ __global__ void __launch_bounds__(320, 1)
     mbar_init(q_full, 1);
     for (int b = 0; b < NB; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&p_full[b], 8);
+      mbar_init(&p_full[b], Cfg::kSoftmaxWarps);
       mbar_init(&buf_free[b], 1);
     }
     mbar_init(o_bar, 1);
     mbar_init(o_final, 1);
     mbar_init(fin_bar, 1);
-    for (int q = 0; q < 4; ++q) mbar_init(&pair_bar[q], 64);
+    for (int q = 0; q < 4; ++q) mbar_init(&part_bar[q], Cfg::kParts * 32);
     fence_barrier_init();
   }
-  if (warp == 9) {
+  if (warp == Cfg::kMmaWarp) {
     tmem_alloc(tmem_slot, Cfg::kTmemCols);
     tmem_relinquish();
   }
@@ -147,7 +169,7 @@ __global__ void __launch_bounds__(320, 1)
   // Let a dependent combine launch now (it waits for this grid to finish).
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-  if (warp == 8) {
+  if (warp == Cfg::kProducerWarp) {
     // ============================ TMA producer ============================
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
@@ -203,7 +225,7 @@ __global__ void __launch_bounds__(320, 1)
       for (int v = u - NSLOT > 0 ? u - NSLOT : 0; v < u; ++v)
         mbar_wait_drain(&slot_full[v % NSLOT], (uint32_t)(v / NSLOT) & 1u, p.wd);
     }
-  } else if (warp == 9) {
+  } else if (warp == Cfg::kMmaWarp) {
     // ============================ MMA issuer ============================
     if (lane == 0) {
       constexpr uint32_t kIdescS = umma_idesc_f16(kBF16, 128, BN, false, false);
@@ -266,23 +288,23 @@ __global__ void __launch_bounds__(320, 1)
       mbar_wait_drain(fin_bar, 0, p.wd);
     }
   } else {
-    // ============ softmax warps: rows 32*(w%4) .. +31, column half w/4 ============
+    // ====== softmax warps: rows 32*(w%4) .. +31, column part w/4 of kParts ======
+    constexpr int kParts = Cfg::kParts;
     const int quarter = warp & 3;
-    const int half = warp >> 2;
+    const int part = warp >> 2;
     const int r = quarter * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const int pos = ((tr.row0 + r) % p.L) + p.off;
     const float c = p.scale_log2;
     const bool c_pos = c >= 0.f;
     const float neutral = c_pos ? -INFINITY : INFINITY;  // never wins the row reduction
-    constexpr int kH = Cfg::kHalf;
+    constexpr int kH = Cfg::kCols;
     constexpr int kOChunks = DV / 16;
-    constexpr int kOC0 = (kOChunks + 1) / 2;
-    const int oc_begin = half == 0 ? 0 : kOC0;
-    const int oc_end = half == 0 ? kOC0 : kOChunks;
+    const int oc_begin = part * kOChunks / kParts;
+    const int oc_end = (part + 1) * kOChunks / kParts;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    uint32_t pair_phase = 0;
+    uint32_t part_phase = 0;
     for (int j = 0; j < nblk; ++j) {
       const int b = j % NB;
       bool w = true;
@@ -293,12 +315,19 @@ __global__ void __launch_bounds__(320, 1)
       }
       tc_fence_after();
       float s[kH];
+      if constexpr (kH == 16) {
+        float s16[16];
+        tmem_ld16(tmem + lane_base + b * BN + part * kH, s16);
 #pragma unroll
-      for (int c32 = 0; c32 < kH / 32; ++c32)
-        tmem_ld32(tmem + lane_base + b * BN + half * kH + c32 * 32, s + c32 * 32);
+        for (int i = 0; i < 16; ++i) s[i] = s16[i];
+      } else {
+#pragma unroll
+        for (int c32 = 0; c32 < kH / 32; ++c32)
+          tmem_ld32(tmem + lane_base + b * BN + part * kH + c32 * 32, s + c32 * 32);
+      }
       tmem_wait_ld();
 
-      // ---- this half's raw row max (masked keys excluded) ----
+      // ---- this part's raw row max (masked keys excluded) ----
       const int kbase = k_lo + j * BN;
       const bool masked = block_needs_mask(p, tr, kbase, BN);
       uint64_t vis = ~0ull;
@@ -306,7 +335,7 @@ __global__ void __launch_bounds__(320, 1)
         vis = 0ull;
 #pragma unroll
         for (int i = 0; i < kH; ++i) {
-          if (key_visible(p, pos, kbase + half * kH + i)) vis |= 1ull << i;
+          if (key_visible(p, pos, kbase + part * kH + i)) vis |= 1ull << i;
           else s[i] = neutral;
         }
       }
@@ -336,20 +365,24 @@ __global__ void __launch_bounds__(320, 1)
         }
         mr[0] = fmin3f(mr[0], mr[1], fminf(mr[2], mr[3]));
       }
-      // ---- combine with the other half of the row (bounded pair barrier).
-      // The barrier also orders this warp's score reads before the partner
+      // ---- combine with the other parts of the row (bounded barrier).  The
+      // barrier also orders every part's score reads before any part
       // overwrites them with P. ----
-      xmax[((j & 1) * 2 + half) * Cfg::kBM + r] = mr[0];
+      xmax[((j & 1) * kParts + part) * Cfg::kBM + r] = mr[0];
       tc_fence_before();
-      mbar_arrive(&pair_bar[quarter]);
-      if (!mbar_wait(&pair_bar[quarter], pair_phase & 1u, p.wd, kWdSoftmax)) {
+      mbar_arrive(&part_bar[quarter]);
+      if (!mbar_wait(&part_bar[quarter], part_phase & 1u, p.wd, kWdSoftmax)) {
         ok = false;
         break;
       }
-      ++pair_phase;
+      ++part_phase;
       tc_fence_after();
-      const float other = xmax[((j & 1) * 2 + (half ^ 1)) * Cfg::kBM + r];
-      const float mraw = c_pos ? fmaxf(mr[0], other) : fminf(mr[0], other);
+      float mraw = mr[0];
+#pragma unroll
+      for (int q = 0; q < kParts; ++q) {
+        const float other = xmax[((j & 1) * kParts + q) * Cfg::kBM + r];
+        mraw = c_pos ? fmaxf(mraw, other) : fminf(mraw, other);
+      }
       const float mblk = isinf(mraw) ? -INFINITY : mraw * c;
       const float m_new = fmaxf(m_used, mblk);
       const bool need = m_new > m_used + 8.0f;
@@ -392,8 +425,12 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
       for (int i = 0; i < kH; i += 2) {
         float2 t = fma2(make_float2(s[i], s[i + 1]), c2, nm2);
-        t.x = fast_exp2(t.x);
-        t.y = fast_exp2(t.y);
+        if (((i >> 1) & 3) < SDPA_TC_POLY_OF4) {
+          t = exp2_poly2(t);  // FMA / ALU pipes
+        } else {
+          t.x = fast_exp2(t.x);  // MUFU
+          t.y = fast_exp2(t.y);
+        }
         if (masked) {
           t.x = ((vis >> i) & 1ull) ? t.x : 0.f;
           t.y = ((vis >> (i + 1)) & 1ull) ? t.y : 0.f;
@@ -404,10 +441,15 @@ __global__ void __launch_bounds__(320, 1)
       const float2 a01 = add2(acc[0], acc[1]), a23 = add2(acc[2], acc[3]);
       const float2 at = add2(a01, a23);
       l += at.x + at.y;
-      // P_j into this warp's columns of buffer b (over the scores of half 0)
+      // P_j into this warp's packed columns of buffer b (over the first
+      // BN/2 score columns)
+      if constexpr (kH == 16) {
+        tmem_st_u8x(tmem + lane_base + b * BN + part * (kH / 2), pk);
+      } else {
 #pragma unroll
-      for (int c16 = 0; c16 < kH / 32; ++c16)
-        tmem_st_u16x(tmem + lane_base + b * BN + half * (kH / 2) + c16 * 16, pk + c16 * 16);
+        for (int c16 = 0; c16 < kH / 32; ++c16)
+          tmem_st_u16x(tmem + lane_base + b * BN + part * (kH / 2) + c16 * 16, pk + c16 * 16);
+      }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -415,13 +457,15 @@ __global__ void __launch_bounds__(320, 1)
     }
 
     // ------------------------------ epilogue ------------------------------
-    // row sum = both halves' partial sums, exchanged through the max buffer the
-    // last block did not use (its last reader passed the last pair barrier)
-    float *xl = xmax + (nblk & 1) * 2 * Cfg::kBM;
-    xl[half * Cfg::kBM + r] = l;
-    mbar_arrive(&pair_bar[quarter]);
-    if (!mbar_wait(&pair_bar[quarter], pair_phase & 1u, p.wd, kWdSoftmax)) ok = false;
-    l += xl[(half ^ 1) * Cfg::kBM + r];
+    // row sum = the parts' partial sums, exchanged through the max buffer the
+    // last block did not use (its last reader passed the last barrier)
+    float *xl = xmax + (nblk & 1) * kParts * Cfg::kBM;
+    xl[part * Cfg::kBM + r] = l;
+    mbar_arrive(&part_bar[quarter]);
+    if (!mbar_wait(&part_bar[quarter], part_phase & 1u, p.wd, kWdSoftmax)) ok = false;
+    l = 0.f;
+#pragma unroll
+    for (int q = 0; q < kParts; ++q) l += xl[q * Cfg::kBM + r];
     if (ok && nblk > 0) {
       bool w = true;
       if (lane == 0) w = mbar_wait(o_final, 0, p.wd, kWdMma);
@@ -434,7 +478,7 @@ __global__ void __launch_bounds__(320, 1)
     float inv = l > 0.f ? 1.f / l : 0.f;
     if (p.splits == 1) {
       inv = finish_row(p, grow, m_used, l);
-      if (p.lse_out != nullptr && valid && half == 0) p.lse_out[grow] = row_lse(m_used, l);
+      if (p.lse_out != nullptr && valid && part == 0) p.lse_out[grow] = row_lse(m_used, l);
       uint8_t *orow = reinterpret_cast<uint8_t *>(p.out) + grow * p.Dv * 2;
 #pragma unroll 1
       for (int c16 = oc_begin; c16 < oc_end; ++c16) {
@@ -477,7 +521,7 @@ __global__ void __launch_bounds__(320, 1)
                             o[q4 * 4 + 3] * inv);
         }
       }
-      if (valid && half == 0)
+      if (valid && part == 0)
         p.part_lse[(long)split * total_rows + grow] = have_o ? row_lse(m_used, l) : -INFINITY;
     }
   }
@@ -485,7 +529,7 @@ __global__ void __launch_bounds__(320, 1)
   // ------------------------------ teardown ------------------------------
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == Cfg::kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, Cfg::kTmemCols);
   }

@@ -31,6 +31,12 @@
 
 #include "params.cuh"
 
+// How many of every four exponential pairs of the softmax go to the FMA-pipe
+// polynomial instead of the MUFU ex2 unit (0-4).  Build-time knob.
+#ifndef SDPA_TC2_POLY_OF4
+#define SDPA_TC2_POLY_OF4 1
+#endif
+
 namespace sdpa {
 
 template <int DQK, int DV, int BN, int NSLOT>
@@ -392,8 +398,12 @@ __global__ void __launch_bounds__(352, 1)
 #pragma unroll
       for (int i = 0; i < kH; i += 2) {
         float2 t = fma2(make_float2(s[i], s[i + 1]), c2, nm2);
-        t.x = fast_exp2(t.x);
-        t.y = fast_exp2(t.y);
+        if (((i >> 1) & 3) < SDPA_TC2_POLY_OF4) {
+          t = exp2_poly2(t);  // FMA / ALU pipes
+        } else {
+          t.x = fast_exp2(t.x);  // MUFU
+          t.y = fast_exp2(t.y);
+        }
         if (masked) {
           t.x = ((vis >> i) & 1ull) ? t.x : 0.f;
           t.y = ((vis >> (i + 1)) & 1ull) ? t.y : 0.f;

@@ -20,6 +20,23 @@ from scaled_dot_product_13_b200.inputs import Problem, make_qkv
 TOL_MAX = {"bf16": 2e-2, "f16": 5e-3}
 TOL_MEAN = 2e-3
 
+# GPU-vs-GPU agreement (two routes, split counts, layouts of the same
+# problem).  Both results are the same softmax up to rounding order: fp32
+# accumulation in another order, P rounded to 16 bits from slightly different
+# exponentials (MUFU or the FMA-pipe polynomial), and one final rounding of O.
+# The last step alone can flip an output by one unit in the last place of the
+# output type, i.e. up to 2^-7 (bf16) / 2^-10 (fp16) of its magnitude, so
+# the bound is an absolute part plus one such unit.
+AGREE_ABS = {"bf16": 4e-3, "f16": 1e-3}
+AGREE_ULP = {"bf16": 2.0 ** -7, "f16": 2.0 ** -10}
+
+
+def agree(a, b, dtype: str) -> bool:
+    """True when |a - b| <= AGREE_ABS + one output ulp of |b|, elementwise."""
+    a = a.float()
+    b = b.float()
+    return bool(((a - b).abs() <= AGREE_ABS[dtype] + AGREE_ULP[dtype] * b.abs()).all())
+
 
 def run_gpu(sdpa, p: Problem, q, k, v, force_path=0, force_splits=0, guard=True):
     """Run one call with an explicit workspace and canary guard bands around

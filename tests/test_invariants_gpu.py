@@ -7,13 +7,10 @@ import pytest
 import torch
 
 from scaled_dot_product_13_b200 import inputs as I
-from tests.gpu_util import TOL_MAX, TOL_MEAN, check_problem, run_gpu
+from tests.gpu_util import agree, TOL_MAX, TOL_MEAN, check_problem, run_gpu
 
 pytestmark = pytest.mark.gpu
 
-# GPU vs GPU agreement between routes / split counts (both are within the
-# oracle tolerance; they differ only by accumulation order)
-AGREE = {"bf16": 4e-3, "f16": 1e-3}
 
 
 def _out(sdpa, p, q, k, v, **kw):
@@ -31,7 +28,7 @@ def test_splits_agree_with_each_other(cuda_lib):
     q, k, v = I.make_qkv(p)
     outs = [_out(cuda_lib, p, q, k, v, force_splits=s) for s in (1, 2, 7, 39)]
     for o in outs[1:]:
-        assert (o - outs[0]).abs().max().item() <= AGREE["f16"]
+        assert agree(o, outs[0], "f16")
 
 
 def test_gqa_equals_repeated_kv(cuda_lib):
@@ -41,7 +38,7 @@ def test_gqa_equals_repeated_kv(cuda_lib):
     pr = p.with_(Hkv=8)
     b = _out(cuda_lib, pr, q, k.repeat_interleave(4, 1).contiguous(),
              v.repeat_interleave(4, 1).contiguous())
-    assert (a - b).abs().max().item() <= AGREE["bf16"]
+    assert agree(a, b, "bf16")
 
 
 def test_window_ge_s_equals_causal(cuda_lib):
@@ -58,7 +55,7 @@ def test_decode_equals_last_prefill_row(cuda_lib):
     q, k, v = I.make_qkv(p)
     full = _out(cuda_lib, p, q, k, v)
     last = _out(cuda_lib, p.with_(L=1), q[:, :, -1:].contiguous(), k, v)
-    assert (full[:, :, -1] - last[:, :, 0]).abs().max().item() <= AGREE["f16"]
+    assert agree(full[:, :, -1], last[:, :, 0], "f16")
 
 
 def test_repeated_calls_are_deterministic(cuda_lib):

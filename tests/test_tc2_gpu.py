@@ -8,7 +8,7 @@ import torch
 import scaled_dot_product_13_b200 as S
 from oracle import sdpa_oracle
 from scaled_dot_product_13_b200 import inputs as I
-from tests.gpu_util import TOL_MAX, TOL_MEAN, check_problem, run_gpu
+from tests.gpu_util import agree, TOL_MAX, TOL_MEAN, check_problem, run_gpu
 
 pytestmark = pytest.mark.gpu
 
@@ -70,8 +70,7 @@ def test_tc2_agrees_with_tc(cuda_lib, case):
     q, k, v = I.make_qkv(p)
     a = run_gpu(cuda_lib, p, q, k, v, force_path=S.PATH_TC2)[0].float()
     b = run_gpu(cuda_lib, p, q, k, v, force_path=S.PATH_TC)[0].float()
-    tol = 4e-3 if dt == "bf16" else 1e-3
-    assert (a - b).abs().max().item() <= tol
+    assert agree(a, b, dt)
 
 
 # More 256-row tiles than SM pairs (several waves of CTA pairs), mixed tile
