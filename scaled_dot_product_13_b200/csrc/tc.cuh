@@ -7,28 +7,27 @@
 //   per-element masks run only on the diagonal, window-edge and tail blocks
 //   (mlx PR #3552, "Implementation").
 //
-// Warp roles (576 threads):
-//   warps 0-15 softmax: warps w, w+4, w+8 and w+12 share query rows
-//              32(w%4) .. +31 (TMEM lanes), each taking one quarter of every
-//              key block's columns; the four exchange their row maxima
-//              through shared memory behind a bounded mbarrier.  Four warps
-//              per scheduler keep the exp / convert chains of one block
-//              overlapped with those of the others.  fp32 online softmax
-//              with a lazily updated running max.  P is rounded to the
-//              16-bit input type and written back into tensor memory over the
-//              scores it came from.  At the end the epilogue (O / l, rounded,
-//              stored), each warp of a row group writing a quarter of O's
+// Warp roles (320 threads with the default two softmax warps per row):
+//   softmax    4 kParts warps: warps w, w+4, ... share query rows
+//              32(w%4) .. +31 (TMEM lanes), each taking 1/kParts of every
+//              key block's columns; they exchange their row maxima through
+//              shared memory behind a bounded mbarrier.  fp32 online softmax
+//              with a lazily updated running max.  P is rounded to the 16-bit
+//              input type and written back into tensor memory over the scores
+//              it came from.  At the end the epilogue (O / l, rounded,
+//              stored), each warp of a row group writing its share of O's
 //              columns.
-//   warp 16    TMA producer: Q once, then K and V blocks in the order the MMA
-//              consumes them (K0, K1, then V_j, K_{j+2} for j = 0, 1, ...)
-//              through a FIFO ring of NSLOT shared-memory slots (128-byte
-//              swizzle, zero fill past S and past the head dim), and L2
-//              prefetches of the blocks further ahead.
-//   warp 17    allocates TMEM and issues tcgen05.mma from one thread:
-//              S_j = Q K_j^T (A = Q from shared memory) into score buffer
-//              j % 3, and O += P_j V_j with A = P_j read from tensor memory,
-//              then S_{j+2}; the tensor core computes the next scores while
-//              the softmax warps work on the current ones.
+//   producer   (the next warp) TMA producer: Q once, then K and V blocks
+//              in the order the MMA consumes them (K0, K1, K2, then V_j,
+//              K_{j+3} for j = 0, 1, ...) through a FIFO ring of NSLOT
+//              shared-memory slots (128-byte swizzle, zero fill past S and
+//              past the head dim), and L2 prefetches of the blocks further
+//              ahead.
+//   MMA        (the last warp) allocates TMEM and issues tcgen05.mma from
+//              one thread: S_j = Q K_j^T (A = Q from shared memory) into
+//              score buffer j % 3, and O += P_j V_j with A = P_j read from
+//              tensor memory, then S_{j+3}: the scores run up to three
+//              blocks ahead of the softmax warps.
 //
 // TMEM (512 columns x 128 lanes x 32 bit): three score buffers of BN
 // columns (P_j overwrites the first BN/2 columns of its buffer as packed
@@ -79,7 +78,7 @@ struct TcCfg {
   static constexpr int kMmaWarp = kSoftmaxWarps + 1;
   static constexpr uint32_t kXBytes = 2 * kParts * kBM * 4;  // [2 bufs][parts][128] row maxima
   static constexpr uint32_t kBarOff = kXOff + kXBytes;
-  static constexpr int kNumBars = 2 * NSLOT + 17;
+  static constexpr int kNumBars = 2 * NSLOT + 15;
   // exact: the dynamic shared-memory base is 1024-byte aligned (checked at run time)
   static constexpr uint32_t kSmemBytes = kBarOff + kNumBars * 8 + 16;
   static constexpr int kThreads = (kSoftmaxWarps + 2) * 32;
@@ -118,9 +117,8 @@ __global__ void __launch_bounds__(TcCfg<DQK, DV, BN, NSLOT>::kThreads, 1)
   uint64_t *q_full = bars + 2 * NSLOT;
   uint64_t *s_full = q_full + 1;      // [3] S_j complete (MMA -> softmax)
   uint64_t *p_full = s_full + NB;     // [3] P_j in TMEM, O rescaled (softmax -> MMA)
-  uint64_t *buf_free = p_full + NB;   // [3] P_j V complete: buffer reusable (MMA -> MMA)
-  uint64_t *o_bar = buf_free + NB;    // one phase per P V
-  uint64_t *o_final = o_bar + 1;      // one phase: every P V of the tile has completed
+  uint64_t *o_bar = p_full + NB;      // [2] P_j V complete, on o_bar[j % 2]
+  uint64_t *o_final = o_bar + 2;      // one phase: every P V of the tile has completed
   uint64_t *fin_bar = o_final + 1;    // teardown drain of the MMA warp
   uint64_t *part_bar = fin_bar + 1;   // [4] softmax warps of one row group (row-max exchange)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(part_bar + 4);
@@ -150,9 +148,9 @@ __global__ void __launch_bounds__(TcCfg<DQK, DV, BN, NSLOT>::kThreads, 1)
     for (int b = 0; b < NB; ++b) {
       mbar_init(&s_full[b], 1);
       mbar_init(&p_full[b], Cfg::kSoftmaxWarps);
-      mbar_init(&buf_free[b], 1);
     }
-    mbar_init(o_bar, 1);
+    mbar_init(&o_bar[0], 1);
+    mbar_init(&o_bar[1], 1);
     mbar_init(o_final, 1);
     mbar_init(fin_bar, 1);
     for (int q = 0; q < 4; ++q) mbar_init(&part_bar[q], Cfg::kParts * 32);
@@ -216,9 +214,10 @@ __global__ void __launch_bounds__(TcCfg<DQK, DV, BN, NSLOT>::kThreads, 1)
       };
       if (nblk > 0) emit(true, 0);
       if (ok && nblk > 1) emit(true, 1);
+      if (ok && nblk > 2) emit(true, 2);
       for (int j = 0; ok && j < nblk; ++j) {
         emit(false, j);
-        if (ok && j + 2 < nblk) emit(true, j + 2);
+        if (ok && j + 3 < nblk) emit(true, j + 3);
       }
       // drain copies still landing (only ever waits after an abort)
       mbar_wait_drain(q_full, 0, p.wd);
@@ -234,13 +233,14 @@ __global__ void __launch_bounds__(TcCfg<DQK, DV, BN, NSLOT>::kThreads, 1)
       const uint32_t slot_addr = smem_u32(sSlots);
       bool ok = mbar_wait(q_full, 0, p.wd, kWdTmaFull);
       int u = 0;
-      // S_n = Q K_n^T into buffer n % 3 (free once P_{n-3} V has completed)
+      // S_n = Q K_n^T into buffer n % 3.  That buffer last held P_{n-3},
+      // whose P V this thread issued earlier; one thread's tcgen05 MMAs run
+      // in issue order, so no wait is needed before overwriting it.
       auto issue_s = [&](int n) -> bool {
         const int slot = u % NSLOT;
         if (!mbar_wait(&slot_full[slot], (uint32_t)(u / NSLOT) & 1u, p.wd, kWdTmaFull)) return false;
         ++u;
         const int b = n % NB;
-        if (!mbar_wait(&buf_free[b], ((uint32_t)(n / NB) & 1u) ^ 1u, p.wd, kWdMma)) return false;
         tc_fence_after();
         const uint32_t kb = slot_addr + slot * Cfg::kSlotBytes;
 #pragma unroll
@@ -269,16 +269,16 @@ __global__ void __launch_bounds__(TcCfg<DQK, DV, BN, NSLOT>::kThreads, 1)
           tc_mma_ts(tmem + Cfg::kOCol, tmem + b * BN + ks * 8, bd, kIdescPV,
                     (j > 0 || ks > 0) ? 1u : 0u);
         }
-        tc_commit(o_bar);
-        tc_commit(&buf_free[b]);
+        tc_commit(&o_bar[j & 1]);
         tc_commit(&slot_empty[slot]);
         return true;
       };
       if (ok && nblk > 0) ok = issue_s(0);
       if (ok && nblk > 1) ok = issue_s(1);
+      if (ok && nblk > 2) ok = issue_s(2);
       for (int j = 0; ok && j < nblk; ++j) {
         ok = issue_pv(j);
-        if (ok && j + 2 < nblk) ok = issue_s(j + 2);
+        if (ok && j + 3 < nblk) ok = issue_s(j + 3);
       }
       // o_bar tells one P V from the next only while at most one is pending;
       // the epilogue needs "all of them", so it gets its own one-shot barrier
@@ -394,11 +394,13 @@ __global__ void __launch_bounds__(TcCfg<DQK, DV, BN, NSLOT>::kThreads, 1)
       }
       if (j > 0 && __any_sync(0xffffffffu, need)) {
         // O holds P_0..P_{j-1} V: wait for the last P V, then rescale this
-        // warp's columns in TMEM.  Parity is unambiguous here: S_j was issued
-        // after P_{j-2} V by the same thread, so S_j's completion implies that
-        // P V completed; P_j V is not issued before p_full: o_bar is in phase
-        // j-1 or j.
-        if (lane == 0) w = mbar_wait(o_bar, (uint32_t)(j - 1) & 1u, p.wd, kWdMma);
+        // warp's columns in TMEM.  P_{j-1} V commits to o_bar[(j-1) % 2] as
+        // that barrier's phase (j-1) / 2.  The parity is unambiguous: S_j was
+        // issued after P_{j-3} V by the same thread, so S_j's completion
+        // implies the barrier's previous phase (P_{j-3} V) completed, and its
+        // next one (P_{j+1} V) waits for p_full of a block not yet done.
+        if (lane == 0)
+          w = mbar_wait(&o_bar[(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1u, p.wd, kWdMma);
         if (!__shfl_sync(0xffffffffu, (int)w, 0)) {
           ok = false;
           break;
