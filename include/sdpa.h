@@ -93,10 +93,13 @@ typedef enum {
                             cta_group::2): each SM loads half of every K/V
                             block; head dims 256/256, 192/128 (routed) and
                             128/128 (on request)                             */
-  SDPA_PATH_WIDE = 4     /* head dims above 256 (up to 512): 16-row groups
+  SDPA_PATH_WIDE = 4,    /* head dims above 256 (up to 512): 16-row groups
                             whose four warps split the output columns, key
                             splits + combine as on SDPA_PATH_SPLITKV; the
                             only path for those head dims                    */
+  SDPA_PATH_TC_DUAL = 5  /* head dims up to 128: two 128-row tiles per CTA
+                            share each K/V block, their softmax phases
+                            interleaved with each other's MMAs (tcgen05)     */
 } sdpa_path;
 
 /*

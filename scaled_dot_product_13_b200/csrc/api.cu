@@ -168,7 +168,8 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
   if (pl.pair < 0)
     return fail(SDPA_ERR_UNSUPPORTED, "no kernel instance covers Dqk=%d, Dv=%d", pb.Dqk, pb.Dv);
   if (force_path != SDPA_PATH_AUTO && force_path != SDPA_PATH_SPLITKV &&
-      force_path != SDPA_PATH_TC && force_path != SDPA_PATH_TC2 && force_path != SDPA_PATH_WIDE)
+      force_path != SDPA_PATH_TC && force_path != SDPA_PATH_TC2 && force_path != SDPA_PATH_WIDE &&
+      force_path != SDPA_PATH_TC_DUAL)
     return fail(SDPA_ERR_INVALID_ARG, "unknown path %d", force_path);
   // head dims above 256 run only on the column-split kernel, and it only on them
   const bool wide = pl.pair == kWidePair;
@@ -193,6 +194,14 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
     // wide heads with at least one full 256-row pair tile: two SMs per tile
     if (path == SDPA_PATH_TC && tc2_preferred_pair(pl.pair) && pl.rows >= kTc2RowThreshold)
       path = SDPA_PATH_TC2;
+    // head dims <= 128: two 128-row tiles per CTA, when the 256-row tiles
+    // alone occupy at least half of the SMs (fewer would rather take the
+    // one-tile kernel's twice as many CTAs) and no window trims the tiles'
+    // key ranges differently (the pair walks the union of both ranges)
+    if (path == SDPA_PATH_TC && tc_dual_supports_pair(pl.pair) && pb.window == 0 &&
+        pl.rows >= kTc2RowThreshold &&
+        (long long)pb.B * pb.Hkv * ((pl.rows + 255) / 256) * 2 >= num_sms)
+      path = SDPA_PATH_TC_DUAL;
   }
   if (path == SDPA_PATH_TC2 && !tc2_supports_pair(pl.pair)) {
     // the smallest two-CTA instance that covers the head dims (zero filled)
@@ -206,8 +215,15 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
     return fail(SDPA_ERR_UNSUPPORTED,
                 "the two-CTA path is built for head dims 256/256, 192/128 and 128/128 (got %d/%d)",
                 pb.Dqk, pb.Dv);
+  if (path == SDPA_PATH_TC_DUAL && !tc_dual_supports_pair(pl.pair))
+    return fail(SDPA_ERR_UNSUPPORTED,
+                "the two-tile path is built for head dims up to 128 (got %d/%d)", pb.Dqk, pb.Dv);
   pl.path = path;
-  if (path == SDPA_PATH_WIDE) {
+  if (path == SDPA_PATH_TC_DUAL) {
+    pl.wr = 0; pl.wk = 0;
+    pl.row_tile = 2 * kTcRows;
+    pl.key_block = 128;
+  } else if (path == SDPA_PATH_WIDE) {
     // one 16-row group (four warps) for decode-sized problems, two otherwise
     pl.wr = pl.rows <= 16 ? 1 : 2;
     pl.wk = 0;
@@ -392,10 +408,11 @@ sdpa_status forward_call(const Problem &pb, const void *q, const void *k, const 
   ln.ev_stop = t_ev_stop;
   cudaEvent_t ev_call = t_ev_call;
   t_ev_start = t_ev_stop = t_ev_call = nullptr;
-  st = pl.path == SDPA_PATH_TC2    ? launch_tc2(ln, &err)
-       : pl.path == SDPA_PATH_TC   ? launch_tc(ln, &err)
-       : pl.path == SDPA_PATH_WIDE ? launch_wide(ln, &err)
-                                   : launch_splitkv(ln, &err);
+  st = pl.path == SDPA_PATH_TC2       ? launch_tc2(ln, &err)
+       : pl.path == SDPA_PATH_TC      ? launch_tc(ln, &err)
+       : pl.path == SDPA_PATH_TC_DUAL ? launch_tc_pp(ln, &err)
+       : pl.path == SDPA_PATH_WIDE    ? launch_wide(ln, &err)
+                                      : launch_splitkv(ln, &err);
   if (st == SDPA_OK && pl.splits > 1) st = launch_combine(ln, &err);
   if (st == SDPA_OK && ev_call) record_event(ev_call, stream);
   if (allocated) {

@@ -102,6 +102,10 @@ sdpa_status launch_splitkv(const Launch &ln, std::string *err);
 sdpa_status launch_tc(const Launch &ln, std::string *err);
 sdpa_status launch_tc2(const Launch &ln, std::string *err);
 sdpa_status launch_wide(const Launch &ln, std::string *err);
+sdpa_status launch_tc_pp(const Launch &ln, std::string *err);
+
+// Head-dim pairs the two-tile kernel is built for (index into kDimPairs).
+constexpr bool tc_dual_supports_pair(int pair) { return pair <= 2; }
 
 // Head-dim pairs the two-CTA kernel is built for (index into kDimPairs), and
 // those the router sends to it by itself (where it measured faster than one

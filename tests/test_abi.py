@@ -164,3 +164,19 @@ def test_plan_head_dims_above_256_take_the_wide_path():
     with pytest.raises(sdpa.SdpaError) as ei:
         sdpa.plan(1, 4, 4, 64, 64, 256, 256, num_sms=148, force_path=sdpa.PATH_WIDE)
     assert ei.value.status == 2
+
+
+def test_plan_two_tile_path_for_small_head_dims():
+    # 20 heads x 1500 rows at D=64: 120 CTAs of two 128-row tiles
+    info = sdpa.plan(1, 20, 20, 1500, 1500, 64, 64, causal=False, num_sms=148)
+    assert info["path"] == sdpa.PATH_TC_DUAL and info["row_tile"] == 256 and info["ctas"] == 120
+    # too few 256-row tiles to fill half the SMs: one tile per CTA
+    info = sdpa.plan(1, 16, 16, 1024, 1024, 72, 72, causal=False, num_sms=148)
+    assert info["path"] == sdpa.PATH_TC
+    # a window trims the two tiles' key ranges differently: one tile per CTA
+    info = sdpa.plan(1, 16, 8, 4096, 4096, 128, 128, causal=True, window_size=1024, num_sms=148)
+    assert info["path"] == sdpa.PATH_TC
+    # head dims above 128 never take it
+    with pytest.raises(sdpa.SdpaError) as ei:
+        sdpa.plan(1, 4, 4, 512, 512, 192, 128, num_sms=148, force_path=sdpa.PATH_TC_DUAL)
+    assert ei.value.status == 2
