@@ -13,7 +13,7 @@ sdpa_status run_tc2(const Launch &ln, std::string *err) {
   constexpr uint32_t kK = (DQK / 64) * (kBN / 2) * 128;
   constexpr uint32_t kV = (DV / 128) * kBN * 128;
   constexpr uint32_t kSlot = kK > kV ? kK : kV;
-  constexpr uint32_t kBudget = 232448u - 4u * 128u * 4u - 48u * 8u - 16u;
+  constexpr uint32_t kBudget = 232448u - 48u * 8u - 16u;
   constexpr int kFit = (int)((kBudget - kQ) / kSlot);
   constexpr int kNSlot = kFit > 8 ? 8 : kFit;
   static_assert(kNSlot >= 2, "at least two K/V slots");

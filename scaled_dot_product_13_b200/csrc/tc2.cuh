@@ -16,12 +16,15 @@
 // of its loads to the even CTA's barriers; the even CTA's MMA thread commits
 // to barriers in both CTAs with two plain commits.
 //
-// Warp roles per CTA (352 threads):
-//   warps 0-7  softmax on this CTA's 128 rows, as in tc.cuh; P_j is written
-//              to this CTA's TMEM and signalled to the even CTA's p_full.
-//   warp 8     TMA producer for this CTA's halves.
-//   warp 9     TMEM allocation (pair); the MMA issuer in the even CTA.
-//   warp 10    odd CTA: forwards its load completions to the even CTA.
+// Warp roles per CTA (224 threads):
+//   warps 0-3  softmax on this CTA's 128 rows, one row per thread with all
+//              BN columns of a block, so a row's max needs no exchange
+//              between warps; lazily moved running max as in tc.cuh.  P_j is
+//              written over the row's own scores in this CTA's TMEM and
+//              signalled to the even CTA's p_full.
+//   warp 4     TMA producer for this CTA's halves.
+//   warp 5     TMEM allocation (pair); the MMA issuer in the even CTA.
+//   warp 6     odd CTA: forwards its load completions to the even CTA.
 //
 // TMEM per CTA: two score buffers of BN columns (P_j over the first BN/2
 // columns of buffer j % 2), O at [2 BN, 2 BN + DV).  A score buffer is reused
@@ -52,13 +55,10 @@ struct Tc2Cfg {
   static constexpr uint32_t kVBytes = kVBoxes * BN * 128;        // this CTA's V half
   static constexpr uint32_t kSlotBytes = kKBytes > kVBytes ? kKBytes : kVBytes;
   static constexpr uint32_t kSlotOff = kQBytes;
-  static constexpr uint32_t kXOff = kSlotOff + NSLOT * kSlotBytes;
-  static constexpr uint32_t kXBytes = 4 * kBM * 4;
-  static constexpr uint32_t kBarOff = kXOff + kXBytes;
-  static constexpr int kNumBars = 3 * NSLOT + 20;
+  static constexpr uint32_t kBarOff = kSlotOff + NSLOT * kSlotBytes;
+  static constexpr int kNumBars = 3 * NSLOT + 16;
   static constexpr uint32_t kSmemBytes = kBarOff + kNumBars * 8 + 16;
-  static constexpr int kThreads = 352;
-  static constexpr int kHalf = BN / 2;
+  static constexpr int kThreads = 224;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr int kOCol = 2 * BN;
   static_assert(DQK % 64 == 0 && (DV == 128 || DV == 256), "pair split needs 64-column halves");
@@ -68,7 +68,7 @@ struct Tc2Cfg {
 };
 
 template <bool kBF16, int DQK, int DV, int BN, int NSLOT>
-__global__ void __launch_bounds__(352, 1)
+__global__ void __launch_bounds__(224, 1)
     tc2_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   using Cfg = Tc2Cfg<DQK, DV, BN, NSLOT>;
@@ -81,7 +81,6 @@ __global__ void __launch_bounds__(352, 1)
   uint8_t *smem = smem_raw;
   uint8_t *sQ = smem;
   uint8_t *sSlots = smem + Cfg::kSlotOff;
-  float *xmax = reinterpret_cast<float *>(smem + Cfg::kXOff);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kBarOff);
   uint64_t *slot_full = bars;                // [NSLOT] this CTA's loads landed
   uint64_t *slot_empty = slot_full + NSLOT;  // [NSLOT] the pair's MMA is done with the slot
@@ -94,8 +93,7 @@ __global__ void __launch_bounds__(352, 1)
   uint64_t *o_final = o_bar + 1;
   uint64_t *fin_bar = o_final + 1;           // all MMAs of the pair complete
   uint64_t *bye_bar = fin_bar + 1;           // teardown: the other CTA is done with us
-  uint64_t *pair_bar = bye_bar + 1;          // [4] softmax warp pairs
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(pair_bar + 4);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bye_bar + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -131,16 +129,15 @@ __global__ void __launch_bounds__(352, 1)
     mbar_init(peer_q, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&p_full[b], 16);
+      mbar_init(&p_full[b], 8);
     }
     mbar_init(o_bar, 1);
     mbar_init(o_final, 1);
     mbar_init(fin_bar, 1);
     mbar_init(bye_bar, 1);
-    for (int q = 0; q < 4; ++q) mbar_init(&pair_bar[q], 64);
     fence_barrier_init();
   }
-  if (warp == 9) {
+  if (warp == 5) {
     tmem_alloc_pair(tmem_slot, Cfg::kTmemCols);
     tmem_relinquish_pair();
   }
@@ -151,7 +148,7 @@ __global__ void __launch_bounds__(352, 1)
   const uint32_t tmem = *tmem_slot;
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-  if (warp == 8) {
+  if (warp == 4) {
     // ====================== TMA producer (this CTA's halves) ======================
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
@@ -198,7 +195,7 @@ __global__ void __launch_bounds__(352, 1)
       for (int v = u - NSLOT > 0 ? u - NSLOT : 0; v < u; ++v)
         mbar_wait_drain(&slot_full[v % NSLOT], (uint32_t)(v / NSLOT) & 1u, p.wd);
     }
-  } else if (warp == 10) {
+  } else if (warp == 6) {
     // ============ odd CTA: relay its load completions to the even CTA ============
     if (!leader && lane == 0) {
       const int nloads = nblk > 0 ? 2 * nblk : 0;
@@ -211,7 +208,7 @@ __global__ void __launch_bounds__(352, 1)
         mbar_arrive_cluster(mapa_shared(smem_u32(&peer_full[slot]), 0));
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == 5) {
     // ====================== MMA issuer (even CTA only) ======================
     if (leader && lane == 0) {
       constexpr uint32_t kIdescS = umma_idesc_f16(kBF16, 256, BN, false, false);
@@ -280,23 +277,16 @@ __global__ void __launch_bounds__(352, 1)
       both(fin_bar);
     }
   } else {
-    // ============ softmax warps on this CTA's 128 rows ============
+    // ====== softmax warps 0-3: one row of this CTA's 128 per thread ======
     const int quarter = warp & 3;
-    const int half = warp >> 2;
     const int r = quarter * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const int pos = ((tr.row0 + r) % p.L) + p.off;
     const float c = p.scale_log2;
     const bool c_pos = c >= 0.f;
     const float neutral = c_pos ? -INFINITY : INFINITY;
-    constexpr int kH = Cfg::kHalf;
-    constexpr int kOChunks = DV / 16;
-    constexpr int kOC0 = (kOChunks + 1) / 2;
-    const int oc_begin = half == 0 ? 0 : kOC0;
-    const int oc_end = half == 0 ? kOC0 : kOChunks;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    uint32_t pair_phase = 0;
     for (int j = 0; j < nblk; ++j) {
       const int b = j & 1;
       bool w = true;
@@ -306,32 +296,28 @@ __global__ void __launch_bounds__(352, 1)
         break;
       }
       tc_fence_after();
-      float s[kH];
+      float s[BN];
 #pragma unroll
-      for (int c32 = 0; c32 < kH / 32; ++c32)
-        tmem_ld32(tmem + lane_base + b * BN + half * kH + c32 * 32, s + c32 * 32);
+      for (int c32 = 0; c32 < BN / 32; ++c32)
+        tmem_ld32(tmem + lane_base + b * BN + c32 * 32, s + c32 * 32);
       tmem_wait_ld();
 
       const int kbase = k_lo + j * BN;
       const bool masked = block_needs_mask(p, tr, kbase, BN);
-      uint64_t vis = ~0ull;
       if (masked) {
-        vis = 0ull;
 #pragma unroll
-        for (int i = 0; i < kH; ++i) {
-          if (key_visible(p, pos, kbase + half * kH + i)) vis |= 1ull << i;
-          else s[i] = neutral;
-        }
+        for (int i = 0; i < BN; ++i)
+          if (!key_visible(p, pos, kbase + i)) s[i] = neutral;
       }
       float mr[4];
 #pragma unroll
-      for (int t = 0; t < 4; ++t) mr[t] = s[t];
+      for (int q4 = 0; q4 < 4; ++q4) mr[q4] = s[q4];
       if (c_pos) {
 #pragma unroll
-        for (int i = 4; i < kH; i += 8) {
+        for (int i = 4; i < BN; i += 8) {
           mr[0] = fmax3f(mr[0], s[i], s[i + 1]);
           mr[1] = fmax3f(mr[1], s[i + 2], s[i + 3]);
-          if (i + 4 < kH) {
+          if (i + 4 < BN) {
             mr[2] = fmax3f(mr[2], s[i + 4], s[i + 5]);
             mr[3] = fmax3f(mr[3], s[i + 6], s[i + 7]);
           }
@@ -339,28 +325,17 @@ __global__ void __launch_bounds__(352, 1)
         mr[0] = fmax3f(mr[0], mr[1], fmaxf(mr[2], mr[3]));
       } else {
 #pragma unroll
-        for (int i = 4; i < kH; i += 8) {
+        for (int i = 4; i < BN; i += 8) {
           mr[0] = fmin3f(mr[0], s[i], s[i + 1]);
           mr[1] = fmin3f(mr[1], s[i + 2], s[i + 3]);
-          if (i + 4 < kH) {
+          if (i + 4 < BN) {
             mr[2] = fmin3f(mr[2], s[i + 4], s[i + 5]);
             mr[3] = fmin3f(mr[3], s[i + 6], s[i + 7]);
           }
         }
         mr[0] = fmin3f(mr[0], mr[1], fminf(mr[2], mr[3]));
       }
-      xmax[((j & 1) * 2 + half) * Cfg::kBM + r] = mr[0];
-      tc_fence_before();
-      mbar_arrive(&pair_bar[quarter]);
-      if (!mbar_wait(&pair_bar[quarter], pair_phase & 1u, p.wd, kWdSoftmax)) {
-        ok = false;
-        break;
-      }
-      ++pair_phase;
-      tc_fence_after();
-      const float other = xmax[((j & 1) * 2 + (half ^ 1)) * Cfg::kBM + r];
-      const float mraw = c_pos ? fmaxf(mr[0], other) : fminf(mr[0], other);
-      const float mblk = isinf(mraw) ? -INFINITY : mraw * c;
+      const float mblk = isinf(mr[0]) ? -INFINITY : mr[0] * c;
       const float m_new = fmaxf(m_used, mblk);
       const bool need = m_new > m_used + 8.0f;
       float alpha = 1.f;
@@ -370,8 +345,9 @@ __global__ void __launch_bounds__(352, 1)
         l *= alpha;
       }
       if (j > 0 && __any_sync(0xffffffffu, need)) {
-        // as in tc.cuh: S_j was issued after P_{j-2} V, and P_j V waits for
-        // p_full, so o_bar is in phase j-1 or j here
+        // S_j was issued after P_{j-2} V by the same thread, and P_j V waits
+        // for p_full: o_bar is in phase j-1 or j here.  The TMEM loads and
+        // stores are warp-wide, so the whole warp rescales its rows.
         if (lane == 0) w = mbar_wait_cluster(o_bar, (uint32_t)(j - 1) & 1u, p.wd, kWdMma);
         if (!__shfl_sync(0xffffffffu, (int)w, 0)) {
           ok = false;
@@ -379,7 +355,7 @@ __global__ void __launch_bounds__(352, 1)
         }
         tc_fence_after();
 #pragma unroll 1
-        for (int c16 = oc_begin; c16 < oc_end; ++c16) {
+        for (int c16 = 0; c16 < DV / 16; ++c16) {
           float o[16];
           tmem_ld16(tmem + lane_base + Cfg::kOCol + c16 * 16, o);
           tmem_wait_ld();
@@ -387,36 +363,34 @@ __global__ void __launch_bounds__(352, 1)
           for (int e = 0; e < 16; ++e) o[e] *= alpha;
           tmem_st16(tmem + lane_base + Cfg::kOCol + c16 * 16, o);
         }
-        tmem_wait_st();
       }
+      // ---- P = exp2(s c - m), row sum, P packed over the row's own scores ----
       const float mref = m_used == -INFINITY ? 0.f : m_used;
       const float2 c2 = make_float2(c, c), nm2 = make_float2(-mref, -mref);
       float2 acc[4];
 #pragma unroll
-      for (int t = 0; t < 4; ++t) acc[t] = make_float2(0.f, 0.f);
-      uint32_t pk[kH / 2];
+      for (int q4 = 0; q4 < 4; ++q4) acc[q4] = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int i = 0; i < kH; i += 2) {
-        float2 t = fma2(make_float2(s[i], s[i + 1]), c2, nm2);
-        if (((i >> 1) & 3) < SDPA_TC2_POLY_OF4) {
-          t = exp2_poly2(t);  // FMA / ALU pipes
-        } else {
-          t.x = fast_exp2(t.x);  // MUFU
-          t.y = fast_exp2(t.y);
+      for (int c32 = 0; c32 < BN / 32; ++c32) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i2 = 0; i2 < 16; ++i2) {
+          const int i = c32 * 32 + 2 * i2;
+          float2 t = fma2(make_float2(s[i], s[i + 1]), c2, nm2);
+          if ((i2 & 3) < SDPA_TC2_POLY_OF4) {
+            t = exp2_poly2(t);  // FMA / ALU pipes
+          } else {
+            t.x = fast_exp2(t.x);  // MUFU
+            t.y = fast_exp2(t.y);
+          }
+          acc[i2 & 3] = add2(acc[i2 & 3], t);
+          pk[i2] = pack2<kBF16>(t.x, t.y);
         }
-        if (masked) {
-          t.x = ((vis >> i) & 1ull) ? t.x : 0.f;
-          t.y = ((vis >> (i + 1)) & 1ull) ? t.y : 0.f;
-        }
-        acc[(i >> 1) & 3] = add2(acc[(i >> 1) & 3], t);
-        pk[i >> 1] = pack2<kBF16>(t.x, t.y);
+        tmem_st_u16x(tmem + lane_base + b * BN + c32 * 16, pk);
       }
       const float2 a01 = add2(acc[0], acc[1]), a23 = add2(acc[2], acc[3]);
       const float2 at = add2(a01, a23);
       l += at.x + at.y;
-#pragma unroll
-      for (int c16 = 0; c16 < kH / 32; ++c16)
-        tmem_st_u16x(tmem + lane_base + b * BN + half * (kH / 2) + c16 * 16, pk + c16 * 16);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -424,11 +398,6 @@ __global__ void __launch_bounds__(352, 1)
     }
 
     // ------------------------------ epilogue ------------------------------
-    float *xl = xmax + (nblk & 1) * 2 * Cfg::kBM;
-    xl[half * Cfg::kBM + r] = l;
-    mbar_arrive(&pair_bar[quarter]);
-    if (!mbar_wait(&pair_bar[quarter], pair_phase & 1u, p.wd, kWdSoftmax)) ok = false;
-    l += xl[(half ^ 1) * Cfg::kBM + r];
     if (ok && nblk > 0) {
       bool w = true;
       if (lane == 0) w = mbar_wait_cluster(o_final, 0, p.wd, kWdMma);
@@ -441,10 +410,10 @@ __global__ void __launch_bounds__(352, 1)
     float inv = l > 0.f ? 1.f / l : 0.f;
     if (p.splits == 1) {
       inv = finish_row(p, grow, m_used, l);
-      if (p.lse_out != nullptr && valid && half == 0) p.lse_out[grow] = row_lse(m_used, l);
+      if (p.lse_out != nullptr && valid) p.lse_out[grow] = row_lse(m_used, l);
       uint8_t *orow = reinterpret_cast<uint8_t *>(p.out) + grow * p.Dv * 2;
 #pragma unroll 1
-      for (int c16 = oc_begin; c16 < oc_end; ++c16) {
+      for (int c16 = 0; c16 < DV / 16; ++c16) {
         float o[16];
         if (have_o) {
           tmem_ld16(tmem + lane_base + Cfg::kOCol + c16 * 16, o);
@@ -466,7 +435,7 @@ __global__ void __launch_bounds__(352, 1)
       const long total_rows = (long)p.B * p.Hq * p.L;
       float *po = p.part_o + ((long)split * total_rows + grow) * p.Dv;
 #pragma unroll 1
-      for (int c16 = oc_begin; c16 < oc_end; ++c16) {
+      for (int c16 = 0; c16 < DV / 16; ++c16) {
         float o[16];
         if (have_o) {
           tmem_ld16(tmem + lane_base + Cfg::kOCol + c16 * 16, o);
@@ -484,7 +453,7 @@ __global__ void __launch_bounds__(352, 1)
                             o[q4 * 4 + 3] * inv);
         }
       }
-      if (valid && half == 0)
+      if (valid)
         p.part_lse[(long)split * total_rows + grow] = have_o ? row_lse(m_used, l) : -INFINITY;
     }
   }
@@ -502,7 +471,7 @@ __global__ void __launch_bounds__(352, 1)
     mbar_wait_cluster_drain(bye_bar, 0, p.wd);
   }
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 5) {
     tc_fence_after();
     tmem_dealloc_pair(tmem, Cfg::kTmemCols);
   }
