@@ -383,10 +383,11 @@ __device__ __forceinline__ float2 sub2(float2 a, float2 b) {
 // shifter (the integer lands in the low mantissa bits of x + shifter),
 // f = x - n in [-1/2, 1/2], 2^f by the degree-3 minimax polynomial of
 // exp2_poly.h, and n added to the exponent field.  x is clamped at -126 so
-// the exponent cannot wrap; results below 2^-126 come out as tiny normals or
-// denormals instead of zero.  Maximum relative error kExp2PolyMaxRelErr.
+// the exponent cannot wrap, and inputs below -126 (-inf included) give 0.
+// Maximum relative error kExp2PolyMaxRelErr.
 __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   const float2 shifter = make_float2(12582912.f, 12582912.f);
+  const bool zx = !(x.x >= -126.f), zy = !(x.y >= -126.f);
   x.x = fmaxf(x.x, -126.f);
   x.y = fmaxf(x.y, -126.f);
   const float2 t = add2(x, shifter);
@@ -395,8 +396,8 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   q = fma2(q, f, make_float2(kExp2C1, kExp2C1));
   q = fma2(q, f, make_float2(kExp2C0, kExp2C0));
   const int nx = __float_as_int(t.x) << 23, ny = __float_as_int(t.y) << 23;
-  return make_float2(__int_as_float(__float_as_int(q.x) + nx),
-                     __int_as_float(__float_as_int(q.y) + ny));
+  return make_float2(zx ? 0.f : __int_as_float(__float_as_int(q.x) + nx),
+                     zy ? 0.f : __int_as_float(__float_as_int(q.y) + ny));
 }
 __device__ __forceinline__ float fmax3f(float a, float b, float c) {
   float d;

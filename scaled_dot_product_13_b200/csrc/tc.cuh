@@ -7,11 +7,12 @@
 //   per-element masks run only on the diagonal, window-edge and tail blocks
 //   (mlx PR #3552, "Implementation").
 //
-// Warp roles (320 threads with the default two softmax warps per row):
+// Warp roles (192 threads with the default one softmax warp per row group):
 //   softmax    4 kParts warps: warps w, w+4, ... share query rows
 //              32(w%4) .. +31 (TMEM lanes), each taking 1/kParts of every
-//              key block's columns; they exchange their row maxima through
-//              shared memory behind a bounded mbarrier.  fp32 online softmax
+//              key block's columns; with kParts > 1 they exchange their row
+//              maxima through shared memory behind a bounded mbarrier (with
+//              one part a thread owns its whole row).  fp32 online softmax
 //              with a lazily updated running max.  P is rounded to the 16-bit
 //              input type and written back into tensor memory over the scores
 //              it came from.  At the end the epilogue (O / l, rounded,
@@ -42,11 +43,11 @@
 
 #include "params.cuh"
 
-// Softmax warps sharing one row of the tile (2 or 4), and how many of every
+// Softmax warps sharing one row of the tile (1, 2 or 4), and how many of every
 // four exponential pairs go to the FMA-pipe polynomial instead of the
 // MUFU ex2 unit (0-4).  Build-time knobs for measurement.
 #ifndef SDPA_TC_PARTS
-#define SDPA_TC_PARTS 2
+#define SDPA_TC_PARTS 1
 #endif
 #ifndef SDPA_TC_POLY_OF4
 #define SDPA_TC_POLY_OF4 0
@@ -296,6 +297,11 @@ __global__ void __launch_bounds__(TcCfg<DQK, DV, BN, NSLOT>::kThreads, 1)
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const int pos = ((tr.row0 + r) % p.L) + p.off;
     const float c = p.scale_log2;
+    // scale 0 weighs every visible key the same: the scores are zeroed and 1
+    // is used as the factor, so a masked key (set to the neutral value below)
+    // still gives exp2(-inf) = 0 and never exp2(-inf * 0) = NaN
+    const bool c_zero = p.scale_log2 == 0.f;
+    const float c_eff = c_zero ? 1.f : c;
     const bool c_pos = c >= 0.f;
     const float neutral = c_pos ? -INFINITY : INFINITY;  // never wins the row reduction
     constexpr int kH = Cfg::kCols;
@@ -328,16 +334,16 @@ __global__ void __launch_bounds__(TcCfg<DQK, DV, BN, NSLOT>::kThreads, 1)
       tmem_wait_ld();
 
       // ---- this part's raw row max (masked keys excluded) ----
+      if (c_zero) {
+#pragma unroll
+        for (int i = 0; i < kH; ++i) s[i] = 0.f;
+      }
       const int kbase = k_lo + j * BN;
       const bool masked = block_needs_mask(p, tr, kbase, BN);
-      uint64_t vis = ~0ull;
       if (masked) {
-        vis = 0ull;
 #pragma unroll
-        for (int i = 0; i < kH; ++i) {
-          if (key_visible(p, pos, kbase + part * kH + i)) vis |= 1ull << i;
-          else s[i] = neutral;
-        }
+        for (int i = 0; i < kH; ++i)
+          if (!key_visible(p, pos, kbase + part * kH + i)) s[i] = neutral;
       }
       float mr[4];
 #pragma unroll
@@ -368,22 +374,24 @@ __global__ void __launch_bounds__(TcCfg<DQK, DV, BN, NSLOT>::kThreads, 1)
       // ---- combine with the other parts of the row (bounded barrier).  The
       // barrier also orders every part's score reads before any part
       // overwrites them with P. ----
-      xmax[((j & 1) * kParts + part) * Cfg::kBM + r] = mr[0];
-      tc_fence_before();
-      mbar_arrive(&part_bar[quarter]);
-      if (!mbar_wait(&part_bar[quarter], part_phase & 1u, p.wd, kWdSoftmax)) {
-        ok = false;
-        break;
-      }
-      ++part_phase;
-      tc_fence_after();
       float mraw = mr[0];
+      if constexpr (kParts > 1) {
+        xmax[((j & 1) * kParts + part) * Cfg::kBM + r] = mr[0];
+        tc_fence_before();
+        mbar_arrive(&part_bar[quarter]);
+        if (!mbar_wait(&part_bar[quarter], part_phase & 1u, p.wd, kWdSoftmax)) {
+          ok = false;
+          break;
+        }
+        ++part_phase;
+        tc_fence_after();
 #pragma unroll
-      for (int q = 0; q < kParts; ++q) {
-        const float other = xmax[((j & 1) * kParts + q) * Cfg::kBM + r];
-        mraw = c_pos ? fmaxf(mraw, other) : fminf(mraw, other);
+        for (int q = 0; q < kParts; ++q) {
+          const float other = xmax[((j & 1) * kParts + q) * Cfg::kBM + r];
+          mraw = c_pos ? fmaxf(mraw, other) : fminf(mraw, other);
+        }
       }
-      const float mblk = isinf(mraw) ? -INFINITY : mraw * c;
+      const float mblk = isinf(mraw) ? -INFINITY : mraw * c_eff;
       const float m_new = fmaxf(m_used, mblk);
       const bool need = m_new > m_used + 8.0f;
       float alpha = 1.f;
@@ -419,7 +427,7 @@ __global__ void __launch_bounds__(TcCfg<DQK, DV, BN, NSLOT>::kThreads, 1)
       }
       // ---- P = exp2(s * c - m) (two lanes per FMA), row sums ----
       const float mref = m_used == -INFINITY ? 0.f : m_used;
-      const float2 c2 = make_float2(c, c), nm2 = make_float2(-mref, -mref);
+      const float2 c2 = make_float2(c_eff, c_eff), nm2 = make_float2(-mref, -mref);
       float2 acc[4];
 #pragma unroll
       for (int t = 0; t < 4; ++t) acc[t] = make_float2(0.f, 0.f);
@@ -432,10 +440,6 @@ __global__ void __launch_bounds__(TcCfg<DQK, DV, BN, NSLOT>::kThreads, 1)
         } else {
           t.x = fast_exp2(t.x);  // MUFU
           t.y = fast_exp2(t.y);
-        }
-        if (masked) {
-          t.x = ((vis >> i) & 1ull) ? t.x : 0.f;
-          t.y = ((vis >> (i + 1)) & 1ull) ? t.y : 0.f;
         }
         acc[(i >> 1) & 3] = add2(acc[(i >> 1) & 3], t);
         pk[i >> 1] = pack2<kBF16>(t.x, t.y);
@@ -461,13 +465,15 @@ __global__ void __launch_bounds__(TcCfg<DQK, DV, BN, NSLOT>::kThreads, 1)
     // ------------------------------ epilogue ------------------------------
     // row sum = the parts' partial sums, exchanged through the max buffer the
     // last block did not use (its last reader passed the last barrier)
-    float *xl = xmax + (nblk & 1) * kParts * Cfg::kBM;
-    xl[part * Cfg::kBM + r] = l;
-    mbar_arrive(&part_bar[quarter]);
-    if (!mbar_wait(&part_bar[quarter], part_phase & 1u, p.wd, kWdSoftmax)) ok = false;
-    l = 0.f;
+    if constexpr (kParts > 1) {
+      float *xl = xmax + (nblk & 1) * kParts * Cfg::kBM;
+      xl[part * Cfg::kBM + r] = l;
+      mbar_arrive(&part_bar[quarter]);
+      if (!mbar_wait(&part_bar[quarter], part_phase & 1u, p.wd, kWdSoftmax)) ok = false;
+      l = 0.f;
 #pragma unroll
-    for (int q = 0; q < kParts; ++q) l += xl[q * Cfg::kBM + r];
+      for (int q = 0; q < kParts; ++q) l += xl[q * Cfg::kBM + r];
+    }
     if (ok && nblk > 0) {
       bool w = true;
       if (lane == 0) w = mbar_wait(o_final, 0, p.wd, kWdMma);

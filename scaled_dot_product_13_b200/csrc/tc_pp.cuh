@@ -280,6 +280,11 @@ __global__ void __launch_bounds__(320, 1)
     }
     const int pos = ((tr.row0 + r) % p.L) + p.off;
     const float c = p.scale_log2;
+    // scale 0 weighs every visible key the same: the scores are zeroed and 1
+    // is used as the factor, so a masked key (set to the neutral value below)
+    // still gives exp2(-inf) = 0 and never exp2(-inf * 0) = NaN
+    const bool c_zero = p.scale_log2 == 0.f;
+    const float c_eff = c_zero ? 1.f : c;
     const bool c_pos = c >= 0.f;
     const float neutral = c_pos ? -INFINITY : INFINITY;
     float m_used = -INFINITY, l = 0.f;
@@ -298,6 +303,10 @@ __global__ void __launch_bounds__(320, 1)
         tmem_ld32(tmem + lane_base + s_col + c32 * 32, s + c32 * 32);
       tmem_wait_ld();
 
+      if (c_zero) {
+#pragma unroll
+        for (int i = 0; i < BN; ++i) s[i] = 0.f;
+      }
       const int kbase = k_lo + j * BN;
       const bool masked = block_needs_mask(p, tr, kbase, BN);
       if (masked) {
@@ -331,7 +340,7 @@ __global__ void __launch_bounds__(320, 1)
         }
         mr[0] = fmin3f(mr[0], mr[1], fminf(mr[2], mr[3]));
       }
-      const float mblk = isinf(mr[0]) ? -INFINITY : mr[0] * c;
+      const float mblk = isinf(mr[0]) ? -INFINITY : mr[0] * c_eff;
       const float m_new = fmaxf(m_used, mblk);
       const bool need = m_new > m_used + 8.0f;
       float alpha = 1.f;
@@ -357,7 +366,7 @@ __global__ void __launch_bounds__(320, 1)
       }
       // ---- P = exp2(s c - m), row sum, packed P over this row's scores ----
       const float mref = m_used == -INFINITY ? 0.f : m_used;
-      const float2 c2 = make_float2(c, c), nm2 = make_float2(-mref, -mref);
+      const float2 c2 = make_float2(c_eff, c_eff), nm2 = make_float2(-mref, -mref);
       float2 acc[4];
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) acc[q4] = make_float2(0.f, 0.f);

@@ -93,3 +93,9 @@ def test_tc2_many_waves(cuda_lib, case):
     _, _, info = check_problem(cuda_lib, p, rows=rows, force_path=S.PATH_TC2, force_splits=fs)
     assert info["path"] == S.PATH_TC2
     assert info["ctas"] > 74
+
+
+@pytest.mark.parametrize("scale", [-0.05, 0.0, 0.3])
+def test_tc2_unusual_scales(cuda_lib, scale):
+    p = I.Problem(1, 4, 2, 300, 450, 256, 256, "bf16", True, 100, scale, 46, "tc2_scales")
+    check_problem(cuda_lib, p, force_path=S.PATH_TC2)

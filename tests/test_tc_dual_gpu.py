@@ -70,3 +70,11 @@ def test_tc_dual_agrees_with_tc(cuda_lib, case):
     a = run_gpu(cuda_lib, p, q, k, v, force_path=S.PATH_TC_DUAL)[0].float()
     b = run_gpu(cuda_lib, p, q, k, v, force_path=S.PATH_TC)[0].float()
     assert agree(a, b, dt)
+
+
+@pytest.mark.parametrize("scale", [-0.09, 0.0, 0.5])
+def test_tc_dual_unusual_scales(cuda_lib, scale):
+    # a negative scale flips which score is the row max; zero weighs every
+    # visible key the same (masked keys must still get weight 0, not NaN)
+    p = I.Problem(1, 4, 2, 300, 420, 64, 64, "bf16", True, 0, scale, 65, "dual_scales")
+    check_problem(cuda_lib, p, force_path=S.PATH_TC_DUAL)
