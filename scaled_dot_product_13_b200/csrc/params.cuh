@@ -109,4 +109,26 @@ __device__ __forceinline__ bool key_visible(const AttnParams &p, int pos, int co
   return col < p.S && (!p.causal || col <= pos) && (p.window == 0 || pos - col < p.window);
 }
 
+// The keys a row at position pos sees form one interval [lo, hi): the window
+// bounds it from below, causality and S from above.  Relative to a block
+// starting at key kbase, key kbase + i is visible iff
+// (unsigned)(i - (lo - kbase)) < (unsigned)(hi - lo): one subtraction and
+// one comparison per key instead of key_visible's three tests.
+struct VisibleRange {
+  int first;      // lo - kbase
+  unsigned span;  // hi - lo (0 when nothing is visible)
+  __device__ __forceinline__ bool operator()(int i) const {
+    return (unsigned)(i - first) < span;
+  }
+};
+
+__device__ __forceinline__ VisibleRange visible_range(const AttnParams &p, int pos, int kbase) {
+  const int lo = p.window > 0 ? max(0, pos - p.window + 1) : 0;
+  const int hi = p.causal ? min(p.S, pos + 1) : p.S;
+  VisibleRange v;
+  v.first = lo - kbase;
+  v.span = hi > lo ? (unsigned)(hi - lo) : 0u;
+  return v;
+}
+
 }  // namespace sdpa

@@ -341,9 +341,10 @@ __global__ void __launch_bounds__(TcCfg<DQK, DV, BN, NSLOT>::kThreads, 1)
       const int kbase = k_lo + j * BN;
       const bool masked = block_needs_mask(p, tr, kbase, BN);
       if (masked) {
+        const VisibleRange vis = visible_range(p, pos, kbase + part * kH);
 #pragma unroll
         for (int i = 0; i < kH; ++i)
-          if (!key_visible(p, pos, kbase + part * kH + i)) s[i] = neutral;
+          if (!vis(i)) s[i] = neutral;
       }
       float mr[4];
 #pragma unroll

@@ -314,9 +314,10 @@ __global__ void __launch_bounds__(224, 1)
       const int kbase = k_lo + j * BN;
       const bool masked = block_needs_mask(p, tr, kbase, BN);
       if (masked) {
+        const VisibleRange vis = visible_range(p, pos, kbase);
 #pragma unroll
         for (int i = 0; i < BN; ++i)
-          if (!key_visible(p, pos, kbase + i)) s[i] = neutral;
+          if (!vis(i)) s[i] = neutral;
       }
       float mr[4];
 #pragma unroll
