@@ -119,9 +119,13 @@ sdpa_status launch_combine(const Launch &ln, std::string *err) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const bool bf16 = ln.pb.dtype == SDPA_BF16, four = ln.pb.Dv > 256;
-  auto kern = bf16 ? (four ? combine_kernel<true, 4> : combine_kernel<true, 2>)
-                   : (four ? combine_kernel<false, 4> : combine_kernel<false, 2>);
+  // output columns per thread: Dv <= 128, <= 256, <= 512
+  const bool bf16 = ln.pb.dtype == SDPA_BF16;
+  const int nc = ln.pb.Dv <= 128 ? 1 : ln.pb.Dv <= 256 ? 2 : 4;
+  auto kern = bf16 ? (nc == 1 ? combine_kernel<true, 1>
+                              : nc == 2 ? combine_kernel<true, 2> : combine_kernel<true, 4>)
+                   : (nc == 1 ? combine_kernel<false, 1>
+                              : nc == 2 ? combine_kernel<false, 2> : combine_kernel<false, 4>);
   cudaError_t e = cudaLaunchKernelEx(&cfg, kern, (const float *)ln.part_o,
                                      (const float *)ln.part_lse, ln.out, ln.lse_out, ln.sinks,
                                      total, ln.pb.Dv, ln.plan.splits, ln.pb.L, ln.pb.Hq);
