@@ -330,16 +330,6 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    dist = None
-    if world > 1:
-        import torch.distributed as dist  # noqa: F811
-        import datetime
-
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
-    device = torch.device("cuda", local)
-    torch.cuda.set_device(device)
-
     probs = I.decode_problems()
     if args.only:
         probs = [p for p in probs + I.verify_problems() + I.window_problems() +
@@ -379,9 +369,19 @@ def main():
                     "e2e": {"value": round(val, 4), "unit": "GB/s (KV, decode)",
                             "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
             print(json.dumps(line), flush=True)
-        if dist is not None:
-            dist.destroy_process_group()
+        # the oracle runs on the host: no device and no process group are
+        # needed, and ranks other than 0 exit without work
         return
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist  # noqa: F811
+        import datetime
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
 
     import scaled_dot_product_13_b200 as sdpa
 
