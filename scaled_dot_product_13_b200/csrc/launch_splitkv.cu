@@ -2,6 +2,7 @@
 #include <cmath>
 
 #include "launch.h"
+#include "combine.cuh"
 #include "splitkv.cuh"
 
 namespace sdpa {
@@ -110,7 +111,7 @@ sdpa_status launch_combine(const Launch &ln, std::string *err) {
   // it, which hides the second launch's latency.
   const long total = (long)ln.pb.B * ln.pb.Hq * ln.pb.L;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)total);
+  cfg.gridDim = dim3((unsigned)total, (unsigned)((ln.pb.Dv + 127) / 128));
   cfg.blockDim = dim3(128);
   cfg.dynamicSmemBytes = (size_t)ln.plan.splits * sizeof(float);
   cfg.stream = ln.stream;
@@ -119,13 +120,7 @@ sdpa_status launch_combine(const Launch &ln, std::string *err) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  // output columns per thread: Dv <= 128, <= 256, <= 512
-  const bool bf16 = ln.pb.dtype == SDPA_BF16;
-  const int nc = ln.pb.Dv <= 128 ? 1 : ln.pb.Dv <= 256 ? 2 : 4;
-  auto kern = bf16 ? (nc == 1 ? combine_kernel<true, 1>
-                              : nc == 2 ? combine_kernel<true, 2> : combine_kernel<true, 4>)
-                   : (nc == 1 ? combine_kernel<false, 1>
-                              : nc == 2 ? combine_kernel<false, 2> : combine_kernel<false, 4>);
+  auto kern = ln.pb.dtype == SDPA_BF16 ? combine_kernel<true> : combine_kernel<false>;
   cudaError_t e = cudaLaunchKernelEx(&cfg, kern, (const float *)ln.part_o,
                                      (const float *)ln.part_lse, ln.out, ln.lse_out, ln.sinks,
                                      total, ln.pb.Dv, ln.plan.splits, ln.pb.L, ln.pb.Hq);

@@ -417,51 +417,63 @@ __global__ void __launch_bounds__(224, 1)
     const bool valid = r < tr.nvalid;
     const long grow = (long)bh * p.R + tr.row0 + r;
     const bool have_o = ok && nblk > 0;
+    // O leaves TMEM kOGroup chunks of 16 columns per wait
+    constexpr int kOChunks = DV / 16;
+    constexpr int kOGroup = kOChunks <= 5 ? kOChunks : 4;
+    static_assert(kOChunks % kOGroup == 0, "whole groups of O chunks");
+    auto load_o = [&](int g, float (&o)[kOGroup][16]) {
+      if (have_o) {
+    #pragma unroll
+        for (int k = 0; k < kOGroup; ++k)
+          tmem_ld16(tmem + lane_base + Cfg::kOCol + (g * kOGroup + k) * 16, o[k]);
+        tmem_wait_ld();
+      } else {
+    #pragma unroll
+        for (int k = 0; k < kOGroup; ++k)
+    #pragma unroll
+          for (int e = 0; e < 16; ++e) o[k][e] = 0.f;
+      }
+    };
     float inv = l > 0.f ? 1.f / l : 0.f;
     if (p.splits == 1) {
       inv = finish_row(p, grow, m_used, l);
       if (p.lse_out != nullptr && valid) p.lse_out[grow] = row_lse(m_used, l);
       uint8_t *orow = reinterpret_cast<uint8_t *>(p.out) + grow * p.Dv * 2;
 #pragma unroll 1
-      for (int c16 = 0; c16 < DV / 16; ++c16) {
-        float o[16];
-        if (have_o) {
-          tmem_ld16(tmem + lane_base + Cfg::kOCol + c16 * 16, o);
-          tmem_wait_ld();
-        } else {
+      for (int g = 0; g < kOChunks / kOGroup; ++g) {
+        float o[kOGroup][16];
+        load_o(g, o);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) o[e] = 0.f;
+        for (int k = 0; k < kOGroup; ++k) {
+          uint32_t w8[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            w8[e] = pack2<kBF16>(o[k][2 * e] * inv, o[k][2 * e + 1] * inv);
+          const int col = (g * kOGroup + k) * 16;
+          if (valid && col + 8 <= p.Dv)
+            *reinterpret_cast<uint4 *>(orow + col * 2) = make_uint4(w8[0], w8[1], w8[2], w8[3]);
+          if (valid && col + 16 <= p.Dv)
+            *reinterpret_cast<uint4 *>(orow + col * 2 + 16) =
+                make_uint4(w8[4], w8[5], w8[6], w8[7]);
         }
-        uint32_t w8[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) w8[e] = pack2<kBF16>(o[2 * e] * inv, o[2 * e + 1] * inv);
-        const int col = c16 * 16;
-        if (valid && col + 8 <= p.Dv)
-          *reinterpret_cast<uint4 *>(orow + col * 2) = make_uint4(w8[0], w8[1], w8[2], w8[3]);
-        if (valid && col + 16 <= p.Dv)
-          *reinterpret_cast<uint4 *>(orow + col * 2 + 16) = make_uint4(w8[4], w8[5], w8[6], w8[7]);
       }
     } else {
       const long total_rows = (long)p.B * p.Hq * p.L;
       float *po = p.part_o + ((long)split * total_rows + grow) * p.Dv;
 #pragma unroll 1
-      for (int c16 = 0; c16 < DV / 16; ++c16) {
-        float o[16];
-        if (have_o) {
-          tmem_ld16(tmem + lane_base + Cfg::kOCol + c16 * 16, o);
-          tmem_wait_ld();
-        } else {
+      for (int g = 0; g < kOChunks / kOGroup; ++g) {
+        float o[kOGroup][16];
+        load_o(g, o);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) o[e] = 0.f;
-        }
+        for (int k = 0; k < kOGroup; ++k)
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const int col = c16 * 16 + q4 * 4;
-          if (valid && col + 4 <= p.Dv)
-            *reinterpret_cast<float4 *>(po + col) =
-                make_float4(o[q4 * 4] * inv, o[q4 * 4 + 1] * inv, o[q4 * 4 + 2] * inv,
-                            o[q4 * 4 + 3] * inv);
-        }
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const int col = (g * kOGroup + k) * 16 + q4 * 4;
+            if (valid && col + 4 <= p.Dv)
+              *reinterpret_cast<float4 *>(po + col) =
+                  make_float4(o[k][q4 * 4] * inv, o[k][q4 * 4 + 1] * inv, o[k][q4 * 4 + 2] * inv,
+                              o[k][q4 * 4 + 3] * inv);
+          }
       }
       if (valid)
         p.part_lse[(long)split * total_rows + grow] = have_o ? row_lse(m_used, l) : -INFINITY;
