@@ -13,6 +13,11 @@
 
 #include "params.cuh"
 
+// splits loaded per round trip to L2 after the first kPre
+#ifndef SDPA_COMBINE_BATCH
+#define SDPA_COMBINE_BATCH 8
+#endif
+
 namespace sdpa {
 
 template <bool kBF16>
@@ -69,15 +74,17 @@ __global__ void __launch_bounds__(128) combine_kernel(const float *__restrict__ 
   for (int t = 0; t < kPre; ++t)
     if (t < splits) acc += s_w[t] * v[t];
   // the remaining splits, kBatch per round trip to L2
-  constexpr int kBatch = 16;
+  constexpr int kBatch = SDPA_COMBINE_BATCH;
   for (int s0 = kPre; s0 < splits; s0 += kBatch) {
     float x[kBatch];
 #pragma unroll
     for (int t = 0; t < kBatch; ++t)
       x[t] = (s0 + t < splits && live) ? __ldcg(src + (long)(s0 + t) * stride) : 0.f;
 #pragma unroll
-    for (int t = 0; t < kBatch; ++t)
-      if (s0 + t < splits) acc += s_w[s0 + t] * x[t];
+    for (int t = 0; t < kBatch; ++t) {
+      const float w = s0 + t < splits ? s_w[s0 + t] : 0.f;
+      acc += w * x[t];
+    }
   }
   if (live) {
     const float o = acc * s_res[0];

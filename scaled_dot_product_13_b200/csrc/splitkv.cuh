@@ -21,6 +21,10 @@
 
 #include "params.cuh"
 
+#ifndef SDPA_SK_SPLITACC
+#define SDPA_SK_SPLITACC 0
+#endif
+
 namespace sdpa {
 
 template <int DQK, int DV, int BN, int WR, int WK, int NST>
@@ -162,6 +166,12 @@ __global__ void __launch_bounds__(SplitKvCfg<DQK, DV, BN, WR, WK, NST>::kThreads
     float sc[kNT][4];
 #pragma unroll
     for (int i = 0; i < kNT; ++i) sc[i][0] = sc[i][1] = sc[i][2] = sc[i][3] = 0.f;
+#if SDPA_SK_SPLITACC
+    // odd k16 steps accumulate separately: two dependent chains of half the length
+    float sc2[kNT][4];
+#pragma unroll
+    for (int i = 0; i < kNT; ++i) sc2[i][0] = sc2[i][1] = sc2[i][2] = sc2[i][3] = 0.f;
+#endif
 #pragma unroll
     for (int ks = 0; ks < kKS; ++ks) {
       uint32_t a0, a1, a2, a3;
@@ -179,10 +189,23 @@ __global__ void __launch_bounds__(SplitKvCfg<DQK, DV, BN, WR, WK, NST>::kThreads
         const uint32_t chunk = ks * 2 + (m & 1);
         uint32_t b0, b1, b2, b3;
         ldsm_x4(sK + (chunk >> 3) * (BN * 128) + sw128_offset(key, chunk & 7), b0, b1, b2, b3);
+#if SDPA_SK_SPLITACC
+        if (ks & 1) {
+          mma_16816<kBF16>(sc2[2 * n2], a0, a1, a2, a3, b0, b1);
+          mma_16816<kBF16>(sc2[2 * n2 + 1], a0, a1, a2, a3, b2, b3);
+          continue;
+        }
+#endif
         mma_16816<kBF16>(sc[2 * n2], a0, a1, a2, a3, b0, b1);
         mma_16816<kBF16>(sc[2 * n2 + 1], a0, a1, a2, a3, b2, b3);
       }
     }
+#if SDPA_SK_SPLITACC
+#pragma unroll
+    for (int i = 0; i < kNT; ++i)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sc[i][e] += sc2[i][e];
+#endif
 
     // ---- scale into the log2 domain, mask, online softmax ----
 #pragma unroll
