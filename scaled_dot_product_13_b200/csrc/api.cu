@@ -259,16 +259,22 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
   // CTAs per split: one per row tile, two per pair tile
   const long long per_tile = pl.path == SDPA_PATH_TC2 ? 2 : 1;
   const long long base = (long long)pb.B * pb.Hkv * pl.row_tiles * per_tile;
+  // resident CTAs per SM (the split-KV kernel runs two where they fit)
+  const long long slots =
+      (long long)num_sms * (path == SDPA_PATH_SPLITKV
+                                ? splitkv_ctas_per_sm(kDimPairs[pl.pair].dqk,
+                                                      kDimPairs[pl.pair].dv, pl.wr)
+                                : 1);
   int splits;
   if (force_splits > 0) {
     splits = std::min(force_splits, nkb);
-  } else if (base >= num_sms || nkb <= kNoSplitBlocks) {
+  } else if (base >= slots || nkb <= kNoSplitBlocks) {
     splits = 1;
   } else {
     // the wide kernel's 32-key blocks are small and its partials wide
     // (Dv up to 512 floats per row and split): give each split more keys
     const int min_blocks = path == SDPA_PATH_WIDE ? kMinBlocksPerSplitWide : kMinBlocksPerSplit;
-    splits = (int)std::max(1LL, num_sms / base);
+    splits = (int)std::max(1LL, slots / base);
     splits = std::min(splits, std::max(1, nkb / min_blocks));
   }
   splits = std::min(splits, kMaxSplits);

@@ -4,9 +4,10 @@
 //   LSE = max_s LSE_s + ln sum_s exp(LSE_s - max),  O = sum_s exp(LSE_s - LSE) O_s
 // Splits that saw no visible key carry LSE_s = -inf and weight 0.  A head's
 // sink (when given) joins as one more term with weight exp(sink - LSE) and
-// no value row.  Warp 0 forms the weights in shared memory while every
-// thread already has its column's partials of the first splits in flight;
-// after one barrier each thread accumulates its output column.
+// no value row.  Every thread loads its column's partials of the first 64
+// splits and one split LSE in the same round trip to L2; two block
+// reductions (max, then the weight sum) form the weights in shared memory,
+// and each thread accumulates its output column.
 // Launched as a programmatic dependent of the split pass: it waits for that
 // grid (griddepcontrol.wait) before touching the partials.
 #pragma once
@@ -27,53 +28,55 @@ __global__ void __launch_bounds__(128) combine_kernel(const float *__restrict__ 
                                                       const float *__restrict__ sinks,
                                                       long total_rows, int Dv, int splits, int L,
                                                       int Hq) {
-  extern __shared__ float s_w[];  // [splits]
-  __shared__ float s_res[2];      // 1 / denominator, LSE
-  constexpr int kPre = 32;        // splits whose partials are loaded before the weights exist
+  extern __shared__ float s_w[];  // [splits]: the split LSEs, then their weights
+  __shared__ float s_red[2][4];   // per-warp max, per-warp weight sum
+  constexpr int kPre = 64;        // splits whose partials go out in the first round trip
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const long row = blockIdx.x;
-  const int tid = threadIdx.x, lane = tid & 31;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int col = blockIdx.y * 128 + tid;  // this thread's output column
   const bool live = col < Dv;
   const long stride = total_rows * Dv;
   const float *src = part_o + row * Dv + col;
-  // the partial loads go out first, in flight while warp 0 forms the weights
+  // One round trip to L2: each thread's partials of the first kPre splits and
+  // one split LSE per thread (up to 128 splits; more take further rounds).
   float v[kPre];
 #pragma unroll
   for (int t = 0; t < kPre; ++t) v[t] = (t < splits && live) ? __ldcg(src + (long)t * stride) : 0.f;
-  if (tid < 32) {
-    // warp 0: max of the split LSEs (and the sink), weights, denominator
-    float mx = -INFINITY;
-    for (int s = lane; s < splits; s += 32) {
-      const float x = __ldcg(part_lse + (long)s * total_rows + row);
-      s_w[s] = x;
-      mx = fmaxf(mx, x);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    const float sink = sinks != nullptr ? sinks[(int)((row / L) % Hq)] : -INFINITY;
-    mx = fmaxf(mx, sink);
-    const float ref = mx == -INFINITY ? 0.f : mx;
-    float den = 0.f;
-    for (int s = lane; s < splits; s += 32) {  // each lane rereads its own entries
-      const float w = __expf(s_w[s] - ref);
-      s_w[s] = w;
-      den += w;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-    if (sinks != nullptr) den += __expf(sink - ref);
-    if (lane == 0) {
-      s_res[0] = den > 0.f ? 1.f / den : 0.f;
-      s_res[1] = den > 0.f ? ref + logf(den) : -INFINITY;
-    }
+  float mx = -INFINITY;
+  for (int s = tid; s < splits; s += 128) {
+    const float x = __ldcg(part_lse + (long)s * total_rows + row);
+    s_w[s] = x;
+    mx = fmaxf(mx, x);
   }
+  // block max of the split LSEs and the sink
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if (lane == 0) s_red[0][warp] = mx;
   __syncthreads();
+  const float sink = sinks != nullptr ? sinks[(int)((row / L) % Hq)] : -INFINITY;
+  mx = fmaxf(fmaxf(fmaxf(s_red[0][0], s_red[0][1]), fmaxf(s_red[0][2], s_red[0][3])), sink);
+  const float ref = mx == -INFINITY ? 0.f : mx;
+  // weights exp(LSE_s - ref); each thread rereads the entries it wrote
+  float den = 0.f;
+  for (int s = tid; s < splits; s += 128) {
+    const float w = __expf(s_w[s] - ref);
+    s_w[s] = w;
+    den += w;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+  if (lane == 0) s_red[1][warp] = den;
+  __syncthreads();
+  den = (s_red[1][0] + s_red[1][1]) + (s_red[1][2] + s_red[1][3]);
+  if (sinks != nullptr) den += __expf(sink - ref);
   float acc = 0.f;
 #pragma unroll
-  for (int t = 0; t < kPre; ++t)
-    if (t < splits) acc += s_w[t] * v[t];
-  // the remaining splits, kBatch per round trip to L2
+  for (int t = 0; t < kPre; ++t) {
+    const float w = t < splits ? s_w[t] : 0.f;
+    acc += w * v[t];
+  }
+  // splits past kPre, kBatch per round trip
   constexpr int kBatch = SDPA_COMBINE_BATCH;
   for (int s0 = kPre; s0 < splits; s0 += kBatch) {
     float x[kBatch];
@@ -87,13 +90,14 @@ __global__ void __launch_bounds__(128) combine_kernel(const float *__restrict__ 
     }
   }
   if (live) {
-    const float o = acc * s_res[0];
+    const float o = den > 0.f ? acc / den : 0.f;
     if constexpr (kBF16)
       reinterpret_cast<__nv_bfloat16 *>(out)[row * Dv + col] = __float2bfloat16_rn(o);
     else
       reinterpret_cast<__half *>(out)[row * Dv + col] = __float2half_rn(o);
   }
-  if (lse_out != nullptr && blockIdx.y == 0 && tid == 0) lse_out[row] = s_res[1];
+  if (lse_out != nullptr && blockIdx.y == 0 && tid == 0)
+    lse_out[row] = den > 0.f ? ref + logf(den) : -INFINITY;
 }
 
 }  // namespace sdpa

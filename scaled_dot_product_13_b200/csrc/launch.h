@@ -30,6 +30,33 @@ constexpr int kWideBN = 32;
 // Key block of the split-KV kernel (keys per pipeline stage).
 constexpr int kSplitKvBN = 64;
 
+// Split-KV shared memory: one Q tile of 16*wr rows plus a ring of K/V stages
+// (64-column TMA boxes of 128 bytes per row).  With two CTAs per SM each gets
+// half of the SM's 228 KB less the 1 KB the hardware reserves per CTA; the
+// budgets keep 2 KB for barriers, alignment slack and static shared memory.
+#ifndef SDPA_SK_TWO_PER_SM
+#define SDPA_SK_TWO_PER_SM 0
+#endif
+constexpr unsigned kSplitKvBudget1 = 232448u - 2048u;
+constexpr unsigned kSplitKvBudget2 = 233472u / 2 - 1024u - 2048u;
+constexpr unsigned splitkv_stage_bytes(int dqk, int dv) {
+  return (unsigned)(((dqk + 63) / 64 + (dv + 63) / 64) * kSplitKvBN * 128);
+}
+constexpr unsigned splitkv_q_bytes(int dqk, int wr) {
+  return (unsigned)(((dqk + 63) / 64) * 16 * wr * 128);
+}
+// Stages that fit the budget next to Q, at most 4.
+constexpr int splitkv_stages(int dqk, int dv, int wr, unsigned budget) {
+  return (int)((budget - splitkv_q_bytes(dqk, wr)) / splitkv_stage_bytes(dqk, dv)) > 4
+             ? 4
+             : (int)((budget - splitkv_q_bytes(dqk, wr)) / splitkv_stage_bytes(dqk, dv));
+}
+// CTAs of one instance resident per SM: two where double buffering fits half
+// the SM's shared memory, else one.
+constexpr int splitkv_ctas_per_sm(int dqk, int dv, int wr) {
+  return SDPA_SK_TWO_PER_SM && splitkv_stages(dqk, dv, wr, kSplitKvBudget2) >= 2 ? 2 : 1;
+}
+
 // Key block of the tcgen05 kernel: 128 keys while two 128-key score buffers
 // plus O fit TMEM and the slots fit shared memory; 64 for head dims > 128.
 constexpr int tc_key_block(int dqk, int dv) { return (dqk > 128 || dv > 128) ? 64 : 128; }

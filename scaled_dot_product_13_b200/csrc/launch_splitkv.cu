@@ -12,15 +12,14 @@ namespace {
 template <bool kBF16, int DQK, int DV, int WR, int WK>
 sdpa_status run_splitkv(const Launch &ln, std::string *err) {
   constexpr int kBN = kSplitKvBN;
-  // stages: as many as fit next to Q in 227 KB, at most 4
-  constexpr uint32_t kStage = ((DQK + 63) / 64 + (DV + 63) / 64) * kBN * 128;
-  constexpr uint32_t kQ = ((DQK + 63) / 64) * 16 * WR * 128;
-  constexpr uint32_t kBudget = 232448u - 2048u;
-  constexpr int kFit = (int)((kBudget - kQ) / kStage);
-  constexpr int kNST = kFit > 4 ? 4 : kFit;
+  // one or two CTAs per SM; stages: as many as fit next to Q, at most 4
+  constexpr int kMinB = splitkv_ctas_per_sm(DQK, DV, WR);
+  constexpr int kNST =
+      splitkv_stages(DQK, DV, WR, kMinB == 2 ? kSplitKvBudget2 : kSplitKvBudget1);
   static_assert(kNST >= 2, "at least double buffering");
   using Cfg = SplitKvCfg<DQK, DV, kBN, WR, WK, kNST>;
-  auto kern = splitkv_kernel<kBF16, DQK, DV, kBN, WR, WK, kNST>;
+  static_assert(kMinB == 1 || Cfg::kSmemBytes + 1024 <= 233472u / 2, "two CTAs per SM");
+  auto kern = splitkv_kernel<kBF16, DQK, DV, kBN, WR, WK, kNST, kMinB>;
   sdpa_status st = prepare_kernel((const void *)kern, Cfg::kThreads, Cfg::kSmemBytes,
                                   "splitkv_kernel", err);
   if (st != SDPA_OK) return st;

@@ -21,10 +21,6 @@
 
 #include "params.cuh"
 
-#ifndef SDPA_SK_SPLITACC
-#define SDPA_SK_SPLITACC 0
-#endif
-
 namespace sdpa {
 
 template <int DQK, int DV, int BN, int WR, int WK, int NST>
@@ -40,10 +36,12 @@ struct SplitKvCfg {
   static constexpr uint32_t kVBytes = kVBoxes * BN * 128;
   static constexpr uint32_t kStageBytes = kKBytes + kVBytes;
   static constexpr uint32_t kRingBytes = NST * kStageBytes;
-  // merge buffer (reuses the ring): per consumer warp, O fragments + m + l
-  static constexpr uint32_t kMergeBytes = kConsumers * 32 * (DV / 2 + 4) * 4;
+  // output staging (reuses the ring): per key slice, the CTA's rows in fp32,
+  // each padded by 8 floats so the fragment stores spread over the banks
+  static constexpr int kOutStride = DV + 8;
+  static constexpr uint32_t kOutBytes = WK * kRT * kOutStride * 4;
   static constexpr uint32_t kBarOffset =
-      kQBytes + (kRingBytes > kMergeBytes ? kRingBytes : kMergeBytes);
+      kQBytes + (kRingBytes > kOutBytes ? kRingBytes : kOutBytes);
   static constexpr uint32_t kSmemBytes = kBarOffset + (2 * NST + 1) * 8 + 1024;  // + align slack
   static_assert(DQK % 16 == 0 && DV % 16 == 0, "head dims padded to 16");
   static_assert(kKW % 16 == 0, "each warp takes whole 16-key chunks");
@@ -51,8 +49,8 @@ struct SplitKvCfg {
   static_assert((kRT * 128) % 1024 == 0 && (BN * 128) % 1024 == 0, "swizzle atoms");
 };
 
-template <bool kBF16, int DQK, int DV, int BN, int WR, int WK, int NST>
-__global__ void __launch_bounds__(SplitKvCfg<DQK, DV, BN, WR, WK, NST>::kThreads, 1)
+template <bool kBF16, int DQK, int DV, int BN, int WR, int WK, int NST, int MINB>
+__global__ void __launch_bounds__(SplitKvCfg<DQK, DV, BN, WR, WK, NST>::kThreads, MINB)
     splitkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   using Cfg = SplitKvCfg<DQK, DV, BN, WR, WK, NST>;
@@ -166,12 +164,6 @@ __global__ void __launch_bounds__(SplitKvCfg<DQK, DV, BN, WR, WK, NST>::kThreads
     float sc[kNT][4];
 #pragma unroll
     for (int i = 0; i < kNT; ++i) sc[i][0] = sc[i][1] = sc[i][2] = sc[i][3] = 0.f;
-#if SDPA_SK_SPLITACC
-    // odd k16 steps accumulate separately: two dependent chains of half the length
-    float sc2[kNT][4];
-#pragma unroll
-    for (int i = 0; i < kNT; ++i) sc2[i][0] = sc2[i][1] = sc2[i][2] = sc2[i][3] = 0.f;
-#endif
 #pragma unroll
     for (int ks = 0; ks < kKS; ++ks) {
       uint32_t a0, a1, a2, a3;
@@ -189,23 +181,10 @@ __global__ void __launch_bounds__(SplitKvCfg<DQK, DV, BN, WR, WK, NST>::kThreads
         const uint32_t chunk = ks * 2 + (m & 1);
         uint32_t b0, b1, b2, b3;
         ldsm_x4(sK + (chunk >> 3) * (BN * 128) + sw128_offset(key, chunk & 7), b0, b1, b2, b3);
-#if SDPA_SK_SPLITACC
-        if (ks & 1) {
-          mma_16816<kBF16>(sc2[2 * n2], a0, a1, a2, a3, b0, b1);
-          mma_16816<kBF16>(sc2[2 * n2 + 1], a0, a1, a2, a3, b2, b3);
-          continue;
-        }
-#endif
         mma_16816<kBF16>(sc[2 * n2], a0, a1, a2, a3, b0, b1);
         mma_16816<kBF16>(sc[2 * n2 + 1], a0, a1, a2, a3, b2, b3);
       }
     }
-#if SDPA_SK_SPLITACC
-#pragma unroll
-    for (int i = 0; i < kNT; ++i)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) sc[i][e] += sc2[i][e];
-#endif
 
     // ---- scale into the log2 domain, mask, online softmax ----
 #pragma unroll
@@ -292,105 +271,100 @@ __global__ void __launch_bounds__(SplitKvCfg<DQK, DV, BN, WR, WK, NST>::kThreads
   l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
   l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
 
-  if constexpr (WK > 1) {
-    // ---- merge the key slices through shared memory (ring is free now) ----
-    // layout: [warp][element][lane] floats, element = 0..DV/2-1 for O, then m_a, m_b, l_a, l_b
-    float *buf = reinterpret_cast<float *>(sRing);
-    constexpr int kE = DV / 2 + 4;
-    asm volatile("bar.sync 1, %0;" ::"n"(Cfg::kConsumers * 32) : "memory");
-    if (kw != 0) {
-      float *mine = buf + warp * kE * 32;
-#pragma unroll
-      for (int i = 0; i < kOT; ++i)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) mine[(i * 4 + e) * 32 + lane] = o[i][e];
-      mine[(DV / 2 + 0) * 32 + lane] = m_a;
-      mine[(DV / 2 + 1) * 32 + lane] = m_b;
-      mine[(DV / 2 + 2) * 32 + lane] = l_a;
-      mine[(DV / 2 + 3) * 32 + lane] = l_b;
-    }
-    asm volatile("bar.sync 1, %0;" ::"n"(Cfg::kConsumers * 32) : "memory");
-    if (kw != 0) return;
-    float mm_a = m_a, mm_b = m_b;
-#pragma unroll
-    for (int k = 1; k < WK; ++k) {
-      const float *other = buf + (k * WR + rw) * kE * 32;
-      mm_a = fmaxf(mm_a, other[(DV / 2 + 0) * 32 + lane]);
-      mm_b = fmaxf(mm_b, other[(DV / 2 + 1) * 32 + lane]);
-    }
-    const float rf_a = mm_a == -INFINITY ? 0.f : mm_a;
-    const float rf_b = mm_b == -INFINITY ? 0.f : mm_b;
-    float w_a = fast_exp2(m_a - rf_a), w_b = fast_exp2(m_b - rf_b);
-    l_a *= w_a;
-    l_b *= w_b;
-#pragma unroll
-    for (int i = 0; i < kOT; ++i) {
-      o[i][0] *= w_a;
-      o[i][1] *= w_a;
-      o[i][2] *= w_b;
-      o[i][3] *= w_b;
-    }
-#pragma unroll
-    for (int k = 1; k < WK; ++k) {
-      const float *other = buf + (k * WR + rw) * kE * 32;
-      const float ow_a = fast_exp2(other[(DV / 2 + 0) * 32 + lane] - rf_a);
-      const float ow_b = fast_exp2(other[(DV / 2 + 1) * 32 + lane] - rf_b);
-      l_a += ow_a * other[(DV / 2 + 2) * 32 + lane];
-      l_b += ow_b * other[(DV / 2 + 3) * 32 + lane];
-#pragma unroll
-      for (int i = 0; i < kOT; ++i) {
-        o[i][0] += ow_a * other[(i * 4 + 0) * 32 + lane];
-        o[i][1] += ow_a * other[(i * 4 + 1) * 32 + lane];
-        o[i][2] += ow_b * other[(i * 4 + 2) * 32 + lane];
-        o[i][3] += ow_b * other[(i * 4 + 3) * 32 + lane];
-      }
-    }
-    m_a = mm_a;
-    m_b = mm_b;
-  }
-
   // ---- epilogue ----
-  float inv_a = l_a > 0.f ? 1.f / l_a : 0.f;
-  float inv_b = l_b > 0.f ? 1.f / l_b : 0.f;
+  // Once every consumer has left the loop the ring is free.  Each warp
+  // weights its key slice of its rows (the WK slices of a row meet through
+  // their (m, l) in shared memory), folds in the row's 1/l, and stages the
+  // result there in fp32; then all consumer threads sum the slices and write
+  // the tile out row by row, four columns per thread and step.
+  __shared__ float2 s_ml[Cfg::kConsumers * 16];  // [key slice][row]: (m, l)
+  float *s_o = reinterpret_cast<float *>(sRing);  // [key slice][row][kOutStride]
+  constexpr int kOutStride = Cfg::kOutStride;
   const bool va = lr_a < tr.nvalid, vb = lr_b < tr.nvalid;
   const long grow_a = (long)bh * p.R + tr.row0 + lr_a;
   const long grow_b = grow_a + 8;
-  const int c0 = (lane & 3) * 2;
-  if (p.splits == 1) {
-    inv_a = finish_row(p, grow_a, m_a, l_a);
-    inv_b = finish_row(p, grow_b, m_b, l_b);
-    if (p.lse_out != nullptr && (lane & 3) == 0) {
-      if (va) p.lse_out[grow_a] = row_lse(m_a, l_a);
-      if (vb) p.lse_out[grow_b] = row_lse(m_b, l_b);
-    }
-    uint32_t *out32 = reinterpret_cast<uint32_t *>(p.out);
-#pragma unroll
-    for (int i = 0; i < kOT; ++i) {
-      const int col = i * 8 + c0;
-      if (col < p.Dv) {
-        if (va) out32[(grow_a * p.Dv + col) >> 1] = pack2<kBF16>(o[i][0] * inv_a, o[i][1] * inv_a);
-        if (vb) out32[(grow_b * p.Dv + col) >> 1] = pack2<kBF16>(o[i][2] * inv_b, o[i][3] * inv_b);
-      }
-    }
-  } else {
-    const long total_rows = (long)p.B * p.Hq * p.L;
-    float *po = p.part_o + (long)split * total_rows * p.Dv;
-#pragma unroll
-    for (int i = 0; i < kOT; ++i) {
-      const int col = i * 8 + c0;
-      if (col < p.Dv) {
-        if (va)
-          *reinterpret_cast<float2 *>(po + grow_a * p.Dv + col) =
-              make_float2(o[i][0] * inv_a, o[i][1] * inv_a);
-        if (vb)
-          *reinterpret_cast<float2 *>(po + grow_b * p.Dv + col) =
-              make_float2(o[i][2] * inv_b, o[i][3] * inv_b);
-      }
-    }
+  const long total_rows = (long)p.B * p.Hq * p.L;
+  asm volatile("bar.sync 1, %0;" ::"n"(Cfg::kConsumers * 32) : "memory");
+  float f_a = 1.f, f_b = 1.f;  // weight of this slice within its row
+  if constexpr (WK > 1) {
     if ((lane & 3) == 0) {
-      float *pl = p.part_lse + (long)split * total_rows;
-      if (va) pl[grow_a] = row_lse(m_a, l_a);
-      if (vb) pl[grow_b] = row_lse(m_b, l_b);
+      s_ml[kw * Cfg::kRT + lr_a] = make_float2(m_a, l_a);
+      s_ml[kw * Cfg::kRT + lr_b] = make_float2(m_b, l_b);
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(Cfg::kConsumers * 32) : "memory");
+    float mm_a = -INFINITY, mm_b = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < WK; ++k) {
+      mm_a = fmaxf(mm_a, s_ml[k * Cfg::kRT + lr_a].x);
+      mm_b = fmaxf(mm_b, s_ml[k * Cfg::kRT + lr_b].x);
+    }
+    // a row with no visible key in any slice keeps m = -inf and l = 0
+    const float rf_a = mm_a == -INFINITY ? 0.f : mm_a;
+    const float rf_b = mm_b == -INFINITY ? 0.f : mm_b;
+    float ls_a = 0.f, ls_b = 0.f;
+#pragma unroll
+    for (int k = 0; k < WK; ++k) {
+      const float2 xa = s_ml[k * Cfg::kRT + lr_a];
+      const float2 xb = s_ml[k * Cfg::kRT + lr_b];
+      ls_a += fast_exp2(xa.x - rf_a) * xa.y;
+      ls_b += fast_exp2(xb.x - rf_b) * xb.y;
+    }
+    f_a = fast_exp2(m_a - rf_a);
+    f_b = fast_exp2(m_b - rf_b);
+    m_a = mm_a;
+    m_b = mm_b;
+    l_a = ls_a;
+    l_b = ls_b;
+  }
+  float inv_a, inv_b;
+  if (p.splits == 1) {
+    inv_a = finish_row(p, grow_a, m_a, l_a);  // folds in the head's sink, if any
+    inv_b = finish_row(p, grow_b, m_b, l_b);
+  } else {
+    inv_a = l_a > 0.f ? 1.f / l_a : 0.f;
+    inv_b = l_b > 0.f ? 1.f / l_b : 0.f;
+  }
+  if (kw == 0 && (lane & 3) == 0) {
+    float *lse = p.splits == 1 ? p.lse_out : p.part_lse + (long)split * total_rows;
+    if (lse != nullptr) {
+      if (va) lse[grow_a] = row_lse(m_a, l_a);
+      if (vb) lse[grow_b] = row_lse(m_b, l_b);
+    }
+  }
+  {
+    const float sa = f_a * inv_a, sb = f_b * inv_b;
+    float *row_a = s_o + (kw * Cfg::kRT + lr_a) * kOutStride + (lane & 3) * 2;
+    float *row_b = row_a + 8 * kOutStride;
+#pragma unroll
+    for (int i = 0; i < kOT; ++i) {
+      *reinterpret_cast<float2 *>(row_a + i * 8) = make_float2(o[i][0] * sa, o[i][1] * sa);
+      *reinterpret_cast<float2 *>(row_b + i * 8) = make_float2(o[i][2] * sb, o[i][3] * sb);
+    }
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(Cfg::kConsumers * 32) : "memory");
+  const int q4 = p.Dv / 4;  // Dv is a multiple of 8
+  const int items = tr.nvalid * q4;
+  const long grow0 = (long)bh * p.R + tr.row0;
+  for (int it = threadIdx.x; it < items; it += Cfg::kConsumers * 32) {
+    const int r = it / q4;
+    const int c = (it - r * q4) * 4;
+    float4 acc = *reinterpret_cast<const float4 *>(s_o + r * kOutStride + c);
+#pragma unroll
+    for (int k = 1; k < WK; ++k) {
+      const float4 x = *reinterpret_cast<const float4 *>(s_o + (k * Cfg::kRT + r) * kOutStride + c);
+      acc.x += x.x;
+      acc.y += x.y;
+      acc.z += x.z;
+      acc.w += x.w;
+    }
+    const long at = (grow0 + r) * p.Dv + c;
+    if (p.splits == 1) {
+      uint2 w;
+      w.x = pack2<kBF16>(acc.x, acc.y);
+      w.y = pack2<kBF16>(acc.z, acc.w);
+      *reinterpret_cast<uint2 *>(reinterpret_cast<uint16_t *>(p.out) + at) = w;
+    } else {
+      *reinterpret_cast<float4 *>(p.part_o + (long)split * total_rows * p.Dv + at) = acc;
     }
   }
   (void)ok;
