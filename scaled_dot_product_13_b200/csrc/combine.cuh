@@ -32,6 +32,9 @@ __global__ void __launch_bounds__(128) combine_kernel(const float *__restrict__ 
   __shared__ float s_red[2][4];   // per-warp max, per-warp weight sum
   constexpr int kPre = 64;        // splits whose partials go out in the first round trip
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  // the next split pass on the stream may start its setup now; it waits for
+  // this grid before it reads or writes global memory
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const long row = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int col = blockIdx.y * 128 + tid;  // this thread's output column

@@ -34,9 +34,6 @@ constexpr int kSplitKvBN = 64;
 // (64-column TMA boxes of 128 bytes per row).  With two CTAs per SM each gets
 // half of the SM's 228 KB less the 1 KB the hardware reserves per CTA; the
 // budgets keep 2 KB for barriers, alignment slack and static shared memory.
-#ifndef SDPA_SK_TWO_PER_SM
-#define SDPA_SK_TWO_PER_SM 0
-#endif
 constexpr unsigned kSplitKvBudget1 = 232448u - 2048u;
 constexpr unsigned kSplitKvBudget2 = 233472u / 2 - 1024u - 2048u;
 constexpr unsigned splitkv_stage_bytes(int dqk, int dv) {
@@ -51,10 +48,15 @@ constexpr int splitkv_stages(int dqk, int dv, int wr, unsigned budget) {
              ? 4
              : (int)((budget - splitkv_q_bytes(dqk, wr)) / splitkv_stage_bytes(dqk, dv));
 }
-// CTAs of one instance resident per SM: two where double buffering fits half
-// the SM's shared memory, else one.
+// CTAs of one instance resident per SM.  The 64-row layout (four warps on
+// their own rows, each doing four times the math per key of a slice warp)
+// runs two per SM where double buffering fits half the shared memory and the
+// registers fit half the file: the second CTA's warps hide the first's
+// latencies (verify L=12..16 at S=32K: 44.4 -> 40.3 us).  The 16- and 32-row
+// layouts keep one per SM: twice the splits cost more in the combine than
+// the pass gains (decode sweep 2113-2125 against 2164-2167 GB/s).
 constexpr int splitkv_ctas_per_sm(int dqk, int dv, int wr) {
-  return SDPA_SK_TWO_PER_SM && splitkv_stages(dqk, dv, wr, kSplitKvBudget2) >= 2 ? 2 : 1;
+  return wr == 4 && dqk + dv <= 256 && splitkv_stages(dqk, dv, wr, kSplitKvBudget2) >= 2 ? 2 : 1;
 }
 
 // Key block of the tcgen05 kernel: 128 keys while two 128-key score buffers

@@ -64,9 +64,22 @@ sdpa_status run_splitkv(const Launch &ln, std::string *err) {
   p.wd.word = ln.wd_word;
   p.wd.limit_ns = ln.wd_limit_ns;
   if (ln.ev_start) record_event(ln.ev_start, ln.stream);
-  kern<<<(unsigned)pl.ctas, Cfg::kThreads, Cfg::kSmemBytes, ln.stream>>>(tq, tk, tv, p);
+  // programmatic stream serialization: the kernel's setup may overlap the
+  // previous grid on the stream; it waits (griddepcontrol.wait) before any
+  // global memory access
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)pl.ctas);
+  cfg.blockDim = dim3(Cfg::kThreads);
+  cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+  cfg.stream = ln.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, p);
   if (ln.ev_stop) record_event(ln.ev_stop, ln.stream);
-  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) {
     *err = std::string("splitkv_kernel launch failed: ") + cudaGetErrorString(e);
     return SDPA_ERR_CUDA;

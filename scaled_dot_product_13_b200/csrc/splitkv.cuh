@@ -86,6 +86,10 @@ __global__ void __launch_bounds__(SplitKvCfg<DQK, DV, BN, WR, WK, NST>::kThreads
     fence_barrier_init();
   }
   __syncthreads();
+  // Launched as a programmatic dependent of whatever precedes it on the
+  // stream: the setup above may overlap that grid's tail, and nothing in
+  // global memory is touched before it has completed.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   // Let the dependent combine launch now: its CTAs wait in griddepcontrol.wait
   // until this grid has finished, so its launch latency overlaps this pass.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
