@@ -109,6 +109,18 @@ def test_plan_packs_verify_rows_per_kv_head():
         assert info["row_tiles"] * info["row_tile"] < 4 * L + info["row_tile"]
 
 
+def test_plan_two_split_kv_ctas_per_sm_only_for_the_64_row_layout():
+    # 33..64 packed rows (four row warps, no key slices) run two CTAs per SM,
+    # so the planner fills twice the SM count; 16- and 32-row layouts one
+    for L, per_sm in ((4, 1), (8, 1), (12, 2), (16, 2)):
+        info = sdpa.plan(1, 32, 8, L, 32768, 128, 128, causal=False, dtype="f16", num_sms=148)
+        assert info["path"] == sdpa.PATH_SPLITKV
+        assert per_sm * 148 - 8 < info["ctas"] <= per_sm * 148, (L, info)
+    # head dims whose stages do not fit half the shared memory stay at one per SM
+    info = sdpa.plan(1, 32, 8, 16, 32768, 256, 256, causal=False, num_sms=148)
+    assert info["ctas"] <= 148
+
+
 def test_plan_forced_splits_and_single_split_needs_no_workspace():
     info = sdpa.plan(1, 8, 2, 3, 1000, 64, 64, causal=True, num_sms=148, force_splits=1)
     assert info["splits"] == 1 and info["workspace_bytes"] == 0 and info["launches"] == 1
