@@ -339,6 +339,13 @@ def secondary(sdpa, probs, steps, warmup, flush, sync_all, device, peaks, kind, 
                       "frac_tensor": round(tf / peaks["bf16_tflops"], 4)})
         d["kv_gbs"] = round(c.kv_bytes / (us * 1e-6) / 1e9, 1)
         d["frac_hbm"] = round(d["kv_gbs"] / peaks["hbm_gbs"], 4)
+        # the call's own roofline: the slower of streaming its KV at the
+        # measured copy bandwidth and its FLOPs at the measured tensor peak
+        # (verify shapes sit near the ridge)
+        floor_us = 1e6 * max(c.kv_bytes / (peaks["hbm_gbs"] * 1e9),
+                             c.flops / (peaks["bf16_tflops"] * 1e12))
+        d["roofline_us"] = round(floor_us, 2)
+        d["frac_roofline"] = round(floor_us / us, 4)
         pts.append(d)
     del cases
     torch.cuda.empty_cache()
