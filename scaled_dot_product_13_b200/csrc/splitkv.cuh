@@ -87,8 +87,28 @@ __global__ void __launch_bounds__(SplitKvCfg<DQK, DV, BN, WR, WK, NST>::kThreads
   }
   __syncthreads();
   // Launched as a programmatic dependent of whatever precedes it on the
-  // stream: the setup above may overlap that grid's tail, and nothing in
-  // global memory is touched before it has completed.
+  // stream: the setup here may overlap that grid's tail.  Before waiting for
+  // it, the producer asks for this CTA's Q tile and first NST key blocks to
+  // be brought into L2.  A prefetch only warms L2, which is where every
+  // write of that grid lands too, so it cannot hand a stale value to the
+  // loads, and those (and every other global access) come after the wait.
+  if (warp == Cfg::kConsumers && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+#pragma unroll
+    for (int bx = 0; bx < Cfg::kQBoxes; ++bx)
+      tma_prefetch_l2_2d(&tm_q, bx * 64, bh * p.R + tr.row0);
+    const int npf = nblocks < NST ? nblocks : NST;
+    for (int t = 0; t < npf; ++t) {
+#pragma unroll
+      for (int bx = 0; bx < Cfg::kQBoxes; ++bx)
+        tma_prefetch_l2_3d(&tm_k, bx * 64, k_lo + t * BN, bh);
+#pragma unroll
+      for (int bx = 0; bx < Cfg::kVBoxes; ++bx)
+        tma_prefetch_l2_3d(&tm_v, bx * 64, k_lo + t * BN, bh);
+    }
+  }
   asm volatile("griddepcontrol.wait;" ::: "memory");
   // Let the dependent combine launch now: its CTAs wait in griddepcontrol.wait
   // until this grid has finished, so its launch latency overlaps this pass.
@@ -97,9 +117,6 @@ __global__ void __launch_bounds__(SplitKvCfg<DQK, DV, BN, WR, WK, NST>::kThreads
   if (warp == Cfg::kConsumers) {
     // ===================== producer warp =====================
     if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
       const int grow0 = bh * p.R + tr.row0;
       mbar_arrive_expect_tx(qbar, Cfg::kQBytes);
 #pragma unroll
