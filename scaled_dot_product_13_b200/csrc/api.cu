@@ -155,7 +155,8 @@ constexpr int kTc2RowThreshold = 256;
 
 // A split must cover at least this many key blocks, and problems of at most
 // kNoSplitBlocks key blocks are not split: below that the combine launch
-// costs more than the parallelism gains.
+// costs more than the parallelism gains.  The split-KV kernel counts in
+// 64-key units (128 and 256 keys) whatever its key block.
 constexpr int kMinBlocksPerSplit = 2;
 constexpr int kMinBlocksPerSplitWide = 8;
 constexpr int kNoSplitBlocks = 4;
@@ -246,7 +247,7 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
       pl.wr = 4; pl.wk = 1;
     }
     pl.row_tile = 16 * pl.wr;
-    pl.key_block = kSplitKvBN;
+    pl.key_block = splitkv_bn(kDimPairs[pl.pair].dqk, kDimPairs[pl.pair].dv);
   }
   pl.row_tiles = (pl.rows + pl.row_tile - 1) / pl.row_tile;
   // keys visible to at least one row: [kbeg, kend)
@@ -268,12 +269,16 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
   int splits;
   if (force_splits > 0) {
     splits = std::min(force_splits, nkb);
-  } else if (base >= slots || nkb <= kNoSplitBlocks) {
+  } else if (base >= slots || (path == SDPA_PATH_SPLITKV ? nkb * bn <= kNoSplitBlocks * 64
+                                                          : nkb <= kNoSplitBlocks)) {
     splits = 1;
   } else {
     // the wide kernel's 32-key blocks are small and its partials wide
-    // (Dv up to 512 floats per row and split): give each split more keys
-    const int min_blocks = path == SDPA_PATH_WIDE ? kMinBlocksPerSplitWide : kMinBlocksPerSplit;
+    // (Dv up to 512 floats per row and split): give each split more keys.
+    // The split-KV kernel's splits cover at least 128 keys whatever its block.
+    const int min_blocks = path == SDPA_PATH_WIDE      ? kMinBlocksPerSplitWide
+                           : path == SDPA_PATH_SPLITKV ? std::max(1, 128 / bn)
+                                                       : kMinBlocksPerSplit;
     splits = (int)std::max(1LL, slots / base);
     splits = std::min(splits, std::max(1, nkb / min_blocks));
   }

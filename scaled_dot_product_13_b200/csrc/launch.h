@@ -28,7 +28,10 @@ constexpr int kWidePair = 6;
 constexpr int kWideBN = 32;
 
 // Key block of the split-KV kernel (keys per pipeline stage).
-constexpr int kSplitKvBN = 64;
+#ifndef SDPA_SK_BN
+#define SDPA_SK_BN 64
+#endif
+constexpr int kSplitKvBN = SDPA_SK_BN;
 
 // Split-KV shared memory: one Q tile of 16*wr rows plus a ring of K/V stages
 // (64-column TMA boxes of 128 bytes per row).  With two CTAs per SM each gets
@@ -36,17 +39,26 @@ constexpr int kSplitKvBN = 64;
 // budgets keep 2 KB for barriers, alignment slack and static shared memory.
 constexpr unsigned kSplitKvBudget1 = 232448u - 2048u;
 constexpr unsigned kSplitKvBudget2 = 233472u / 2 - 1024u - 2048u;
-constexpr unsigned splitkv_stage_bytes(int dqk, int dv) {
-  return (unsigned)(((dqk + 63) / 64 + (dv + 63) / 64) * kSplitKvBN * 128);
+constexpr unsigned splitkv_stage_bytes(int dqk, int dv, int bn = kSplitKvBN) {
+  return (unsigned)(((dqk + 63) / 64 + (dv + 63) / 64) * bn * 128);
+}
+// Key block of one instance: kSplitKvBN where two stages of it fit next to a
+// 64-row Q tile, else 64.
+constexpr int splitkv_bn(int dqk, int dv) {
+  return 2 * splitkv_stage_bytes(dqk, dv, kSplitKvBN) + ((dqk + 63) / 64) * 64 * 128 <= 232448u - 2048u
+             ? kSplitKvBN
+             : 64;
 }
 constexpr unsigned splitkv_q_bytes(int dqk, int wr) {
   return (unsigned)(((dqk + 63) / 64) * 16 * wr * 128);
 }
 // Stages that fit the budget next to Q, at most 4.
 constexpr int splitkv_stages(int dqk, int dv, int wr, unsigned budget) {
-  return (int)((budget - splitkv_q_bytes(dqk, wr)) / splitkv_stage_bytes(dqk, dv)) > 4
+  return (int)((budget - splitkv_q_bytes(dqk, wr)) /
+               splitkv_stage_bytes(dqk, dv, splitkv_bn(dqk, dv))) > 4
              ? 4
-             : (int)((budget - splitkv_q_bytes(dqk, wr)) / splitkv_stage_bytes(dqk, dv));
+             : (int)((budget - splitkv_q_bytes(dqk, wr)) /
+                     splitkv_stage_bytes(dqk, dv, splitkv_bn(dqk, dv)));
 }
 // CTAs of one instance resident per SM.  The 64-row layout (four warps on
 // their own rows, each doing four times the math per key of a slice warp)

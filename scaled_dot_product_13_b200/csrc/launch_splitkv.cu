@@ -11,7 +11,7 @@ namespace {
 
 template <bool kBF16, int DQK, int DV, int WR, int WK>
 sdpa_status run_splitkv(const Launch &ln, std::string *err) {
-  constexpr int kBN = kSplitKvBN;
+  constexpr int kBN = splitkv_bn(DQK, DV);
   // one or two CTAs per SM; stages: as many as fit next to Q, at most 4
   constexpr int kMinB = splitkv_ctas_per_sm(DQK, DV, WR);
   constexpr int kNST =
