@@ -47,6 +47,13 @@
  * found on the host are returned before anything is enqueued.  Launch errors
  * are returned as SDPA_ERR_CUDA.  Faults inside a kernel surface later, like
  * any CUDA error, and sdpa_device_status() reports a watchdog expiry.
+ * Stream order holds as for plain launches.  The split-KV pass and the
+ * combine are launched with programmatic stream serialization: their setup
+ * (and, for the split pass, an L2 prefetch of its first inputs) may overlap
+ * the previous kernel on the stream, but neither reads nor writes global
+ * memory before that kernel has completed.  A kernel the caller launches
+ * after a call with the same attribute must likewise wait
+ * (griddepcontrol.wait / cudaGridDependencySynchronize) before it reads `out`.
  *
  * Thread safety: calls from several host threads are safe; the last error
  * message is kept per thread.
