@@ -240,7 +240,10 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
     pl.key_block = tc_key_block(kDimPairs[pl.pair].dqk, kDimPairs[pl.pair].dv);
   } else {
     if (pl.rows <= 16) {
-      pl.wr = 1; pl.wk = 4;
+      // one 16-row group: 16 keys per warp of every key block
+      pl.wr = 1;
+      pl.wk = splitkv_bn(kDimPairs[pl.pair].dqk, kDimPairs[pl.pair].dv) / 16;
+      if (pl.wk > 8) pl.wk = 8;
     } else if (pl.rows <= 32) {
       pl.wr = 2; pl.wk = 2;
     } else {

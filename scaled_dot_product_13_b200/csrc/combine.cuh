@@ -16,7 +16,7 @@
 
 // splits loaded per round trip to L2 after the first kPre
 #ifndef SDPA_COMBINE_BATCH
-#define SDPA_COMBINE_BATCH 8
+#define SDPA_COMBINE_BATCH 16
 #endif
 
 namespace sdpa {

@@ -90,6 +90,10 @@ sdpa_status run_splitkv(const Launch &ln, std::string *err) {
 template <bool kBF16, int DQK, int DV>
 sdpa_status run_layout(const Launch &ln, std::string *err) {
   const Plan &pl = ln.plan;
+  if constexpr (splitkv_bn(DQK, DV) >= 128) {
+    // 128-key blocks: eight warps of 16 keys each for one 16-row group
+    if (pl.wr == 1 && pl.wk == 8) return run_splitkv<kBF16, DQK, DV, 1, 8>(ln, err);
+  }
   if (pl.wr == 1 && pl.wk == 4) return run_splitkv<kBF16, DQK, DV, 1, 4>(ln, err);
   if (pl.wr == 2 && pl.wk == 2) return run_splitkv<kBF16, DQK, DV, 2, 2>(ln, err);
   if (pl.wr == 4 && pl.wk == 1) return run_splitkv<kBF16, DQK, DV, 4, 1>(ln, err);
