@@ -330,9 +330,11 @@ def secondary(sdpa, probs, steps, warmup, flush, sync_all, device, peaks, kind, 
     call_ms, main_ms, _ = time_cases(sdpa, cases, steps, warmup, flush, sync_all, graphs)
     pts = []
     for c, cm, mm in zip(cases, call_ms, main_ms):
-        us = 1e3 * statistics.median(cm)
-        d = {"name": c.p.name, "us": round(us, 2), "path": c.info["path"],
-             "splits": c.info["splits"]}
+        # mean over the timed steps: the device timer's coarse steps make a
+        # median jump between neighbouring values
+        us = 1e3 * statistics.mean(cm)
+        d = {"name": c.p.name, "us": round(us, 2), "us_median": round(1e3 * statistics.median(cm), 2),
+             "path": c.info["path"], "splits": c.info["splits"]}
         if kind == "tflops":
             tf = c.flops / (us * 1e-6) / 1e12
             d.update({"tflops": round(tf, 1),
@@ -389,8 +391,8 @@ def main():
                 "launch": "eager" if args.eager else "the step's calls captured in one CUDA graph, replayed",
                 "timing": "step = events around the back-to-back calls of one step; per call "
                           "(points) = library events before the split pass and after the combine, "
-                          "each call replayed alone after an L2 flush; main-kernel time from probe "
-                          "replays with an event after the split pass",
+                          "each call replayed alone after an L2 flush, mean over the timed steps; "
+                          "main-kernel time from probe replays with an event after the split pass",
                 "parallelism": f"replicas x{world} (independent KV-head units, no collective)"}
 
     if args.impl == "reference":
@@ -475,12 +477,13 @@ def main():
                 "algorithmic_bytes_per_launch": cases[big].kv_bytes}
     points = []
     for c, cm, mm, om in zip(cases, call_ms, main_ms, outer_ms):
-        us = 1e3 * statistics.median(cm)
+        us = 1e3 * statistics.mean(cm)
         points.append({"name": c.p.name, "us": round(us, 2),
+                       "us_median": round(1e3 * statistics.median(cm), 2),
                        "us_p10": round(1e3 * float(np.percentile(cm, 10)), 2),
                        "us_p90": round(1e3 * float(np.percentile(cm, 90)), 2),
-                       "main_kernel_us": round(1e3 * statistics.median(mm), 2),
-                       "outer_us": round(1e3 * statistics.median(om), 2),
+                       "main_kernel_us": round(1e3 * statistics.mean(mm), 2),
+                       "outer_us": round(1e3 * statistics.mean(om), 2),
                        "kv_gbs": round(c.kv_bytes / (us * 1e-6) / 1e9, 1),
                        "frac_hbm": round(c.kv_bytes / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
                        "splits": c.info["splits"], "ctas": c.info["ctas"]})
@@ -496,7 +499,7 @@ def main():
 
     extra = {}
     if not args.no_secondary:
-        sec_steps = max(3, min(args.steps, 10))
+        sec_steps = max(3, min(args.steps, 20))
         gr = not args.eager
         extra["prefill"] = secondary(sdpa, I.window_problems() + I.encoder_problems(), sec_steps,
                                      3, flush, sync_all, device, peaks, "tflops", gr)
