@@ -174,7 +174,7 @@ def time_cases(sdpa, cases, steps, warmup, flush, sync_all, graphs=True):
     """Per call: flush L2 (untimed), then run the call with CUDA events
     recorded by the library on its launch stream.
 
-    Two interleaved runners per call.  The timed one records an event before
+    Two runners per call, replayed in turn.  The timed one records an event before
     the main kernel and one after the call's last launch (the combine, when
     split): call time = the device time of the library's work.  Nothing sits
     between the split pass and the combine there, so the combine keeps its
@@ -213,23 +213,24 @@ def time_cases(sdpa, cases, steps, warmup, flush, sync_all, graphs=True):
     timed = [runner(c, h[0], None, h[1]) for c, h in zip(cases, hooks)]
     probes = [runner(c, h[2], h[3], h[4]) for c, h in zip(cases, hooks)]
     torch.cuda.synchronize()
-    for it in range(warmup + steps):
-        evs = []
-        for run, probe in zip(timed, probes):
+    # One call at a time: its warm-up replays, then its timed ones.  Replays of
+    # different calls interleaved would make a call pay for the SMs' switch
+    # between shared-memory configurations of unlike kernels (one-tile
+    # tcgen05 after split-KV, say), which a call repeated in a loop does not.
+    for i, (run, probe) in enumerate(zip(timed, probes)):
+        h = hooks[i]
+        for it in range(warmup + steps):
             flush_l2(flush)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             run()
             e1.record(stream)
-            evs.append((e0, e1))
             flush_l2(flush)
             probe()
-        if it == warmup - 1:
-            sync_all()
-        if it >= warmup:
-            torch.cuda.synchronize()
-            for i, (e0, e1) in enumerate(evs):
-                h = hooks[i]
+            if it == warmup - 1:
+                sync_all()
+            if it >= warmup:
+                torch.cuda.synchronize()
                 call_ms[i].append(h[0].elapsed_time(h[1]))
                 main_ms[i].append(h[2].elapsed_time(h[3]))
                 outer_ms[i].append(e0.elapsed_time(e1))
@@ -503,8 +504,10 @@ def main():
         gr = not args.eager
         extra["prefill"] = secondary(sdpa, I.window_problems() + I.encoder_problems(), sec_steps,
                                      3, flush, sync_all, device, peaks, "tflops", gr)
-        extra["verify"] = secondary(sdpa, I.verify_problems(), sec_steps, 3, flush, sync_all,
-                                    device, peaks, "tflops", gr)
+        # the verify sweep checks monotonicity in L between calls whose times
+        # differ by about a microsecond: 60 samples per call (cheap at ~40 us)
+        extra["verify"] = secondary(sdpa, I.verify_problems(), max(sec_steps, 60), 3, flush,
+                                    sync_all, device, peaks, "tflops", gr)
         extra["tiny"] = secondary(sdpa, [I.tiny_problem()], sec_steps, 3, flush, sync_all,
                                   device, peaks, "tflops", gr)
         extra["wide"] = secondary(sdpa, I.wide_problems(), sec_steps, 3, flush, sync_all,
