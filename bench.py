@@ -325,6 +325,29 @@ def oracle_sample(cases, budget_s=12.0):
     return nbytes / dt / 1e9, dt, cores, calls
 
 
+def verify_checks(points):
+    """Monotonicity and cliff checks of the verify sweep, per S.
+
+    Monotone: t(L_next) >= 0.97 t(L) for consecutive L.  No cliff over
+    L in [8, 64]: t(L_next) / t(L) <= max(1.25, L_next / L) (the pages' cliff
+    was a 2.3x jump for 1.5x the rows).  Points are named verify_s<S>_l<L>."""
+    by_s = {}
+    for p in points:
+        s_part, l_part = p["name"].split("_")[1:3]
+        by_s.setdefault(int(s_part[1:]), []).append((int(l_part[1:]), p["us"]))
+    out = {}
+    for S, pts in sorted(by_s.items()):
+        pts.sort()
+        mono = all(b[1] >= 0.97 * a[1] for a, b in zip(pts, pts[1:]))
+        ratios = [(a[0], b[0], b[1] / a[1]) for a, b in zip(pts, pts[1:]) if a[0] >= 8]
+        cliff = [r for r in ratios if r[2] > max(1.25, r[1] / r[0])]
+        worst = max(ratios, key=lambda r: r[2] / max(1.25, r[1] / r[0])) if ratios else None
+        out[f"s{S}"] = {"monotone": mono, "no_cliff": not cliff,
+                        "worst_step": None if worst is None else
+                        {"from_L": worst[0], "to_L": worst[1], "ratio": round(worst[2], 3)}}
+    return out
+
+
 def secondary(sdpa, probs, steps, warmup, flush, sync_all, device, peaks, kind, graphs=True):
     """Time a list of problems (one call each per step); return a summary."""
     cases = [Case(sdpa, p, device) for p in probs]
@@ -508,6 +531,7 @@ def main():
         # differ by about a microsecond: 60 samples per call (cheap at ~40 us)
         extra["verify"] = secondary(sdpa, I.verify_problems(), max(sec_steps, 60), 3, flush,
                                     sync_all, device, peaks, "tflops", gr)
+        extra["verify_checks"] = verify_checks(extra["verify"])
         extra["tiny"] = secondary(sdpa, [I.tiny_problem()], sec_steps, 3, flush, sync_all,
                                   device, peaks, "tflops", gr)
         extra["wide"] = secondary(sdpa, I.wide_problems(), sec_steps, 3, flush, sync_all,
