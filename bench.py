@@ -549,12 +549,26 @@ def main():
                     "ms_per_step": round(float(np.mean(e2e_ms)), 3)},
             "points": points}
     line.update(extra)
+    if extra:
+        # compact per-call figures last on the line (prefill at the very end),
+        # so that a reader who keeps only the end of the output still sees
+        # every call: [name, path, us, fraction of the call's own roofline]
+        def brief(rows):
+            return [[d["name"], d["path"], round(d["us"], 1), round(d["frac_roofline"], 3)]
+                    for d in rows]
+        line["summary"] = {
+            "decode": [[d["name"], round(d["us"], 1), round(d["frac_hbm"], 3)] for d in points],
+            "verify": brief(extra["verify"]), "verify_checks": extra["verify_checks"],
+            "tiny": brief(extra["tiny"]), "wide": brief(extra["wide"]),
+            "prefill": brief(extra["prefill"])}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         host_cases = [HostCase(p) for p in I.decode_problems()]
         val, secs, cores, calls = oracle_sample(host_cases, budget_s=10.0)
         line["cpu_baseline"] = {"value": round(val, 4), "unit": "GB/s (KV, decode)",
                                 "cores": cores, "kind": "oracle",
                                 "sample": f"{calls} decode calls of the sweep ({secs:.1f} s, fp64)"}
+    if "summary" in line:
+        line["summary"] = line.pop("summary")
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:

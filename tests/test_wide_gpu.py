@@ -75,8 +75,9 @@ def test_wide_sinks_offset_lse(cuda_lib):
 
 @pytest.mark.parametrize("idx", [0, 1, 2])
 def test_wide_bench_workloads(cuda_lib, idx):
-    """The head-dim-512 bench workloads at full size; the prefill on sampled rows."""
+    """The head-dim-512 bench workloads at full size; the prefill on 256 sampled
+    query rows per head."""
     p = I.wide_problems()[idx]
-    rows = I.sample_rows(p.L, 64, seed=p.seed) if p.L > 256 else None
+    rows = I.sample_rows(p.L, 256, seed=p.seed) if p.L > 256 else None
     _, _, info = check_problem(cuda_lib, p, rows=rows)
     assert info["path"] == S.PATH_WIDE
