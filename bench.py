@@ -348,10 +348,49 @@ def verify_checks(points):
     return out
 
 
-def secondary(sdpa, probs, steps, warmup, flush, sync_all, device, peaks, kind, graphs=True):
-    """Time a list of problems (one call each per step); return a summary."""
+def time_stream(sdpa, c, flush, l2_bytes, reps=6, warmup=2, max_copies=32,
+                max_bytes=4 << 30):
+    """Back-to-back throughput of one call: n calls in a row on n copies of the
+    inputs whose total exceeds 2x L2 (so every call reads its inputs from HBM),
+    captured in one CUDA graph; events around each replay, L2 flushed before
+    it.  Returns microseconds per call (mean over ``reps`` replays).  One call
+    alone carries its launch edges; here they overlap the neighbouring calls,
+    as in a model that runs attention layer after layer."""
+    per = sum(t.numel() * t.element_size() for t in (c.q, c.k, c.v))
+    n = max(1, min(max_copies, -(-2 * l2_bytes // per) + 1, max(1, max_bytes // per)))
+    copies = [(c.q, c.k, c.v)] + [tuple(t.clone() for t in (c.q, c.k, c.v)) for _ in range(n - 1)]
+    stream = torch.cuda.current_stream()
+
+    def body():
+        for q, k, v in copies:
+            sdpa.forward_ws(q, k, v, c.ws, scale=c.p.sm_scale, causal=c.p.causal,
+                            window_size=c.p.window, out=c.out)
+
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        body()
+    torch.cuda.synchronize()
+    ts = []
+    for it in range(warmup + reps):
+        flush_l2(flush)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if it >= warmup:
+            ts.append(e0.elapsed_time(e1) * 1e3 / n)
+    del g, copies
+    return statistics.mean(ts), n
+
+
+def secondary(sdpa, probs, steps, warmup, flush, sync_all, device, peaks, kind, graphs=True,
+              stream=False):
+    """Time a list of problems (one call each per step); return a summary.
+    With ``stream``, each problem is also timed back to back (``us_stream``)."""
     cases = [Case(sdpa, p, device) for p in probs]
     call_ms, main_ms, _ = time_cases(sdpa, cases, steps, warmup, flush, sync_all, graphs)
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
     pts = []
     for c, cm, mm in zip(cases, call_ms, main_ms):
         # mean over the timed steps: the device timer's coarse steps make a
@@ -372,6 +411,13 @@ def secondary(sdpa, probs, steps, warmup, flush, sync_all, device, peaks, kind, 
                              c.flops / (peaks["bf16_tflops"] * 1e12))
         d["roofline_us"] = round(floor_us, 2)
         d["frac_roofline"] = round(floor_us / us, 4)
+        if stream:
+            us_s, n = time_stream(sdpa, c, flush, l2)
+            d["us_stream"] = round(us_s, 2)
+            d["stream_copies"] = n
+            d["frac_roofline_stream"] = round(floor_us / us_s, 4)
+            if kind == "tflops":
+                d["tflops_stream"] = round(c.flops / (us_s * 1e-6) / 1e12, 1)
         pts.append(d)
     del cases
     torch.cuda.empty_cache()
@@ -414,9 +460,11 @@ def main():
                       "474 MB of KV exceed L2) and before every call timed alone",
                 "launch": "eager" if args.eager else "the step's calls captured in one CUDA graph, replayed",
                 "timing": "step = events around the back-to-back calls of one step; per call "
-                          "(points) = library events before the split pass and after the combine, "
-                          "each call replayed alone after an L2 flush, mean over the timed steps; "
-                          "main-kernel time from probe replays with an event after the split pass",
+                          "(points) = library events before the split pass and after the call's "
+                          "last launch, each call replayed alone after an L2 flush, mean over the "
+                          "timed steps; main-kernel time from probe replays with an event after "
+                          "the split pass; prefill and verify us_stream = calls back to back on "
+                          "rotating input copies totalling more than 2x L2, per call",
                 "parallelism": f"replicas x{world} (independent KV-head units, no collective)"}
 
     if args.impl == "reference":
@@ -526,11 +574,11 @@ def main():
         sec_steps = max(3, min(args.steps, 20))
         gr = not args.eager
         extra["prefill"] = secondary(sdpa, I.window_problems() + I.encoder_problems(), sec_steps,
-                                     3, flush, sync_all, device, peaks, "tflops", gr)
+                                     3, flush, sync_all, device, peaks, "tflops", gr, stream=True)
         # the verify sweep checks monotonicity in L between calls whose times
         # differ by about a microsecond: 60 samples per call (cheap at ~40 us)
         extra["verify"] = secondary(sdpa, I.verify_problems(), max(sec_steps, 60), 3, flush,
-                                    sync_all, device, peaks, "tflops", gr)
+                                    sync_all, device, peaks, "tflops", gr, stream=True)
         extra["verify_checks"] = verify_checks(extra["verify"])
         extra["tiny"] = secondary(sdpa, [I.tiny_problem()], sec_steps, 3, flush, sync_all,
                                   device, peaks, "tflops", gr)
@@ -552,10 +600,12 @@ def main():
     if extra:
         # compact per-call figures last on the line (prefill at the very end),
         # so that a reader who keeps only the end of the output still sees
-        # every call: [name, path, us, fraction of the call's own roofline]
+        # every call: [name, path, us alone, fraction of the call's own
+        # roofline, and for prefill and verify us back to back, its fraction]
         def brief(rows):
-            return [[d["name"], d["path"], round(d["us"], 1), round(d["frac_roofline"], 3)]
-                    for d in rows]
+            return [[d["name"], d["path"], round(d["us"], 1), round(d["frac_roofline"], 3)] +
+                    ([round(d["us_stream"], 1), round(d["frac_roofline_stream"], 3)]
+                     if "us_stream" in d else []) for d in rows]
         line["summary"] = {
             "decode": [[d["name"], round(d["us"], 1), round(d["frac_hbm"], 3)] for d in points],
             "verify": brief(extra["verify"]), "verify_checks": extra["verify_checks"],

@@ -175,7 +175,8 @@ SDPA_API sdpa_status sdpa_forward_ws(const void *q, const void *k, const void *v
  * The caller still passes q, k, v and out.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *     before any stream capture.  If the device's context is replaced later
+ *     (cudaDeviceReset), the next call looks the address up again.
  *   - Problems whose split workspace (sdpa_workspace_bytes) exceeds 16 MiB
  *     are rejected with SDPA_ERR_RESOURCES and a message; use sdpa_forward or
  *     sdpa_forward_ws for them.

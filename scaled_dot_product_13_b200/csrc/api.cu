@@ -15,6 +15,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -48,6 +49,26 @@ sdpa_status fail_str(sdpa_status st, const std::string &msg) {
   t_last_error = msg;
   return st;
 }
+
+// Test-only fault injection on the host, read once when the library loads
+// (no device fault is involved; the injected failure is a host-side error
+// return, taken before anything is enqueued):
+//   SDPA_TEST_FAIL_ALLOC=1      the stream-ordered workspace allocation of the
+//                               allocating entry points fails;
+//   SDPA_TEST_SMEM_LIMIT=<n>    the pre-launch resource check compares each
+//                               kernel's shared memory with n bytes instead of
+//                               the device's limit.
+struct TestHooks {
+  bool fail_alloc = false;
+  long long smem_limit = -1;
+  TestHooks() {
+    const char *a = getenv("SDPA_TEST_FAIL_ALLOC");
+    fail_alloc = a != nullptr && a[0] != '\0' && a[0] != '0';
+    const char *m = getenv("SDPA_TEST_SMEM_LIMIT");
+    if (m != nullptr && m[0] != '\0') smem_limit = atoll(m);
+  }
+};
+const TestHooks g_test_hooks;
 
 uint64_t wait_limit() {
   const uint64_t v = g_wait_limit_ns.load();
@@ -325,7 +346,29 @@ void fill_info(const Plan &pl, sdpa_plan_info *info) {
 constexpr int kMaxDevices = 64;
 std::mutex g_dev_mu;
 unsigned int *g_wd_ptr[kMaxDevices];
+unsigned long long g_wd_ctx[kMaxDevices];  // context id the address belongs to
 int g_num_sms[kMaxDevices];
+
+// cuCtxGetCurrent and cuCtxGetId from the driver (no libcuda link).
+struct CtxFns {
+  PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  PFN_cuCtxGetId_v12000 get_id = nullptr;
+};
+const CtxFns &ctx_fns() {
+  static CtxFns f;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      f.get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      f.get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  return f;
+}
 
 sdpa_status device_state(int *dev_out, int *sms_out, unsigned int **wd_out) {
   int dev = 0;
@@ -334,22 +377,33 @@ sdpa_status device_state(int *dev_out, int *sms_out, unsigned int **wd_out) {
     return fail(SDPA_ERR_CUDA, "no usable CUDA device: %s", cudaGetErrorString(e));
   if (dev < 0 || dev >= kMaxDevices) return fail(SDPA_ERR_CUDA, "device index %d too large", dev);
   std::lock_guard<std::mutex> lk(g_dev_mu);
-  if (!g_wd_ptr[dev]) {
-    cudaDeviceProp prop;
-    e = cudaGetDeviceProperties(&prop, dev);
-    if (e != cudaSuccess)
-      return fail(SDPA_ERR_CUDA, "cudaGetDeviceProperties: %s", cudaGetErrorString(e));
-    if (prop.major != 10 || prop.minor != 0)
-      return fail(SDPA_ERR_UNSUPPORTED,
-                  "libsdpa is built for sm_100a (B200); device %d is sm_%d%d", dev, prop.major,
-                  prop.minor);
-    void *ptr = nullptr;
-    e = cudaGetSymbolAddress(&ptr, g_sdpa_watchdog_word);
-    if (e != cudaSuccess)
-      return fail(SDPA_ERR_CUDA, "cudaGetSymbolAddress(watchdog): %s", cudaGetErrorString(e));
-    g_num_sms[dev] = prop.multiProcessorCount;
-    g_wd_ptr[dev] = static_cast<unsigned int *>(ptr);
+  // A device address looked up in one context is stale once that context is
+  // gone (cudaDeviceReset, say): the cache is keyed on the current context's
+  // id, which the driver never reuses within a process.
+  unsigned long long ctx = 0;
+  if (g_wd_ptr[dev] && current_context_id(&ctx) == SDPA_OK && ctx == g_wd_ctx[dev]) {
+    *dev_out = dev;
+    *sms_out = g_num_sms[dev];
+    *wd_out = g_wd_ptr[dev];
+    return SDPA_OK;
   }
+  cudaDeviceProp prop;
+  e = cudaGetDeviceProperties(&prop, dev);
+  if (e != cudaSuccess)
+    return fail(SDPA_ERR_CUDA, "cudaGetDeviceProperties: %s", cudaGetErrorString(e));
+  if (prop.major != 10 || prop.minor != 0)
+    return fail(SDPA_ERR_UNSUPPORTED,
+                "libsdpa is built for sm_100a (B200); device %d is sm_%d%d", dev, prop.major,
+                prop.minor);
+  void *ptr = nullptr;
+  e = cudaGetSymbolAddress(&ptr, g_sdpa_watchdog_word);
+  if (e != cudaSuccess)
+    return fail(SDPA_ERR_CUDA, "cudaGetSymbolAddress(watchdog): %s", cudaGetErrorString(e));
+  // the lookup made the device's context current
+  if (current_context_id(&ctx) != SDPA_OK) ctx = 0;
+  g_num_sms[dev] = prop.multiProcessorCount;
+  g_wd_ptr[dev] = static_cast<unsigned int *>(ptr);
+  g_wd_ctx[dev] = ctx;
   *dev_out = dev;
   *sms_out = g_num_sms[dev];
   *wd_out = g_wd_ptr[dev];
@@ -393,10 +447,12 @@ sdpa_status forward_call(const Problem &pb, const void *q, const void *k, const 
   bool allocated = false;
   if (pl.ws_bytes > 0) {
     if (own_ws) {
-      cudaError_t e = cudaMallocAsync(&ws, pl.ws_bytes, stream);
+      cudaError_t e = g_test_hooks.fail_alloc ? cudaErrorMemoryAllocation
+                                              : cudaMallocAsync(&ws, pl.ws_bytes, stream);
       if (e != cudaSuccess)
-        return fail(SDPA_ERR_CUDA, "cudaMallocAsync(%zu bytes) for the split workspace: %s",
-                    pl.ws_bytes, cudaGetErrorString(e));
+        return fail(SDPA_ERR_CUDA, "cudaMallocAsync(%zu bytes) for the split workspace: %s%s",
+                    pl.ws_bytes, cudaGetErrorString(e),
+                    g_test_hooks.fail_alloc ? " (injected by SDPA_TEST_FAIL_ALLOC)" : "");
       allocated = true;
     } else {
       if (ws == nullptr || ws_bytes < pl.ws_bytes)
@@ -438,6 +494,21 @@ sdpa_status forward_call(const Problem &pb, const void *q, const void *k, const 
   }
   if (st != SDPA_OK) return fail_str(st, err);
   return SDPA_OK;
+}
+
+sdpa_status current_context_id(unsigned long long *id) {
+  const CtxFns &f = ctx_fns();
+  CUcontext ctx = nullptr;
+  if (!f.get_current || !f.get_id || f.get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr)
+    return SDPA_ERR_CUDA;
+  return f.get_id(ctx, id) == CUDA_SUCCESS ? SDPA_OK : SDPA_ERR_CUDA;
+}
+
+sdpa_status validate_call(const Problem &pb, const void *q, const void *k, const void *v,
+                          const void *out) {
+  sdpa_status st = validate_shape(pb);
+  if (st != SDPA_OK) return st;
+  return validate_pointers(pb, q, k, v, out);
 }
 
 sdpa_status plan_call(const Problem &pb, int force_path, int force_splits, Plan *plan) {
@@ -507,6 +578,8 @@ sdpa_status prepare_kernel(const void *func, int threads, size_t smem, const cha
   }
   int max_optin = 0;
   cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (g_test_hooks.smem_limit >= 0 && g_test_hooks.smem_limit < max_optin)
+    max_optin = (int)g_test_hooks.smem_limit;
   char buf[256];
   if (attr.maxThreadsPerBlock < threads) {
     snprintf(buf, sizeof(buf), "%s: compiled kernel allows %d threads per block, launch needs %d",

@@ -126,6 +126,15 @@ sdpa_status forward_call(const Problem &pb, const void *q, const void *k, const 
                          bool own_ws, cudaStream_t stream, const float *sinks = nullptr,
                          float *lse_out = nullptr);
 
+// Host-side argument checks of every entry point (shape, then pointers); no
+// CUDA call.
+sdpa_status validate_call(const Problem &pb, const void *q, const void *k, const void *v,
+                          const void *out);
+
+// Id of the calling thread's current CUDA context (unique within the process,
+// never reused), or SDPA_ERR_CUDA when no context is current.
+sdpa_status current_context_id(unsigned long long *id);
+
 // Validate and plan for the current device without enqueuing anything.
 sdpa_status plan_call(const Problem &pb, int force_path, int force_splits, Plan *plan);
 

@@ -14,8 +14,9 @@
 // The array is a file-scope __device__ variable, so every GPU that loads the
 // library holds kNoAllocScratchBytes of device memory for it until the
 // process exits.  Host code cannot use the variable's name as a device
-// address; the address is looked up with cudaGetSymbolAddress once per
-// device, on the first call made while that device is current.
+// address; the address is looked up with cudaGetSymbolAddress on the first
+// call made while a device is current (and again if that device's context
+// has been replaced since).
 #include <cuda_runtime.h>
 
 #include <cstdio>
@@ -38,8 +39,12 @@ namespace {
 constexpr int kMaxDev = 64;
 std::mutex g_mu;
 void *g_scratch[kMaxDev];
+unsigned long long g_scratch_ctx[kMaxDev];  // context the address belongs to
 
-// Device address of the scratch array on the current device (looked up once).
+// Device address of the scratch array in the current device's context.  It is
+// looked up once per context: on the first call made on a device, and again
+// if that device's context was replaced since (after cudaDeviceReset, say, the
+// old address would be stale).
 sdpa_status scratch_address(void **out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -47,13 +52,17 @@ sdpa_status scratch_address(void **out) {
     return set_error(SDPA_ERR_CUDA, std::string("no usable CUDA device: ") + cudaGetErrorString(e));
   if (dev < 0 || dev >= kMaxDev) return set_error(SDPA_ERR_CUDA, "device index too large");
   std::lock_guard<std::mutex> lk(g_mu);
-  if (g_scratch[dev] == nullptr) {
+  unsigned long long ctx = 0;
+  if (g_scratch[dev] == nullptr || current_context_id(&ctx) != SDPA_OK ||
+      ctx != g_scratch_ctx[dev]) {
     void *ptr = nullptr;
     e = cudaGetSymbolAddress((void **)&ptr, g_sdpa_noalloc_scratch);
     if (e != cudaSuccess || ptr == nullptr)
       return set_error(SDPA_ERR_CUDA, std::string("cudaGetSymbolAddress(scratch): ") +
                                           cudaGetErrorString(e));
+    if (current_context_id(&ctx) != SDPA_OK) ctx = 0;
     g_scratch[dev] = ptr;
+    g_scratch_ctx[dev] = ctx;
   }
   *out = g_scratch[dev];
   return SDPA_OK;
@@ -75,8 +84,12 @@ extern "C" SDPA_API sdpa_status sdpa_forward_noalloc(const void *q, const void *
   pb.scale = scale; pb.causal = causal; pb.window = window_size; pb.dtype = dtype;
   pb.q_offset = S - L;  // queries end at the last key
   pb.has_q_offset = 0;
+  // host-side checks first, in the same order as sdpa_forward, before any
+  // CUDA call
+  sdpa_status st = validate_call(pb, q, k, v, out);
+  if (st != SDPA_OK) return st;
   Plan pl;
-  sdpa_status st = plan_call(pb, SDPA_PATH_AUTO, 0, &pl);
+  st = plan_call(pb, SDPA_PATH_AUTO, 0, &pl);
   if (st != SDPA_OK) return st;
   if (pl.ws_bytes > kNoAllocScratchBytes) {
     char buf[256];

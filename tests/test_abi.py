@@ -76,6 +76,18 @@ def test_forward_rejects_null_pointers_before_any_cuda_call(lib):
     assert b"non-NULL" in lib.sdpa_last_error_message()
 
 
+def test_noalloc_rejects_null_pointers_before_any_cuda_call(lib):
+    # same order of checks as sdpa_forward: shape, then pointers, then device
+    st = lib.sdpa_forward_noalloc(None, None, None, None, 1, 1, 1, 1, 1, 64, 64, 1.0, 0, 0, 0,
+                                  None)
+    assert st == 1
+    assert b"non-NULL" in lib.sdpa_last_error_message()
+    st = lib.sdpa_forward_noalloc(0x1000, 0x2000, 0x3000, 0x4000, 1, 6, 4, 1, 1, 64, 64, 1.0, 0,
+                                  0, 0, None)
+    assert st == 1
+    assert b"multiple of Hkv" in lib.sdpa_last_error_message()
+
+
 def test_forward_rejects_misaligned_pointers(lib):
     st = lib.sdpa_forward(0x1000, 0x2008, 0x3000, 0x4000, 1, 1, 1, 1, 1, 64, 64, 1.0, 0, 0, 0,
                           None)

@@ -4,8 +4,8 @@ The no-allocation entry point serves callers that cannot call cudaMalloc or
 cudaMallocAsync: split partials go to the library's fixed per-device scratch
 array instead of a workspace the call or the caller allocates.  Its output
 must match the allocating entry point within the GPU tolerance, on two calls
-in a row (the second call runs on scratch that still holds the first call's
-contents).  This file is collected last so that a stop at the first failure
+in a row that follow a call on other inputs of the same shape (so the scratch
+holds stale partials that differ from the right ones).  This file is collected last so that a stop at the first failure
 has already run every other test; it also passes on its own in a fresh
 process.
 """
@@ -31,6 +31,12 @@ CASES = [
 def test_noalloc_matches_allocating_entry_point(cuda_lib, p):
     q, k, v = (t.cuda() for t in I.make_qkv(p))
     ref = cuda_lib.forward(q, k, v, scale=p.sm_scale, causal=p.causal, window_size=p.window)
+    cuda_lib.device_status()
+    # leave partials of other inputs in the shared scratch first, so that an
+    # element the attention pass failed to write would show up as a mismatch
+    other = torch.empty_like(ref)
+    cuda_lib.forward_noalloc(-q, k.flip(2), v * 0.5, scale=p.sm_scale, causal=p.causal,
+                             window_size=p.window, out=other)
     cuda_lib.device_status()
     for _ in range(2):
         out = torch.full_like(ref, float("nan"))
