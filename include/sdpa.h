@@ -104,9 +104,12 @@ typedef enum {
                             whose four warps split the output columns, key
                             splits + combine as on SDPA_PATH_SPLITKV; the
                             only path for those head dims                    */
-  SDPA_PATH_TC_DUAL = 5  /* head dims up to 128: two 128-row tiles per CTA
+  SDPA_PATH_TC_DUAL = 5, /* head dims up to 128: two 128-row tiles per CTA
                             share each K/V block, their softmax phases
                             interleaved with each other's MMAs (tcgen05)     */
+  SDPA_PATH_TC_KSPLIT = 6 /* head dims up to 128: one 128-row tile per CTA
+                            whose two softmax groups take alternate key
+                            blocks, merged in the epilogue (tcgen05)        */
 } sdpa_path;
 
 /*

@@ -191,7 +191,7 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
     return fail(SDPA_ERR_UNSUPPORTED, "no kernel instance covers Dqk=%d, Dv=%d", pb.Dqk, pb.Dv);
   if (force_path != SDPA_PATH_AUTO && force_path != SDPA_PATH_SPLITKV &&
       force_path != SDPA_PATH_TC && force_path != SDPA_PATH_TC2 && force_path != SDPA_PATH_WIDE &&
-      force_path != SDPA_PATH_TC_DUAL)
+      force_path != SDPA_PATH_TC_DUAL && force_path != SDPA_PATH_TC_KSPLIT)
     return fail(SDPA_ERR_INVALID_ARG, "unknown path %d", force_path);
   // head dims above 256 run only on the column-split kernel, and it only on them
   const bool wide = pl.pair == kWidePair;
@@ -237,13 +237,18 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
     return fail(SDPA_ERR_UNSUPPORTED,
                 "the two-CTA path is built for head dims 256/256, 192/128 and 128/128 (got %d/%d)",
                 pb.Dqk, pb.Dv);
-  if (path == SDPA_PATH_TC_DUAL && !tc_dual_supports_pair(pl.pair))
+  if ((path == SDPA_PATH_TC_DUAL || path == SDPA_PATH_TC_KSPLIT) &&
+      !tc_dual_supports_pair(pl.pair))
     return fail(SDPA_ERR_UNSUPPORTED,
-                "the two-tile path is built for head dims up to 128 (got %d/%d)", pb.Dqk, pb.Dv);
+                "the two-tile paths are built for head dims up to 128 (got %d/%d)", pb.Dqk, pb.Dv);
   pl.path = path;
   if (path == SDPA_PATH_TC_DUAL) {
     pl.wr = 0; pl.wk = 0;
     pl.row_tile = 2 * kTcRows;
+    pl.key_block = 128;
+  } else if (path == SDPA_PATH_TC_KSPLIT) {
+    pl.wr = 0; pl.wk = 0;
+    pl.row_tile = kTcRows;
     pl.key_block = 128;
   } else if (path == SDPA_PATH_WIDE) {
     // one 16-row group (four warps) for decode-sized problems, two otherwise
@@ -480,7 +485,7 @@ sdpa_status forward_call(const Problem &pb, const void *q, const void *k, const 
   t_ev_start = t_ev_stop = t_ev_call = nullptr;
   st = pl.path == SDPA_PATH_TC2       ? launch_tc2(ln, &err)
        : pl.path == SDPA_PATH_TC      ? launch_tc(ln, &err)
-       : pl.path == SDPA_PATH_TC_DUAL ? launch_tc_pp(ln, &err)
+       : pl.path == SDPA_PATH_TC_DUAL || pl.path == SDPA_PATH_TC_KSPLIT ? launch_tc_pp(ln, &err)
        : pl.path == SDPA_PATH_WIDE    ? launch_wide(ln, &err)
                                       : launch_splitkv(ln, &err);
   if (st == SDPA_OK && pl.splits > 1) st = launch_combine(ln, &err);
@@ -526,9 +531,45 @@ sdpa_status set_error(sdpa_status st, const std::string &msg) { return fail_str(
 // ---------------------------------------------------------------------------
 // shared helpers declared in launch.h
 // ---------------------------------------------------------------------------
-bool encode_tma(CUtensorMap *map, sdpa_dtype dt, int rank, const void *base,
-                const uint64_t *dims, const uint64_t *strides_bytes, const uint32_t *box,
-                std::string *err) {
+namespace {
+// Recently encoded tensor maps of this host thread.  A descriptor depends only
+// on its arguments (no device state), so an eager loop of calls on the same
+// tensors reuses it instead of encoding it again; a few entries cover Q, K
+// and V of the last calls.
+struct TmaCacheEntry {
+  bool used;
+  int dt;  // CUtensorMapDataType
+  int rank;
+  const void *base;
+  uint64_t dims[3], strides[2];
+  uint32_t box[3];
+  CUtensorMap map;
+};
+constexpr int kTmaCacheSize = 12;
+thread_local TmaCacheEntry t_tma_cache[kTmaCacheSize];
+thread_local int t_tma_next = 0;
+
+bool tma_key_equal(const TmaCacheEntry &e, int dt, int rank, const void *base,
+                   const uint64_t *dims, const uint64_t *strides, const uint32_t *box) {
+  if (!e.used || e.dt != dt || e.rank != rank || e.base != base) return false;
+  for (int i = 0; i < rank; ++i)
+    if (e.dims[i] != dims[i] || e.box[i] != box[i]) return false;
+  for (int i = 0; i < rank - 1; ++i)
+    if (e.strides[i] != strides[i]) return false;
+  return true;
+}
+}  // namespace
+
+namespace {
+bool encode_tma_typed(CUtensorMap *map, int dt, int rank, const void *base, const uint64_t *dims,
+                      const uint64_t *strides_bytes, const uint32_t *box, std::string *err) {
+  if (rank >= 2 && rank <= 3) {
+    for (const TmaCacheEntry &e : t_tma_cache)
+      if (tma_key_equal(e, dt, rank, base, dims, strides_bytes, box)) {
+        *map = e.map;
+        return true;
+      }
+  }
   auto fn = encode_fn();
   if (!fn) {
     *err = "cuTensorMapEncodeTiled is not available from the driver";
@@ -542,8 +583,7 @@ bool encode_tma(CUtensorMap *map, sdpa_dtype dt, int rank, const void *base,
     estr[i] = 1;
   }
   for (int i = 0; i < rank - 1; ++i) gstr[i] = strides_bytes[i];
-  CUresult r = fn(map, dt == SDPA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-                  (cuuint32_t)rank, const_cast<void *>(base), gdim, gstr, bdim, estr,
+  CUresult r = fn(map, (CUtensorMapDataType)dt, (cuuint32_t)rank, const_cast<void *>(base), gdim, gstr, bdim, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
@@ -553,7 +593,55 @@ bool encode_tma(CUtensorMap *map, sdpa_dtype dt, int rank, const void *base,
     *err = buf;
     return false;
   }
+  if (rank >= 2 && rank <= 3) {
+    TmaCacheEntry &e = t_tma_cache[t_tma_next];
+    t_tma_next = (t_tma_next + 1) % kTmaCacheSize;
+    e.used = true;
+    e.dt = dt;
+    e.rank = rank;
+    e.base = base;
+    for (int i = 0; i < rank; ++i) {
+      e.dims[i] = dims[i];
+      e.box[i] = box[i];
+    }
+    for (int i = 0; i < rank - 1; ++i) e.strides[i] = strides_bytes[i];
+    e.map = *map;
+  }
   return true;
+}
+}  // namespace
+
+bool encode_tma(CUtensorMap *map, sdpa_dtype dt, int rank, const void *base,
+                const uint64_t *dims, const uint64_t *strides_bytes, const uint32_t *box,
+                std::string *err) {
+  return encode_tma_typed(map,
+                          dt == SDPA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                          : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                          rank, base, dims, strides_bytes, box, err);
+}
+
+bool encode_tma_f32(CUtensorMap *map, int rank, const void *base, const uint64_t *dims,
+                    const uint64_t *strides_bytes, const uint32_t *box, std::string *err) {
+  return encode_tma_typed(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, rank, base, dims, strides_bytes,
+                          box, err);
+}
+
+bool encode_out_maps(const Launch &ln, CUtensorMap *to, CUtensorMap *tp, std::string *err) {
+  const Problem &pb = ln.pb;
+  const Plan &pl = ln.plan;
+  const uint64_t slabs = (uint64_t)pb.B * pb.Hkv;
+  memset(to, 0, sizeof(*to));
+  memset(tp, 0, sizeof(*tp));
+  if (pl.splits == 1) {
+    const uint64_t dims[3] = {(uint64_t)pb.Dv, (uint64_t)pl.rows, slabs};
+    const uint64_t strides[2] = {(uint64_t)pb.Dv * 2, (uint64_t)pl.rows * pb.Dv * 2};
+    const uint32_t box[3] = {64, 128, 1};
+    return encode_tma(to, pb.dtype, 3, ln.out, dims, strides, box, err);
+  }
+  const uint64_t dims[3] = {(uint64_t)pb.Dv, (uint64_t)pl.rows, slabs * pl.splits};
+  const uint64_t strides[2] = {(uint64_t)pb.Dv * 4, (uint64_t)pl.rows * pb.Dv * 4};
+  const uint32_t box[3] = {32, 128, 1};
+  return encode_tma_f32(tp, 3, ln.part_o, dims, strides, box, err);
 }
 
 sdpa_status prepare_kernel(const void *func, int threads, size_t smem, const char *name,

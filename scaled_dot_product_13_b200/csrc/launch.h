@@ -147,6 +147,17 @@ bool encode_tma(CUtensorMap *map, sdpa_dtype dt, int rank, const void *base,
                 const uint64_t *dims, const uint64_t *strides_bytes, const uint32_t *box,
                 std::string *err);
 
+// The same for an fp32 tensor (split partials).
+bool encode_tma_f32(CUtensorMap *map, int rank, const void *base, const uint64_t *dims,
+                    const uint64_t *strides_bytes, const uint32_t *box, std::string *err);
+
+// Tensor maps of a call's output for the TMA-store epilogues, in boxes of 128
+// rows: `to` views out as [B*Hkv][R][Dv] (16-bit, 64-column boxes) when the
+// call is not split, `tp` views the fp32 partials as [splits*B*Hkv][R][Dv]
+// (32-column boxes) when it is; a packed-row slab is contiguous in both, so a
+// box never spills into the next slab.  The unused map is zeroed.
+bool encode_out_maps(const Launch &ln, CUtensorMap *to, CUtensorMap *tp, std::string *err);
+
 // Per-path launchers (return SDPA_OK or an error with *err set).
 sdpa_status launch_splitkv(const Launch &ln, std::string *err);
 sdpa_status launch_tc(const Launch &ln, std::string *err);

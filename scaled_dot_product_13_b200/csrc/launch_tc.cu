@@ -32,7 +32,7 @@ sdpa_status run_tc(const Launch &ln, std::string *err) {
 
   const Problem &pb = ln.pb;
   const Plan &pl = ln.plan;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to, tp;
   {
     const uint64_t dims[2] = {(uint64_t)pb.Dqk, (uint64_t)pb.B * pb.Hq * pb.L};
     const uint64_t strides[1] = {(uint64_t)pb.Dqk * 2};
@@ -51,6 +51,7 @@ sdpa_status run_tc(const Launch &ln, std::string *err) {
     const uint32_t box[3] = {64, (uint32_t)kBN, 1};
     if (!encode_tma(&tv, pb.dtype, 3, ln.v, dims, strides, box, err)) return SDPA_ERR_CUDA;
   }
+  if (!encode_out_maps(ln, &to, &tp, err)) return SDPA_ERR_CUDA;
   AttnParams p;
   p.B = pb.B; p.Hq = pb.Hq; p.Hkv = pb.Hkv; p.L = pb.L; p.S = pb.S; p.Dqk = pb.Dqk; p.Dv = pb.Dv;
   p.R = pl.rows;
@@ -70,7 +71,7 @@ sdpa_status run_tc(const Launch &ln, std::string *err) {
   p.wd.word = ln.wd_word;
   p.wd.limit_ns = ln.wd_limit_ns;
   if (ln.ev_start) record_event(ln.ev_start, ln.stream);
-  kern<<<(unsigned)pl.ctas, Cfg::kThreads, Cfg::kSmemBytes, ln.stream>>>(tq, tk, tv, p);
+  kern<<<(unsigned)pl.ctas, Cfg::kThreads, Cfg::kSmemBytes, ln.stream>>>(tq, tk, tv, to, tp, p);
   if (ln.ev_stop) record_event(ln.ev_stop, ln.stream);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {

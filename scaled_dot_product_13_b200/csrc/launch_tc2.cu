@@ -25,7 +25,7 @@ sdpa_status run_tc2(const Launch &ln, std::string *err) {
 
   const Problem &pb = ln.pb;
   const Plan &pl = ln.plan;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to, tp;
   {
     const uint64_t dims[2] = {(uint64_t)pb.Dqk, (uint64_t)pb.B * pb.Hq * pb.L};
     const uint64_t strides[1] = {(uint64_t)pb.Dqk * 2};
@@ -44,6 +44,7 @@ sdpa_status run_tc2(const Launch &ln, std::string *err) {
     const uint32_t box[3] = {64, (uint32_t)kBN, 1};
     if (!encode_tma(&tv, pb.dtype, 3, ln.v, dims, strides, box, err)) return SDPA_ERR_CUDA;
   }
+  if (!encode_out_maps(ln, &to, &tp, err)) return SDPA_ERR_CUDA;
   AttnParams p;
   p.B = pb.B; p.Hq = pb.Hq; p.Hkv = pb.Hkv; p.L = pb.L; p.S = pb.S; p.Dqk = pb.Dqk; p.Dv = pb.Dv;
   p.R = pl.rows;
@@ -76,7 +77,7 @@ sdpa_status run_tc2(const Launch &ln, std::string *err) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (ln.ev_start) record_event(ln.ev_start, ln.stream);
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, to, tp, p);
   if (ln.ev_stop) record_event(ln.ev_stop, ln.stream);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) {

@@ -1,4 +1,6 @@
-// Launch unit of the two-tile (ping-pong) tcgen05 kernel.
+// Launch unit of the two-tile (ping-pong) tcgen05 kernel: two 128-row tiles
+// per CTA (SDPA_PATH_TC_DUAL) or one tile whose two softmax groups take
+// alternate key blocks (SDPA_PATH_TC_KSPLIT).
 #include "launch.h"
 #include "tc_pp.cuh"
 
@@ -6,26 +8,27 @@ namespace sdpa {
 
 namespace {
 
-template <bool kBF16, int DQK, int DV>
+template <bool kBF16, int DQK, int DV, bool kKSplit>
 sdpa_status run_tc_pp(const Launch &ln, std::string *err) {
   constexpr int kBN = 128;
-  constexpr uint32_t kQ = 2u * ((DQK + 63) / 64) * 128 * 128;
+  constexpr uint32_t kQ = (kKSplit ? 1u : 2u) * ((DQK + 63) / 64) * 128 * 128;
   constexpr uint32_t kK = ((DQK + 63) / 64) * kBN * 128;
   constexpr uint32_t kV = ((DV + 63) / 64) * kBN * 128;
   constexpr uint32_t kSlot = kK > kV ? kK : kV;
-  constexpr uint32_t kBudget = 232448u - (2u * 8u + 10u) * 8u - 16u;
+  constexpr uint32_t kBudget =
+      232448u - (2u * 8u + 10u) * 8u - 16u - (kKSplit ? 2u * 128u * 8u : 0u);
   constexpr int kFit = (int)((kBudget - kQ) / kSlot);
   constexpr int kNSlot = kFit > 8 ? 8 : kFit;
   static_assert(kNSlot >= 2, "at least two K/V slots");
-  using Cfg = PpCfg<DQK, DV, kBN, kNSlot>;
-  auto kern = tc_pp_attn_kernel<kBF16, DQK, DV, kBN, kNSlot>;
+  using Cfg = PpCfg<DQK, DV, kBN, kNSlot, kKSplit>;
+  auto kern = tc_pp_attn_kernel<kBF16, DQK, DV, kBN, kNSlot, kKSplit>;
   sdpa_status st = prepare_kernel((const void *)kern, Cfg::kThreads, Cfg::kSmemBytes,
                                   "tc_pp_attn_kernel", err);
   if (st != SDPA_OK) return st;
 
   const Problem &pb = ln.pb;
   const Plan &pl = ln.plan;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to, tp;
   {
     const uint64_t dims[2] = {(uint64_t)pb.Dqk, (uint64_t)pb.B * pb.Hq * pb.L};
     const uint64_t strides[1] = {(uint64_t)pb.Dqk * 2};
@@ -44,6 +47,7 @@ sdpa_status run_tc_pp(const Launch &ln, std::string *err) {
     const uint32_t box[3] = {64, (uint32_t)kBN, 1};
     if (!encode_tma(&tv, pb.dtype, 3, ln.v, dims, strides, box, err)) return SDPA_ERR_CUDA;
   }
+  if (!encode_out_maps(ln, &to, &tp, err)) return SDPA_ERR_CUDA;
   AttnParams p;
   p.B = pb.B; p.Hq = pb.Hq; p.Hkv = pb.Hkv; p.L = pb.L; p.S = pb.S; p.Dqk = pb.Dqk; p.Dv = pb.Dv;
   p.R = pl.rows;
@@ -63,7 +67,7 @@ sdpa_status run_tc_pp(const Launch &ln, std::string *err) {
   p.wd.word = ln.wd_word;
   p.wd.limit_ns = ln.wd_limit_ns;
   if (ln.ev_start) record_event(ln.ev_start, ln.stream);
-  kern<<<(unsigned)pl.ctas, Cfg::kThreads, Cfg::kSmemBytes, ln.stream>>>(tq, tk, tv, p);
+  kern<<<(unsigned)pl.ctas, Cfg::kThreads, Cfg::kSmemBytes, ln.stream>>>(tq, tk, tv, to, tp, p);
   if (ln.ev_stop) record_event(ln.ev_stop, ln.stream);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -75,10 +79,13 @@ sdpa_status run_tc_pp(const Launch &ln, std::string *err) {
 
 template <bool kBF16>
 sdpa_status run_dtype(const Launch &ln, std::string *err) {
+  const bool ks = ln.plan.path == SDPA_PATH_TC_KSPLIT;
   switch (ln.plan.pair) {
-    case 0: return run_tc_pp<kBF16, 64, 64>(ln, err);
-    case 1: return run_tc_pp<kBF16, 80, 80>(ln, err);
-    case 2: return run_tc_pp<kBF16, 128, 128>(ln, err);
+    case 0: return ks ? run_tc_pp<kBF16, 64, 64, true>(ln, err) : run_tc_pp<kBF16, 64, 64, false>(ln, err);
+    case 1: return ks ? run_tc_pp<kBF16, 80, 80, true>(ln, err) : run_tc_pp<kBF16, 80, 80, false>(ln, err);
+    case 2:
+      return ks ? run_tc_pp<kBF16, 128, 128, true>(ln, err)
+                : run_tc_pp<kBF16, 128, 128, false>(ln, err);
   }
   *err = "internal: no two-tile instance for this head-dim pair";
   return SDPA_ERR_UNSUPPORTED;

@@ -346,6 +346,26 @@ __device__ __forceinline__ void tmem_st_u8x(uint32_t taddr, const uint32_t *v) {
                : "memory");
 }
 
+// TMA store of one box from shared memory to a 3-D tiled tensor (rows or
+// columns past the tensor's extent are not written), and the bulk-group
+// bookkeeping: commit the stores issued so far, and wait until they have
+// completed (their writes done, their shared-memory source free), so that
+// the writes are complete when the kernel is.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, const void *src, int x, int y,
+                                             int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_group0() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 // Prefetch one box of a tiled tensor into L2 (no shared memory, no barrier).
 __device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap *map, int x, int y) {
   asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(
@@ -556,6 +576,25 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
                "r"(d)
                : "memory");
+}
+
+// Output staging for TMA stores: boxes of 128 rows x 128 bytes, 128-byte
+// swizzled, 1024-byte aligned ([box][row][128 B]).  A thread writes its own
+// row; the swizzle spreads a warp's 32 rows over all banks.
+//   16 values of a 16-bit type, columns [16 c16, 16 c16 + 16): 64 per box
+__device__ __forceinline__ void stage_16bit_x16(uint8_t *stage, int row, int c16,
+                                                const uint32_t (&w8)[8]) {
+  const uint32_t box = smem_u32(stage + (c16 >> 2) * (128 * 128));
+  const uint32_t ch = (uint32_t)(c16 & 3) * 2;
+  st_shared_v4(box + sw128_offset(row, ch), w8[0], w8[1], w8[2], w8[3]);
+  st_shared_v4(box + sw128_offset(row, ch + 1), w8[4], w8[5], w8[6], w8[7]);
+}
+//   4 fp32 values, columns [4 c4, 4 c4 + 4): 32 per box
+__device__ __forceinline__ void stage_f32_x4(uint8_t *stage, int row, int c4, float a, float b,
+                                             float c, float d) {
+  const uint32_t box = smem_u32(stage + (c4 >> 3) * (128 * 128));
+  st_shared_v4(box + sw128_offset(row, (uint32_t)(c4 & 7)), __float_as_uint(a), __float_as_uint(b),
+               __float_as_uint(c), __float_as_uint(d));
 }
 
 // Instruction descriptor, kind::f16, fp32 accumulate, dense.

@@ -92,12 +92,17 @@ struct TcCfg {
   static_assert(kCols == 16 || kCols % 32 == 0, "TMEM load / store widths");
   static_assert(kBufs * BN + DV <= 512, "TMEM columns");
   static_assert(kSmemBytes <= 232448, "shared memory");
+  // the epilogue stages the tile's output rows in the K/V slots: 64 columns of
+  // a 16-bit type, or 32 fp32 split partials, per 16 KB box
+  static constexpr int kF32Boxes = (DV + 31) / 32;
+  static_assert(kF32Boxes * kBM * 128 <= NSLOT * kSlotBytes, "output staging");
 };
 
 template <bool kBF16, int DQK, int DV, int BN, int NSLOT>
 __global__ void __launch_bounds__(TcCfg<DQK, DV, BN, NSLOT>::kThreads, 1)
     tc_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                   const __grid_constant__ CUtensorMap tm_p, const AttnParams p) {
   using Cfg = TcCfg<DQK, DV, BN, NSLOT>;
   constexpr int NB = Cfg::kBufs;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -484,54 +489,61 @@ __global__ void __launch_bounds__(TcCfg<DQK, DV, BN, NSLOT>::kThreads, 1)
     const bool valid = r < tr.nvalid;
     const long grow = (long)bh * p.R + tr.row0 + r;
     const bool have_o = ok && nblk > 0;
-    float inv = l > 0.f ? 1.f / l : 0.f;
-    if (p.splits == 1) {
-      inv = finish_row(p, grow, m_used, l);
+    // Output rows are staged in the K/V slots (free: o_final fired once every
+    // MMA of the CTA had completed) in the TMA store's swizzled box layout,
+    // then one thread stores them in boxes of 128 rows; rows past the slab
+    // and columns past Dv are clipped by the tensor map.
+    const long total_rows = (long)p.B * p.Hq * p.L;
+    const bool split_out = p.splits > 1;
+    uint8_t *stage = sSlots;
+    auto load_o = [&](int c16, float (&o)[16]) {
+      if (have_o) {
+        tmem_ld16(tmem + lane_base + Cfg::kOCol + c16 * 16, o);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) o[e] = 0.f;
+      }
+    };
+    if (!split_out) {
+      const float inv = finish_row(p, grow, m_used, l);  // folds in the sink, if any
       if (p.lse_out != nullptr && valid && part == 0) p.lse_out[grow] = row_lse(m_used, l);
-      uint8_t *orow = reinterpret_cast<uint8_t *>(p.out) + grow * p.Dv * 2;
 #pragma unroll 1
       for (int c16 = oc_begin; c16 < oc_end; ++c16) {
         float o[16];
-        if (have_o) {
-          tmem_ld16(tmem + lane_base + Cfg::kOCol + c16 * 16, o);
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) o[e] = 0.f;
-        }
+        load_o(c16, o);
         uint32_t w8[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) w8[e] = pack2<kBF16>(o[2 * e] * inv, o[2 * e + 1] * inv);
-        const int col = c16 * 16;
-        if (valid && col + 8 <= p.Dv)
-          *reinterpret_cast<uint4 *>(orow + col * 2) = make_uint4(w8[0], w8[1], w8[2], w8[3]);
-        if (valid && col + 16 <= p.Dv)
-          *reinterpret_cast<uint4 *>(orow + col * 2 + 16) = make_uint4(w8[4], w8[5], w8[6], w8[7]);
+        stage_16bit_x16(stage, r, c16, w8);
       }
     } else {
-      const long total_rows = (long)p.B * p.Hq * p.L;
-      float *po = p.part_o + ((long)split * total_rows + grow) * p.Dv;
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      if (valid && part == 0)
+        p.part_lse[(long)split * total_rows + grow] = have_o ? row_lse(m_used, l) : -INFINITY;
 #pragma unroll 1
       for (int c16 = oc_begin; c16 < oc_end; ++c16) {
         float o[16];
-        if (have_o) {
-          tmem_ld16(tmem + lane_base + Cfg::kOCol + c16 * 16, o);
-          tmem_wait_ld();
-        } else {
+        load_o(c16, o);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) o[e] = 0.f;
-        }
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const int col = c16 * 16 + q4 * 4;
-          if (valid && col + 4 <= p.Dv)
-            *reinterpret_cast<float4 *>(po + col) =
-                make_float4(o[q4 * 4] * inv, o[q4 * 4 + 1] * inv, o[q4 * 4 + 2] * inv,
-                            o[q4 * 4 + 3] * inv);
-        }
+        for (int q4 = 0; q4 < 4; ++q4)
+          stage_f32_x4(stage, r, c16 * 4 + q4, o[q4 * 4] * inv, o[q4 * 4 + 1] * inv,
+                       o[q4 * 4 + 2] * inv, o[q4 * 4 + 3] * inv);
       }
-      if (valid && part == 0)
-        p.part_lse[(long)split * total_rows + grow] = have_o ? row_lse(m_used, l) : -INFINITY;
+    }
+    fence_proxy_async_smem();
+    asm volatile("bar.sync 1, %0;" ::"n"(Cfg::kSoftmaxWarps * 32) : "memory");  // softmax warps
+    if (warp == 0 && lane == 0 && tr.nvalid > 0) {
+      if (!split_out) {
+        for (int bx = 0; bx < Cfg::kVBoxes && bx * 64 < p.Dv; ++bx)
+          tma_store_3d(&tm_o, stage + bx * (Cfg::kBM * 128), bx * 64, tr.row0, bh);
+      } else {
+        for (int bx = 0; bx < Cfg::kF32Boxes && bx * 32 < p.Dv; ++bx)
+          tma_store_3d(&tm_p, stage + bx * (Cfg::kBM * 128), bx * 32, tr.row0,
+                       split * BH + bh);
+      }
+      bulk_commit_group();
+      bulk_wait_group0();
     }
   }
 

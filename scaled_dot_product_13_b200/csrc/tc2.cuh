@@ -65,12 +65,19 @@ struct Tc2Cfg {
   static_assert(BN == 128, "key block");
   static_assert(2 * BN + DV <= 512, "TMEM columns");
   static_assert(kSmemBytes <= 232448, "shared memory");
+  // the epilogue stages the CTA's 128 output rows in its K/V slots: 64
+  // columns of a 16-bit type, or 32 fp32 split partials, per 16 KB box
+  static constexpr int kOutBoxes = (DV + 63) / 64;
+  static constexpr int kF32Boxes = (DV + 31) / 32;
+  static_assert(kF32Boxes * kBM * 128 <= NSLOT * kSlotBytes, "output staging");
 };
 
 template <bool kBF16, int DQK, int DV, int BN, int NSLOT>
 __global__ void __launch_bounds__(224, 1)
     tc2_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+                    const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_o,
+                    const __grid_constant__ CUtensorMap tm_p, const AttnParams p) {
   using Cfg = Tc2Cfg<DQK, DV, BN, NSLOT>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // same layout in both CTAs, so both take this exit together
@@ -434,11 +441,16 @@ __global__ void __launch_bounds__(224, 1)
           for (int e = 0; e < 16; ++e) o[k][e] = 0.f;
       }
     };
-    float inv = l > 0.f ? 1.f / l : 0.f;
-    if (p.splits == 1) {
-      inv = finish_row(p, grow, m_used, l);
+    // Output rows are staged in this CTA's K/V slots (free: o_final fired
+    // once every MMA of the pair had completed) in the TMA store's swizzled
+    // box layout, then one thread stores them in boxes of 128 rows; rows past
+    // the slab and columns past Dv are clipped by the tensor map.
+    const long total_rows = (long)p.B * p.Hq * p.L;
+    const bool split_out = p.splits > 1;
+    uint8_t *stage = sSlots;
+    if (!split_out) {
+      const float inv = finish_row(p, grow, m_used, l);  // folds in the sink, if any
       if (p.lse_out != nullptr && valid) p.lse_out[grow] = row_lse(m_used, l);
-      uint8_t *orow = reinterpret_cast<uint8_t *>(p.out) + grow * p.Dv * 2;
 #pragma unroll 1
       for (int g = 0; g < kOChunks / kOGroup; ++g) {
         float o[kOGroup][16];
@@ -449,17 +461,13 @@ __global__ void __launch_bounds__(224, 1)
 #pragma unroll
           for (int e = 0; e < 8; ++e)
             w8[e] = pack2<kBF16>(o[k][2 * e] * inv, o[k][2 * e + 1] * inv);
-          const int col = (g * kOGroup + k) * 16;
-          if (valid && col + 8 <= p.Dv)
-            *reinterpret_cast<uint4 *>(orow + col * 2) = make_uint4(w8[0], w8[1], w8[2], w8[3]);
-          if (valid && col + 16 <= p.Dv)
-            *reinterpret_cast<uint4 *>(orow + col * 2 + 16) =
-                make_uint4(w8[4], w8[5], w8[6], w8[7]);
+          stage_16bit_x16(stage, r, g * kOGroup + k, w8);
         }
       }
     } else {
-      const long total_rows = (long)p.B * p.Hq * p.L;
-      float *po = p.part_o + ((long)split * total_rows + grow) * p.Dv;
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      if (valid)
+        p.part_lse[(long)split * total_rows + grow] = have_o ? row_lse(m_used, l) : -INFINITY;
 #pragma unroll 1
       for (int g = 0; g < kOChunks / kOGroup; ++g) {
         float o[kOGroup][16];
@@ -467,16 +475,24 @@ __global__ void __launch_bounds__(224, 1)
 #pragma unroll
         for (int k = 0; k < kOGroup; ++k)
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            const int col = (g * kOGroup + k) * 16 + q4 * 4;
-            if (valid && col + 4 <= p.Dv)
-              *reinterpret_cast<float4 *>(po + col) =
-                  make_float4(o[k][q4 * 4] * inv, o[k][q4 * 4 + 1] * inv, o[k][q4 * 4 + 2] * inv,
-                              o[k][q4 * 4 + 3] * inv);
-          }
+          for (int q4 = 0; q4 < 4; ++q4)
+            stage_f32_x4(stage, r, (g * kOGroup + k) * 4 + q4, o[k][q4 * 4] * inv,
+                         o[k][q4 * 4 + 1] * inv, o[k][q4 * 4 + 2] * inv, o[k][q4 * 4 + 3] * inv);
       }
-      if (valid)
-        p.part_lse[(long)split * total_rows + grow] = have_o ? row_lse(m_used, l) : -INFINITY;
+    }
+    fence_proxy_async_smem();
+    asm volatile("bar.sync 1, 128;" ::: "memory");  // the four softmax warps
+    if (warp == 0 && lane == 0 && tr.nvalid > 0) {
+      if (!split_out) {
+        for (int bx = 0; bx < Cfg::kOutBoxes && bx * 64 < p.Dv; ++bx)
+          tma_store_3d(&tm_o, stage + bx * (Cfg::kBM * 128), bx * 64, tr.row0, bh);
+      } else {
+        for (int bx = 0; bx < Cfg::kF32Boxes && bx * 32 < p.Dv; ++bx)
+          tma_store_3d(&tm_p, stage + bx * (Cfg::kBM * 128), bx * 32, tr.row0,
+                       split * BH + bh);
+      }
+      bulk_commit_group();
+      bulk_wait_group0();
     }
   }
 

@@ -31,6 +31,19 @@
 //              P_B(j) V_j, S_B(j+1).  Each K/V slot is released after its
 //              second use.
 //
+// Key-split mode (KSPLIT): one 128-row tile whose two softmax groups take
+// alternate key blocks instead of separate rows.  Group 0 takes blocks 0, 2,
+// 4, ... of the CTA's key range and group 1 blocks 1, 3, 5, ...; both use the
+// same Q tile, each K/V block is loaded once and used once (load order K_0,
+// K_1, V_0, K_2, V_1, K_3, ...; MMA order S_0(0), S_1(0), then per block b:
+// P(b) V_b, S(b + 2)).  Each group keeps its own running max, sum and O, and
+// the epilogue merges the two like two key splits (m = max(m_0, m_1),
+// O = (O_0 2^(m_0 - m) + O_1 2^(m_1 - m)) / (l_0 2^(m_0 - m) + l_1 2^(m_1 - m))),
+// each group writing half of the output columns.  This gives 128 rows the
+// same overlap of two softmax phases with each other's MMAs that the
+// row-pair mode gives 256 rows: for verify windows and short prefill whose
+// rows per KV head fill one 128-row tile, with keys to spare.
+//
 // TMEM: tile t uses columns [256 t, 256 t + BN) for S (P over the first BN/2
 // of them) and [256 t + BN, 256 t + BN + DV) for O.  With one score buffer
 // per tile, S_t(j+1) overwrites P_t(j) right after P_t(j) V is issued: one
@@ -43,7 +56,7 @@
 
 namespace sdpa {
 
-template <int DQK, int DV, int BN, int NSLOT>
+template <int DQK, int DV, int BN, int NSLOT, bool KSPLIT = false>
 struct PpCfg {
   static constexpr int kBM = 128;  // rows per tile
   static constexpr int kQBoxes = (DQK + 63) / 64;
@@ -51,12 +64,15 @@ struct PpCfg {
   static constexpr int kKS = DQK / 16;
   static constexpr int kPVK = BN / 16;
   static constexpr uint32_t kQTileBytes = kQBoxes * kBM * 128;
-  static constexpr uint32_t kQBytes = 2 * kQTileBytes;
+  static constexpr uint32_t kQBytes = (KSPLIT ? 1 : 2) * kQTileBytes;
   static constexpr uint32_t kKBytes = kQBoxes * BN * 128;
   static constexpr uint32_t kVBytes = kVBoxes * BN * 128;
   static constexpr uint32_t kSlotBytes = kKBytes > kVBytes ? kKBytes : kVBytes;
   static constexpr uint32_t kSlotOff = kQBytes;
-  static constexpr uint32_t kBarOff = kSlotOff + NSLOT * kSlotBytes;
+  // key-split merge: (m, l) of every row from each group
+  static constexpr uint32_t kXOff = kSlotOff + NSLOT * kSlotBytes;
+  static constexpr uint32_t kXBytes = KSPLIT ? 2 * kBM * 8 : 0;
+  static constexpr uint32_t kBarOff = kXOff + kXBytes;
   static constexpr int kNumBars = 2 * NSLOT + 10;
   static constexpr uint32_t kSmemBytes = kBarOff + kNumBars * 8 + 16;
   static constexpr int kThreads = 320;
@@ -67,14 +83,22 @@ struct PpCfg {
   static_assert(BN == 128, "key block");
   static_assert(BN + DV <= kTileCols, "TMEM columns per tile");
   static_assert(kSmemBytes <= 232448, "shared memory");
+  // the epilogue stages each tile's output rows in the K/V slots: 64 columns
+  // of a 16-bit type, or 32 fp32 split partials, per 16 KB box
+  static constexpr int kF32Boxes = (DV + 31) / 32;
+  static constexpr uint32_t kStage16 = kVBoxes * kBM * 128;
+  static constexpr uint32_t kStageF32 = kF32Boxes * kBM * 128;
+  static_assert((KSPLIT ? 1 : 2) * kStageF32 <= NSLOT * kSlotBytes, "output staging");
 };
 
-template <bool kBF16, int DQK, int DV, int BN, int NSLOT>
+template <bool kBF16, int DQK, int DV, int BN, int NSLOT, bool KSPLIT>
 __global__ void __launch_bounds__(320, 1)
     tc_pp_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
-                      const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
-  using Cfg = PpCfg<DQK, DV, BN, NSLOT>;
+                      const __grid_constant__ CUtensorMap tm_v,
+                      const __grid_constant__ CUtensorMap tm_o,
+                      const __grid_constant__ CUtensorMap tm_p, const AttnParams p) {
+  using Cfg = PpCfg<DQK, DV, BN, NSLOT, KSPLIT>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if ((smem_u32(smem_raw) & 1023u) != 0u) {
     if (threadIdx.x == 0) wd_record(p.wd, kWdSmemAlign);
@@ -96,18 +120,18 @@ __global__ void __launch_bounds__(320, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // --- work item: (batch*KV head) fastest, then split, then the 256-row
-  // tile, heaviest first ---
+  // --- work item: (batch*KV head) fastest, then split, then the row tile
+  // (256 rows, or 128 in key-split mode), heaviest first ---
   int bid = blockIdx.x;
   const int BH = p.B * p.Hkv;
   const int bh = bid % BH;
   bid /= BH;
   const int split = bid % p.splits;
   const int pair_tile = p.row_tiles - 1 - bid / p.splits;
-  const TileRows tpair = tile_rows(p, pair_tile, 2 * Cfg::kBM);
+  const TileRows tpair = tile_rows(p, pair_tile, (KSPLIT ? 1 : 2) * Cfg::kBM);
   int k_lo, k_hi;
   tile_key_range(p, tpair, BN, split, k_lo, k_hi);
-  const int nblk = (k_hi - k_lo) / BN;
+  const int nblk = (k_hi - k_lo) / BN;  // key blocks of the CTA (both groups together)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NSLOT; ++s) {
@@ -142,14 +166,55 @@ __global__ void __launch_bounds__(320, 1)
       const int grow0 = bh * p.R + tpair.row0;
       mbar_arrive_expect_tx(q_full, Cfg::kQBytes);
 #pragma unroll
-      for (int t = 0; t < 2; ++t)
+      for (int t = 0; t < (KSPLIT ? 1 : 2); ++t)
 #pragma unroll
         for (int bx = 0; bx < Cfg::kQBoxes; ++bx)
           tma_load_2d(sQ + t * Cfg::kQTileBytes + bx * (Cfg::kBM * 128), &tm_q, q_full, bx * 64,
                       grow0 + t * Cfg::kBM);
       int u = 0;
       bool ok = true;
-      for (int j = 0; ok && j < nblk; ++j) {
+      if constexpr (KSPLIT) {
+        // K_0, K_1, then V_b, K_{b+2} for b = 0, 1, ...: the order the MMA
+        // thread consumes them, each block used once
+        auto emit = [&](bool is_k, int blk) {
+          const int slot = u % NSLOT;
+          if (!mbar_wait(&slot_empty[slot], ((uint32_t)(u / NSLOT) & 1u) ^ 1u, p.wd,
+                         kWdTmaEmpty)) {
+            ok = false;
+            return;
+          }
+          uint8_t *dst = sSlots + slot * Cfg::kSlotBytes;
+          const int k0 = k_lo + blk * BN;
+          if (is_k) {
+            mbar_arrive_expect_tx(&slot_full[slot], Cfg::kKBytes);
+#pragma unroll
+            for (int bx = 0; bx < Cfg::kQBoxes; ++bx)
+              tma_load_3d(dst + bx * (BN * 128), &tm_k, &slot_full[slot], bx * 64, k0, bh);
+            const int pf = blk + Cfg::kPrefetch;
+            if (pf < nblk) {
+#pragma unroll
+              for (int bx = 0; bx < Cfg::kQBoxes; ++bx)
+                tma_prefetch_l2_3d(&tm_k, bx * 64, k_lo + pf * BN, bh);
+#pragma unroll
+              for (int bx = 0; bx < Cfg::kVBoxes; ++bx)
+                tma_prefetch_l2_3d(&tm_v, bx * 64, k_lo + pf * BN, bh);
+            }
+          } else {
+            mbar_arrive_expect_tx(&slot_full[slot], Cfg::kVBytes);
+#pragma unroll
+            for (int bx = 0; bx < Cfg::kVBoxes; ++bx)
+              tma_load_3d(dst + bx * (BN * 128), &tm_v, &slot_full[slot], bx * 64, k0, bh);
+          }
+          ++u;
+        };
+        if (nblk > 0) emit(true, 0);
+        if (ok && nblk > 1) emit(true, 1);
+        for (int b = 0; ok && b < nblk; ++b) {
+          emit(false, b);
+          if (ok && b + 2 < nblk) emit(true, b + 2);
+        }
+      }
+      for (int j = 0; !KSPLIT && ok && j < nblk; ++j) {
         const int k0 = k_lo + j * BN;
         for (int kv = 0; ok && kv < 2; ++kv, ++u) {
           const int slot = u % NSLOT;
@@ -226,35 +291,91 @@ __global__ void __launch_bounds__(320, 1)
         tc_fence_after();
         return true;
       };
-      if (ok && nblk > 0) {
-        ok = wait_load(0);
-        if (ok) {
-          tc_fence_after();
-          issue_s(0, 0);
-          issue_s(1, 0);
-          tc_commit(&slot_empty[slot_of(0)]);
-        }
-      }
-      for (int j = 0; ok && j < nblk; ++j) {
-        const bool more = j + 1 < nblk;
-        // tile A: P_A(j) V_j, then S_A(j+1)
-        ok = wait_load(2 * j + 1) && wait_p(0, j);
-        if (!ok) break;
-        issue_pv(0, j);
-        if (more) {
-          ok = wait_load(2 * j + 2);
+      if constexpr (KSPLIT) {
+        // key-split order: S_0(0) from K_0, S_1(0) from K_1, then per block b
+        // of the CTA (group b % 2): P(b) V_b, then S of the group's next block
+        // (K_{b+2}) into the buffer P(b) V_b has just been issued to read
+        int u = 0;
+        auto take = [&](int &slot) -> bool {  // the next load of the ring, in order
+          slot = u % NSLOT;
+          const bool w =
+              mbar_wait(&slot_full[slot], (uint32_t)(u / NSLOT) & 1u, p.wd, kWdTmaFull);
+          ++u;
+          return w;
+        };
+        auto s_into = [&](int t, int slot) {
+          const uint32_t kb = slot_addr + slot * Cfg::kSlotBytes;
+#pragma unroll
+          for (int ks = 0; ks < Cfg::kKS; ++ks) {
+            const uint64_t a =
+                umma_desc_sw128(q_addr + (ks >> 2) * (Cfg::kBM * 128) + (ks & 3) * 32, 16, 1024);
+            const uint64_t bd =
+                umma_desc_sw128(kb + (ks >> 2) * (BN * 128) + (ks & 3) * 32, 16, 1024);
+            tc_mma_ss(tmem + t * Cfg::kTileCols, a, bd, kIdescS, ks > 0 ? 1u : 0u);
+          }
+          tc_commit(&s_full[t]);
+          tc_commit(&slot_empty[slot]);
+        };
+        auto pv_from = [&](int t, int slot, bool first) {
+          const uint32_t vb = slot_addr + slot * Cfg::kSlotBytes;
+#pragma unroll
+          for (int ks = 0; ks < Cfg::kPVK; ++ks) {
+            const uint64_t bd = umma_desc_sw128_mn(vb + ks * 2048, BN * 128, 1024);
+            tc_mma_ts(tmem + t * Cfg::kTileCols + BN, tmem + t * Cfg::kTileCols + ks * 8, bd,
+                      kIdescPV, (!first || ks > 0) ? 1u : 0u);
+          }
+          tc_commit(&slot_empty[slot]);
+        };
+        int slot = 0;
+        for (int b = 0; ok && b < 2 && b < nblk; ++b) {
+          ok = take(slot);
           if (!ok) break;
           tc_fence_after();
-          issue_s(0, j + 1);
+          s_into(b, slot);
         }
-        // tile B: P_B(j) V_j, then S_B(j+1); each slot's second use frees it
-        ok = wait_p(1, j);
-        if (!ok) break;
-        issue_pv(1, j);
-        tc_commit(&slot_empty[slot_of(2 * j + 1)]);
-        if (more) {
-          issue_s(1, j + 1);
-          tc_commit(&slot_empty[slot_of(2 * j + 2)]);
+        for (int b = 0; ok && b < nblk; ++b) {
+          const int t = b & 1;
+          ok = take(slot) && wait_p(t, b >> 1);
+          if (!ok) break;
+          pv_from(t, slot, b < 2);
+          if (b + 2 < nblk) {
+            ok = take(slot);
+            if (!ok) break;
+            tc_fence_after();
+            s_into(t, slot);
+          }
+        }
+      } else {
+        if (ok && nblk > 0) {
+          ok = wait_load(0);
+          if (ok) {
+            tc_fence_after();
+            issue_s(0, 0);
+            issue_s(1, 0);
+            tc_commit(&slot_empty[slot_of(0)]);
+          }
+        }
+        for (int j = 0; ok && j < nblk; ++j) {
+          const bool more = j + 1 < nblk;
+          // tile A: P_A(j) V_j, then S_A(j+1)
+          ok = wait_load(2 * j + 1) && wait_p(0, j);
+          if (!ok) break;
+          issue_pv(0, j);
+          if (more) {
+            ok = wait_load(2 * j + 2);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(0, j + 1);
+          }
+          // tile B: P_B(j) V_j, then S_B(j+1); each slot's second use frees it
+          ok = wait_p(1, j);
+          if (!ok) break;
+          issue_pv(1, j);
+          tc_commit(&slot_empty[slot_of(2 * j + 1)]);
+          if (more) {
+            issue_s(1, j + 1);
+            tc_commit(&slot_empty[slot_of(2 * j + 2)]);
+          }
         }
       }
       if (ok && nblk > 0) {
@@ -272,7 +393,7 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const uint32_t s_col = (uint32_t)(t * Cfg::kTileCols);
     const uint32_t o_col = s_col + BN;
-    TileRows tr = tile_rows(p, pair_tile * 2 + t, Cfg::kBM);
+    TileRows tr = KSPLIT ? tpair : tile_rows(p, pair_tile * 2 + t, Cfg::kBM);
     if (tr.nvalid <= 0) {  // past the slab: compute on zeros, store nothing
       tr.nvalid = 0;
       tr.pos_min = tpair.pos_min;
@@ -289,7 +410,10 @@ __global__ void __launch_bounds__(320, 1)
     const float neutral = c_pos ? -INFINITY : INFINITY;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < nblk; ++j) {
+    // blocks of this group: all of the CTA's (row pairs), or every other one
+    // starting at block t (key split)
+    const int nb = KSPLIT ? (nblk - t + 1) / 2 : nblk;
+    for (int j = 0; j < nb; ++j) {
       bool w = true;
       if (lane == 0) w = mbar_wait(&s_full[t], (uint32_t)j & 1u, p.wd, kWdMma);
       if (!__shfl_sync(0xffffffffu, (int)w, 0)) {
@@ -307,7 +431,7 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
         for (int i = 0; i < BN; ++i) s[i] = 0.f;
       }
-      const int kbase = k_lo + j * BN;
+      const int kbase = k_lo + (KSPLIT ? 2 * j + t : j) * BN;
       const bool masked = block_needs_mask(p, tr, kbase, BN);
       if (masked) {
         const VisibleRange vis = visible_range(p, pos, kbase);
@@ -395,75 +519,111 @@ __global__ void __launch_bounds__(320, 1)
     }
 
     // ------------------------------ epilogue ------------------------------
+    // Output rows go to shared memory in the TMA store's swizzled box layout
+    // (the K/V slots are free once o_final has fired: every MMA of the CTA
+    // has completed by then), then one thread stores the boxes; rows past
+    // the slab and columns past Dv are clipped by the tensor map.  In
+    // key-split mode the two groups' (m, l, O) are merged first and each
+    // group stages half of the columns.
     if (ok && nblk > 0) {
       bool w = true;
-      if (lane == 0) w = mbar_wait(&o_final[t], 0, p.wd, kWdMma);
+      if (lane == 0) {
+        if constexpr (KSPLIT)
+          w = mbar_wait(&o_final[0], 0, p.wd, kWdMma) && mbar_wait(&o_final[1], 0, p.wd, kWdMma);
+        else
+          w = mbar_wait(&o_final[t], 0, p.wd, kWdMma);
+      }
       ok = __shfl_sync(0xffffffffu, (int)w, 0) != 0;
       tc_fence_after();
     }
+    constexpr int kOChunks = DV / 16;
+    float m_row = m_used, l_row = l, f0 = 1.f, f1 = 0.f;
+    bool have0, have1;  // group (tile) 0 / 1 holds O that this thread reads
+    int oc_begin = 0, oc_end = kOChunks;
+    if constexpr (KSPLIT) {
+      float2 *xml = reinterpret_cast<float2 *>(smem + Cfg::kXOff);  // [group][row]
+      xml[t * Cfg::kBM + r] = make_float2(m_used, l);
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      const float2 other = xml[(1 - t) * Cfg::kBM + r];
+      m_row = fmaxf(m_used, other.x);
+      const float mref = m_row == -INFINITY ? 0.f : m_row;
+      const float f_self = m_used == -INFINITY ? 0.f : exp2f(m_used - mref);
+      const float f_other = other.x == -INFINITY ? 0.f : exp2f(other.x - mref);
+      l_row = l * f_self + other.y * f_other;
+      f0 = t == 0 ? f_self : f_other;
+      f1 = t == 0 ? f_other : f_self;
+      have0 = ok && nblk > 0;
+      have1 = ok && nblk > 1;  // group 1 has a block
+      constexpr int kHalf = (kOChunks + 1) / 2;
+      oc_begin = t == 0 ? 0 : kHalf;
+      oc_end = t == 0 ? kHalf : kOChunks;
+    } else {
+      have0 = ok && nblk > 0;  // this tile's own O
+      have1 = false;
+    }
+    // 16 output columns of this row from TMEM (both groups' O, weighted, in
+    // key-split mode; the tile's own O otherwise)
+    auto load_o = [&](int c16, float (&o)[16]) {
+      float a[16], b[16];
+      const uint32_t own = KSPLIT ? (uint32_t)BN : o_col;
+      if (have0) tmem_ld16(tmem + lane_base + own + c16 * 16, a);
+      if (KSPLIT && have1) tmem_ld16(tmem + lane_base + Cfg::kTileCols + BN + c16 * 16, b);
+      if (have0 || have1) tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+        o[e] = (have0 ? a[e] * f0 : 0.f) + (KSPLIT && have1 ? b[e] * f1 : 0.f);
+    };
     const bool valid = r < tr.nvalid;
     const long grow = (long)bh * p.R + tr.row0 + r;
-    const bool have_o = ok && nblk > 0;
-    // O leaves TMEM kOGroup chunks of 16 columns per wait
-    constexpr int kOChunks = DV / 16;
-    constexpr int kOGroup = kOChunks <= 5 ? kOChunks : 4;
-    static_assert(kOChunks % kOGroup == 0, "whole groups of O chunks");
-    auto load_o = [&](int g, float (&o)[kOGroup][16]) {
-      if (have_o) {
-    #pragma unroll
-        for (int k = 0; k < kOGroup; ++k)
-          tmem_ld16(tmem + lane_base + o_col + (g * kOGroup + k) * 16, o[k]);
-        tmem_wait_ld();
-      } else {
-    #pragma unroll
-        for (int k = 0; k < kOGroup; ++k)
-    #pragma unroll
-          for (int e = 0; e < 16; ++e) o[k][e] = 0.f;
-      }
-    };
-    float inv = l > 0.f ? 1.f / l : 0.f;
-    if (p.splits == 1) {
-      inv = finish_row(p, grow, m_used, l);
-      if (p.lse_out != nullptr && valid) p.lse_out[grow] = row_lse(m_used, l);
-      uint8_t *orow = reinterpret_cast<uint8_t *>(p.out) + grow * p.Dv * 2;
+    const long total_rows = (long)p.B * p.Hq * p.L;
+    const bool split_out = p.splits > 1;
+    uint8_t *stage =
+        sSlots + (KSPLIT ? 0 : t * (split_out ? Cfg::kStageF32 : Cfg::kStage16));
+    if (!split_out) {
+      const float inv = finish_row(p, grow, m_row, l_row);  // folds in the sink, if any
+      if (p.lse_out != nullptr && valid && (!KSPLIT || t == 0))
+        p.lse_out[grow] = row_lse(m_row, l_row);
 #pragma unroll 1
-      for (int g = 0; g < kOChunks / kOGroup; ++g) {
-        float o[kOGroup][16];
-        load_o(g, o);
+      for (int c16 = oc_begin; c16 < oc_end; ++c16) {
+        float o[16];
+        load_o(c16, o);
+        uint32_t w8[8];
 #pragma unroll
-        for (int k = 0; k < kOGroup; ++k) {
-          uint32_t w8[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            w8[e] = pack2<kBF16>(o[k][2 * e] * inv, o[k][2 * e + 1] * inv);
-          const int col = (g * kOGroup + k) * 16;
-          if (valid && col + 8 <= p.Dv)
-            *reinterpret_cast<uint4 *>(orow + col * 2) = make_uint4(w8[0], w8[1], w8[2], w8[3]);
-          if (valid && col + 16 <= p.Dv)
-            *reinterpret_cast<uint4 *>(orow + col * 2 + 16) =
-                make_uint4(w8[4], w8[5], w8[6], w8[7]);
-        }
+        for (int e = 0; e < 8; ++e) w8[e] = pack2<kBF16>(o[2 * e] * inv, o[2 * e + 1] * inv);
+        stage_16bit_x16(stage, r, c16, w8);
       }
     } else {
-      const long total_rows = (long)p.B * p.Hq * p.L;
-      float *po = p.part_o + ((long)split * total_rows + grow) * p.Dv;
+      const float inv = l_row > 0.f ? 1.f / l_row : 0.f;
+      if (valid && (!KSPLIT || t == 0))
+        p.part_lse[(long)split * total_rows + grow] = have0 ? row_lse(m_row, l_row) : -INFINITY;
 #pragma unroll 1
-      for (int g = 0; g < kOChunks / kOGroup; ++g) {
-        float o[kOGroup][16];
-        load_o(g, o);
+      for (int c16 = oc_begin; c16 < oc_end; ++c16) {
+        float o[16];
+        load_o(c16, o);
 #pragma unroll
-        for (int k = 0; k < kOGroup; ++k)
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            const int col = (g * kOGroup + k) * 16 + q4 * 4;
-            if (valid && col + 4 <= p.Dv)
-              *reinterpret_cast<float4 *>(po + col) =
-                  make_float4(o[k][q4 * 4] * inv, o[k][q4 * 4 + 1] * inv, o[k][q4 * 4 + 2] * inv,
-                              o[k][q4 * 4 + 3] * inv);
-          }
+        for (int q4 = 0; q4 < 4; ++q4)
+          stage_f32_x4(stage, r, c16 * 4 + q4, o[q4 * 4] * inv, o[q4 * 4 + 1] * inv,
+                       o[q4 * 4 + 2] * inv, o[q4 * 4 + 3] * inv);
       }
-      if (valid)
-        p.part_lse[(long)split * total_rows + grow] = have_o ? row_lse(m_used, l) : -INFINITY;
+    }
+    fence_proxy_async_smem();
+    if constexpr (KSPLIT)
+      asm volatile("bar.sync 1, 256;" ::: "memory");  // both groups
+    else if (t == 0)  // this tile's four warps
+      asm volatile("bar.sync 2, 128;" ::: "memory");
+    else
+      asm volatile("bar.sync 3, 128;" ::: "memory");
+    if ((KSPLIT ? warp == 0 : quarter == 0) && lane == 0 && tr.nvalid > 0) {
+      if (!split_out) {
+        for (int bx = 0; bx < Cfg::kVBoxes && bx * 64 < p.Dv; ++bx)
+          tma_store_3d(&tm_o, stage + bx * (Cfg::kBM * 128), bx * 64, tr.row0, bh);
+      } else {
+        for (int bx = 0; bx < Cfg::kF32Boxes && bx * 32 < p.Dv; ++bx)
+          tma_store_3d(&tm_p, stage + bx * (Cfg::kBM * 128), bx * 32, tr.row0,
+                       split * BH + bh);
+      }
+      bulk_commit_group();
+      bulk_wait_group0();
     }
   }
 
