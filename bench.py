@@ -384,6 +384,30 @@ def time_stream(sdpa, c, flush, l2_bytes, reps=6, warmup=2, max_copies=32,
     return statistics.mean(ts), n
 
 
+def time_alone(sdpa, c, flush, reps=20, warmup=3):
+    """One call captured alone in a CUDA graph, replayed after an L2 flush,
+    with events around the replay on the stream (no event inside the graph).
+    Returns microseconds per call (mean over ``reps``)."""
+    stream = torch.cuda.current_stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        sdpa.forward_ws(c.q, c.k, c.v, c.ws, scale=c.p.sm_scale, causal=c.p.causal,
+                        window_size=c.p.window, out=c.out)
+    torch.cuda.synchronize()
+    ts = []
+    for it in range(warmup + reps):
+        flush_l2(flush)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if it >= warmup:
+            ts.append(e0.elapsed_time(e1) * 1e3)
+    del g
+    return statistics.mean(ts)
+
+
 def secondary(sdpa, probs, steps, warmup, flush, sync_all, device, peaks, kind, graphs=True,
               stream=False):
     """Time a list of problems (one call each per step); return a summary.
@@ -393,10 +417,16 @@ def secondary(sdpa, probs, steps, warmup, flush, sync_all, device, peaks, kind, 
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     pts = []
     for c, cm, mm in zip(cases, call_ms, main_ms):
-        # mean over the timed steps: the device timer's coarse steps make a
-        # median jump between neighbouring values
-        us = 1e3 * statistics.mean(cm)
-        d = {"name": c.p.name, "us": round(us, 2), "us_median": round(1e3 * statistics.median(cm), 2),
+        # the call timed alone: a graph holding only the call, replayed after
+        # an L2 flush, events on the stream around the replay.  us_events is
+        # the same call bracketed by events the library records inside the
+        # graph, which carry several microseconds of their own (mean over the
+        # timed steps: the device timer's coarse steps make a median jump
+        # between neighbouring values)
+        us = time_alone(sdpa, c, flush, reps=max(steps, 20)) if graphs else 1e3 * statistics.mean(cm)
+        d = {"name": c.p.name, "us": round(us, 2),
+             "us_events": round(1e3 * statistics.mean(cm), 2),
+             "us_events_median": round(1e3 * statistics.median(cm), 2),
              "path": c.info["path"], "splits": c.info["splits"]}
         if kind == "tflops":
             tf = c.flops / (us * 1e-6) / 1e12
@@ -463,7 +493,9 @@ def main():
                           "(points) = library events before the split pass and after the call's "
                           "last launch, each call replayed alone after an L2 flush, mean over the "
                           "timed steps; main-kernel time from probe replays with an event after "
-                          "the split pass; prefill and verify us_stream = calls back to back on "
+                          "the split pass; prefill, verify, tiny and wide us = a graph of the call "
+                          "alone replayed after an L2 flush, events around the replay (us_events: "
+                          "library events inside the graph); us_stream = calls back to back on "
                           "rotating input copies totalling more than 2x L2, per call",
                 "parallelism": f"replicas x{world} (independent KV-head units, no collective)"}
 
@@ -573,8 +605,13 @@ def main():
     if not args.no_secondary:
         sec_steps = max(3, min(args.steps, 20))
         gr = not args.eager
-        extra["prefill"] = secondary(sdpa, I.window_problems() + I.encoder_problems(), sec_steps,
+        # the 32K causal call runs last: seconds of full tensor load lower the
+        # clock under the power cap for a while, which would slow the calls
+        # timed right after it
+        win = I.window_problems()
+        extra["prefill"] = secondary(sdpa, win[:3] + I.encoder_problems() + win[3:], sec_steps,
                                      3, flush, sync_all, device, peaks, "tflops", gr, stream=True)
+        time.sleep(1.0)
         # the verify sweep checks monotonicity in L between calls whose times
         # differ by about a microsecond: 60 samples per call (cheap at ~40 us)
         extra["verify"] = secondary(sdpa, I.verify_problems(), max(sec_steps, 60), 3, flush,

@@ -131,4 +131,39 @@ __device__ __forceinline__ VisibleRange visible_range(const AttnParams &p, int p
   return v;
 }
 
+// Maximum (or minimum) of a row's N scores of one block, in four chains of
+// three-input max (min) operations.
+template <int N>
+__device__ __forceinline__ float row_reduce_max(const float (&s)[N]) {
+  float mr[4];
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) mr[q4] = s[q4];
+#pragma unroll
+  for (int i = 4; i < N; i += 8) {
+    mr[0] = fmax3f(mr[0], s[i], s[i + 1]);
+    mr[1] = fmax3f(mr[1], s[i + 2], s[i + 3]);
+    if (i + 4 < N) {
+      mr[2] = fmax3f(mr[2], s[i + 4], s[i + 5]);
+      mr[3] = fmax3f(mr[3], s[i + 6], s[i + 7]);
+    }
+  }
+  return fmax3f(mr[0], mr[1], fmaxf(mr[2], mr[3]));
+}
+template <int N>
+__device__ __forceinline__ float row_reduce_min(const float (&s)[N]) {
+  float mr[4];
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) mr[q4] = s[q4];
+#pragma unroll
+  for (int i = 4; i < N; i += 8) {
+    mr[0] = fmin3f(mr[0], s[i], s[i + 1]);
+    mr[1] = fmin3f(mr[1], s[i + 2], s[i + 3]);
+    if (i + 4 < N) {
+      mr[2] = fmin3f(mr[2], s[i + 4], s[i + 5]);
+      mr[3] = fmin3f(mr[3], s[i + 6], s[i + 7]);
+    }
+  }
+  return fmin3f(mr[0], mr[1], fminf(mr[2], mr[3]));
+}
+
 }  // namespace sdpa

@@ -314,43 +314,26 @@ __global__ void __launch_bounds__(224, 1)
         tmem_ld32(tmem + lane_base + b * BN + c32 * 32, s + c32 * 32);
       tmem_wait_ld();
 
-      if (c_zero) {
-#pragma unroll
-        for (int i = 0; i < BN; ++i) s[i] = 0.f;
-      }
       const int kbase = k_lo + j * BN;
       const bool masked = block_needs_mask(p, tr, kbase, BN);
-      if (masked) {
-        const VisibleRange vis = visible_range(p, pos, kbase);
-#pragma unroll
-        for (int i = 0; i < BN; ++i)
-          if (!vis(i)) s[i] = neutral;
-      }
-      float mr[4];
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) mr[q4] = s[q4];
-      if (c_pos) {
-#pragma unroll
-        for (int i = 4; i < BN; i += 8) {
-          mr[0] = fmax3f(mr[0], s[i], s[i + 1]);
-          mr[1] = fmax3f(mr[1], s[i + 2], s[i + 3]);
-          if (i + 4 < BN) {
-            mr[2] = fmax3f(mr[2], s[i + 4], s[i + 5]);
-            mr[3] = fmax3f(mr[3], s[i + 6], s[i + 7]);
-          }
-        }
-        mr[0] = fmax3f(mr[0], mr[1], fmaxf(mr[2], mr[3]));
+      // The common block (positive scale, no masked key) takes the plain
+      // reduction; the rare ones (scale 0, masked keys, negative scale) their
+      // own copy, so that their per-element work is not folded into it.
+      float mr[1];
+      if (!masked && c_pos && !c_zero) {
+        mr[0] = row_reduce_max(s);
       } else {
+        if (c_zero) {
 #pragma unroll
-        for (int i = 4; i < BN; i += 8) {
-          mr[0] = fmin3f(mr[0], s[i], s[i + 1]);
-          mr[1] = fmin3f(mr[1], s[i + 2], s[i + 3]);
-          if (i + 4 < BN) {
-            mr[2] = fmin3f(mr[2], s[i + 4], s[i + 5]);
-            mr[3] = fmin3f(mr[3], s[i + 6], s[i + 7]);
-          }
+          for (int i = 0; i < BN; ++i) s[i] = 0.f;
         }
-        mr[0] = fmin3f(mr[0], mr[1], fminf(mr[2], mr[3]));
+        if (masked) {
+          const VisibleRange vis = visible_range(p, pos, kbase);
+#pragma unroll
+          for (int i = 0; i < BN; ++i)
+            if (!vis(i)) s[i] = neutral;
+        }
+        mr[0] = c_pos ? row_reduce_max(s) : row_reduce_min(s);
       }
       const float mblk = isinf(mr[0]) ? -INFINITY : mr[0] * c_eff;
       const float m_new = fmaxf(m_used, mblk);
