@@ -186,6 +186,7 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
                       Plan *out) {
   Plan pl;
   memset(&pl, 0, sizeof(pl));
+  pl.col_halves = 1;
   pl.pair = pick_pair(pb.Dqk, pb.Dv);
   if (pl.pair < 0)
     return fail(SDPA_ERR_UNSUPPORTED, "no kernel instance covers Dqk=%d, Dv=%d", pb.Dqk, pb.Dv);
@@ -193,12 +194,19 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
       force_path != SDPA_PATH_TC && force_path != SDPA_PATH_TC2 && force_path != SDPA_PATH_WIDE &&
       force_path != SDPA_PATH_TC_DUAL && force_path != SDPA_PATH_TC_KSPLIT)
     return fail(SDPA_ERR_INVALID_ARG, "unknown path %d", force_path);
-  // head dims above 256 run only on the column-split kernel, and it only on them
+  // head dims above 256 run on the column-split warp-tile kernel (decode and
+  // short verify windows) or on the tcgen05 kernel in column halves; the
+  // column-split kernel only on them
   const bool wide = pl.pair == kWidePair;
-  if (force_path != SDPA_PATH_AUTO && (force_path == SDPA_PATH_WIDE) != wide)
+  if (force_path == SDPA_PATH_WIDE && !wide)
     return fail(SDPA_ERR_UNSUPPORTED,
-                wide ? "head dims above 256 (got Dqk=%d, Dv=%d) run only on the wide path"
-                     : "the wide path is built for head dims above 256 (got Dqk=%d, Dv=%d)",
+                "the wide path is built for head dims above 256 (got Dqk=%d, Dv=%d)", pb.Dqk,
+                pb.Dv);
+  if (wide && force_path != SDPA_PATH_AUTO && force_path != SDPA_PATH_WIDE &&
+      force_path != SDPA_PATH_TC)
+    return fail(SDPA_ERR_UNSUPPORTED,
+                "head dims above 256 (got Dqk=%d, Dv=%d) run on the wide path or the tcgen05 "
+                "path",
                 pb.Dqk, pb.Dv);
   if (force_splits < 0) return fail(SDPA_ERR_INVALID_ARG, "force_splits must be >= 0");
   if (num_sms < 1) num_sms = 148;
@@ -210,7 +218,9 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
   // split-KV kernel on 16-row warp tiles.  Both split the keys when the
   // tiles alone do not fill the GPU.
   int path = force_path;
-  if (path == SDPA_PATH_AUTO && wide) path = SDPA_PATH_WIDE;
+  // head dims above 256: packed rows that fill a 128-row tile take tcgen05
+  if (path == SDPA_PATH_AUTO && wide)
+    path = pl.rows >= kTcRowThreshold ? SDPA_PATH_TC : SDPA_PATH_WIDE;
   if (path == SDPA_PATH_AUTO) {
     path = pl.rows >= kTcRowThreshold ? SDPA_PATH_TC : SDPA_PATH_SPLITKV;
     // wide heads with at least one full 256-row pair tile: two SMs per tile
@@ -264,6 +274,7 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
     pl.wr = 0; pl.wk = 0;
     pl.row_tile = kTcRows;
     pl.key_block = tc_key_block(kDimPairs[pl.pair].dqk, kDimPairs[pl.pair].dv);
+    if (wide) pl.col_halves = (pb.Dv + kTcWideHalf - 1) / kTcWideHalf;
   } else {
     if (pl.rows <= 16) {
       // one 16-row group: 16 keys per warp of every key block
@@ -286,9 +297,11 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
   const int bn = pl.key_block;
   pl.split_base = (kbeg / bn) * bn;
   const int nkb = std::max(1, (kend + bn - 1) / bn - kbeg / bn);
-  // CTAs per split: one per row tile, two per pair tile
+  // CTAs per split: one per row tile, two per pair tile, two per row tile
+  // (one per column half) for the tcgen05 kernel at head dims above 256
   const long long per_tile = pl.path == SDPA_PATH_TC2 ? 2 : 1;
-  const long long base = (long long)pb.B * pb.Hkv * pl.row_tiles * per_tile;
+  const bool tc_wide = path == SDPA_PATH_TC && wide;
+  const long long base = (long long)pb.B * pb.Hkv * pl.row_tiles * per_tile * pl.col_halves;
   // resident CTAs per SM (the split-KV kernel runs two where they fit)
   const long long slots =
       (long long)num_sms * (path == SDPA_PATH_SPLITKV
@@ -299,15 +312,16 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
   if (force_splits > 0) {
     splits = std::min(force_splits, nkb);
   } else if (base >= slots || (path == SDPA_PATH_SPLITKV ? nkb * bn <= kNoSplitBlocks * 64
-                                                          : nkb <= kNoSplitBlocks)) {
+                                : tc_wide              ? nkb * bn <= kNoSplitBlocks * 128
+                                                       : nkb <= kNoSplitBlocks)) {
     splits = 1;
   } else {
     // the wide kernel's 32-key blocks are small and its partials wide
     // (Dv up to 512 floats per row and split): give each split more keys.
     // The split-KV kernel's splits cover at least 128 keys whatever its block.
-    const int min_blocks = path == SDPA_PATH_WIDE      ? kMinBlocksPerSplitWide
-                           : path == SDPA_PATH_SPLITKV ? std::max(1, 128 / bn)
-                                                       : kMinBlocksPerSplit;
+    const int min_blocks = path == SDPA_PATH_WIDE || tc_wide ? kMinBlocksPerSplitWide
+                           : path == SDPA_PATH_SPLITKV      ? std::max(1, 128 / bn)
+                                                            : kMinBlocksPerSplit;
     splits = (int)std::max(1LL, slots / base);
     splits = std::min(splits, std::max(1, nkb / min_blocks));
   }
@@ -316,7 +330,7 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
   if (force_splits == 0) splits = (nkb + bps - 1) / bps;
   pl.splits = splits;
   pl.keys_per_split = bps * bn;
-  pl.ctas = (base / per_tile) * splits;
+  pl.ctas = (base / per_tile) * splits;  // all CTAs: grid.x * col_halves
   if (pl.ctas > 0x7fffffffLL)
     return fail(SDPA_ERR_UNSUPPORTED, "problem needs %lld CTAs, above the grid limit", pl.ctas);
   pl.launches = splits > 1 ? 2 : 1;

@@ -72,8 +72,16 @@ constexpr int splitkv_ctas_per_sm(int dqk, int dv, int wr) {
 }
 
 // Key block of the tcgen05 kernel: 128 keys while two 128-key score buffers
-// plus O fit TMEM and the slots fit shared memory; 64 for head dims > 128.
-constexpr int tc_key_block(int dqk, int dv) { return (dqk > 128 || dv > 128) ? 64 : 128; }
+// plus O fit TMEM and the slots fit shared memory; 64 for head dims > 128;
+// 32 for head dims above 256 (a 128 KB Q tile leaves three 32 KB slots).
+constexpr int tc_key_block(int dqk, int dv) {
+  return (dqk > 256 || dv > 256) ? 32 : (dqk > 128 || dv > 128) ? 64 : 128;
+}
+
+// Output columns per CTA of the tcgen05 kernel for head dims above 256: O of
+// 128 rows at Dv = 512 would take all of TMEM, so each CTA owns one half of V
+// and O (grid.y = 2) and computes the full scores.
+constexpr int kTcWideHalf = 256;
 
 // Rows of one tcgen05 tile.
 constexpr int kTcRows = 128;
@@ -100,6 +108,7 @@ struct Plan {
   int splits;
   long long ctas;
   int launches;
+  int col_halves;      // tcgen05 kernel at head dims above 256: 2 (grid.y), else 1
   size_t ws_o_bytes, ws_lse_bytes, ws_bytes;
 };
 

@@ -71,7 +71,9 @@ sdpa_status run_tc(const Launch &ln, std::string *err) {
   p.wd.word = ln.wd_word;
   p.wd.limit_ns = ln.wd_limit_ns;
   if (ln.ev_start) record_event(ln.ev_start, ln.stream);
-  kern<<<(unsigned)pl.ctas, Cfg::kThreads, Cfg::kSmemBytes, ln.stream>>>(tq, tk, tv, to, tp, p);
+  // head dims above 256: one CTA per half of V and O (grid.y)
+  const dim3 grid((unsigned)(pl.ctas / pl.col_halves), (unsigned)pl.col_halves);
+  kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, ln.stream>>>(tq, tk, tv, to, tp, p);
   if (ln.ev_stop) record_event(ln.ev_stop, ln.stream);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -90,6 +92,7 @@ sdpa_status run_dtype(const Launch &ln, std::string *err) {
     case 3: return run_tc<kBF16, 192, 128>(ln, err);
     case 4: return run_tc<kBF16, 192, 192>(ln, err);
     case 5: return run_tc<kBF16, 256, 256>(ln, err);
+    case 6: return run_tc<kBF16, 512, kTcWideHalf>(ln, err);
   }
   *err = "internal: no tcgen05 instance for this head-dim pair";
   return SDPA_ERR_UNSUPPORTED;

@@ -88,14 +88,17 @@ struct TcCfg {
   static constexpr int kOCol = kBufs * BN;
   static constexpr int kPrefetch = SDPA_TC_PREFETCH;
   static_assert(DQK % 16 == 0 && DV % 16 == 0 && DV >= 16 && DV <= 256, "head dims");
-  static_assert(BN == 64 || BN == 128, "key block");
+  static_assert(BN == 32 || BN == 64 || BN == 128, "key block");
   static_assert(kCols == 16 || kCols % 32 == 0, "TMEM load / store widths");
   static_assert(kBufs * BN + DV <= 512, "TMEM columns");
   static_assert(kSmemBytes <= 232448, "shared memory");
   // the epilogue stages the tile's output rows in the K/V slots: 64 columns of
   // a 16-bit type, or 32 fp32 split partials, per 16 KB box
   static constexpr int kF32Boxes = (DV + 31) / 32;
-  static_assert(kF32Boxes * kBM * 128 <= NSLOT * kSlotBytes, "output staging");
+  // ... in the K/V slots, or in the Q tile's memory where the slots are too
+  // small (head dims 512: Q is done with once the last S has completed)
+  static constexpr bool kStageInQ = kF32Boxes * kBM * 128 > NSLOT * kSlotBytes;
+  static_assert(!kStageInQ || kF32Boxes * kBM * 128 <= kQBytes, "output staging");
 };
 
 template <bool kBF16, int DQK, int DV, int BN, int NSLOT>
@@ -131,6 +134,10 @@ __global__ void __launch_bounds__(TcCfg<DQK, DV, BN, NSLOT>::kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // Output columns of this CTA: all of them, or (head dims above 256, one CTA
+  // per 256-column half of V and O, blockIdx.y) the half starting at dv0;
+  // each half computes the full scores.
+  const int dv0 = (int)blockIdx.y * DV;
 
   // --- work item: (batch*KV head) fastest, then split, then row tile with
   // the tiles that see the most keys first ---
@@ -214,7 +221,7 @@ __global__ void __launch_bounds__(TcCfg<DQK, DV, BN, NSLOT>::kThreads, 1)
           mbar_arrive_expect_tx(&slot_full[slot], Cfg::kVBytes);
 #pragma unroll
           for (int bx = 0; bx < Cfg::kVBoxes; ++bx)
-            tma_load_3d(dst + bx * (BN * 128), &tm_v, &slot_full[slot], bx * 64, k0, bh);
+            tma_load_3d(dst + bx * (BN * 128), &tm_v, &slot_full[slot], dv0 + bx * 64, k0, bh);
         }
         ++u;
       };
@@ -478,7 +485,7 @@ __global__ void __launch_bounds__(TcCfg<DQK, DV, BN, NSLOT>::kThreads, 1)
     // and columns past Dv are clipped by the tensor map.
     const long total_rows = (long)p.B * p.Hq * p.L;
     const bool split_out = p.splits > 1;
-    uint8_t *stage = sSlots;
+    uint8_t *stage = Cfg::kStageInQ ? sQ : sSlots;
     auto load_o = [&](int c16, float (&o)[16]) {
       if (have_o) {
         tmem_ld16(tmem + lane_base + Cfg::kOCol + c16 * 16, o);
@@ -490,7 +497,8 @@ __global__ void __launch_bounds__(TcCfg<DQK, DV, BN, NSLOT>::kThreads, 1)
     };
     if (!split_out) {
       const float inv = finish_row(p, grow, m_used, l);  // folds in the sink, if any
-      if (p.lse_out != nullptr && valid && part == 0) p.lse_out[grow] = row_lse(m_used, l);
+      if (p.lse_out != nullptr && valid && part == 0 && dv0 == 0)
+        p.lse_out[grow] = row_lse(m_used, l);
 #pragma unroll 1
       for (int c16 = oc_begin; c16 < oc_end; ++c16) {
         float o[16];
@@ -502,7 +510,7 @@ __global__ void __launch_bounds__(TcCfg<DQK, DV, BN, NSLOT>::kThreads, 1)
       }
     } else {
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      if (valid && part == 0)
+      if (valid && part == 0 && dv0 == 0)
         p.part_lse[(long)split * total_rows + grow] = have_o ? row_lse(m_used, l) : -INFINITY;
 #pragma unroll 1
       for (int c16 = oc_begin; c16 < oc_end; ++c16) {
@@ -518,11 +526,11 @@ __global__ void __launch_bounds__(TcCfg<DQK, DV, BN, NSLOT>::kThreads, 1)
     asm volatile("bar.sync 1, %0;" ::"n"(Cfg::kSoftmaxWarps * 32) : "memory");  // softmax warps
     if (warp == 0 && lane == 0 && tr.nvalid > 0) {
       if (!split_out) {
-        for (int bx = 0; bx < Cfg::kVBoxes && bx * 64 < p.Dv; ++bx)
-          tma_store_3d(&tm_o, stage + bx * (Cfg::kBM * 128), bx * 64, tr.row0, bh);
+        for (int bx = 0; bx < Cfg::kVBoxes && dv0 + bx * 64 < p.Dv; ++bx)
+          tma_store_3d(&tm_o, stage + bx * (Cfg::kBM * 128), dv0 + bx * 64, tr.row0, bh);
       } else {
-        for (int bx = 0; bx < Cfg::kF32Boxes && bx * 32 < p.Dv; ++bx)
-          tma_store_3d(&tm_p, stage + bx * (Cfg::kBM * 128), bx * 32, tr.row0,
+        for (int bx = 0; bx < Cfg::kF32Boxes && dv0 + bx * 32 < p.Dv; ++bx)
+          tma_store_3d(&tm_p, stage + bx * (Cfg::kBM * 128), dv0 + bx * 32, tr.row0,
                        split * BH + bh);
       }
       bulk_commit_group();

@@ -169,22 +169,32 @@ def test_forward_without_device_fails_loudly(lib):
     assert b"CUDA" in lib.sdpa_last_error_message() or b"device" in lib.sdpa_last_error_message()
 
 
-def test_plan_head_dims_above_256_take_the_wide_path():
-    # decode at head dim 512: one 16-row group, keys split over the SMs
+def test_plan_head_dims_above_256():
+    # decode at head dim 512: one 16-row group on the wide path, keys split
     info = sdpa.plan(1, 16, 1, 1, 8192, 512, 512, causal=True, num_sms=148)
     assert info["path"] == sdpa.PATH_WIDE and (info["dqk_pad"], info["dv_pad"]) == (512, 512)
     assert info["row_tile"] == 16 and info["key_block"] == 32 and info["splits"] > 1
-    # prefill: two 16-row groups per CTA
-    info = sdpa.plan(1, 8, 8, 1024, 1024, 512, 512, causal=True, num_sms=148)
-    assert info["path"] == sdpa.PATH_WIDE and info["row_tile"] == 32
+    # short verify windows (fewer than 65 packed rows) stay on the wide path
+    assert sdpa.plan(1, 8, 2, 12, 4096, 512, 512, num_sms=148)["path"] == sdpa.PATH_WIDE
+    # prefill: the tcgen05 kernel in two column halves (two CTAs per row tile)
+    info = sdpa.plan(1, 8, 8, 4096, 4096, 512, 512, causal=True, num_sms=148)
+    assert info["path"] == sdpa.PATH_TC and info["row_tile"] == 128 and info["key_block"] == 32
+    assert info["ctas"] == 8 * 32 * 2 and info["splits"] == 1
+    # few row tiles: keys split, each split at least 256 keys
+    info = sdpa.plan(1, 8, 2, 64, 8192, 512, 512, num_sms=148)
+    assert info["path"] == sdpa.PATH_TC and info["splits"] > 1
+    assert info["keys_per_split"] >= 256 and info["ctas"] == 2 * 2 * 2 * info["splits"]
     # mixed dims above 256 run on the 512/512 instance
     assert sdpa.plan(1, 4, 4, 64, 64, 320, 128, num_sms=148)["path"] == sdpa.PATH_WIDE
-    assert sdpa.plan(1, 4, 4, 64, 64, 128, 384, num_sms=148)["path"] == sdpa.PATH_WIDE
-    # no other path takes them, and the wide path takes nothing else
-    for path in (sdpa.PATH_SPLITKV, sdpa.PATH_TC, sdpa.PATH_TC2):
+    assert sdpa.plan(1, 4, 4, 128, 128, 128, 384, num_sms=148)["path"] == sdpa.PATH_TC
+    # the split-KV and pair kernels do not take them, and the wide path
+    # takes nothing else
+    for path in (sdpa.PATH_SPLITKV, sdpa.PATH_TC2, sdpa.PATH_TC_DUAL):
         with pytest.raises(sdpa.SdpaError) as ei:
             sdpa.plan(1, 4, 4, 64, 64, 512, 512, num_sms=148, force_path=path)
         assert ei.value.status == 2 and "wide" in ei.value.message
+    assert sdpa.plan(1, 4, 4, 64, 64, 512, 512, num_sms=148,
+                     force_path=sdpa.PATH_TC)["path"] == sdpa.PATH_TC
     with pytest.raises(sdpa.SdpaError) as ei:
         sdpa.plan(1, 4, 4, 64, 64, 256, 256, num_sms=148, force_path=sdpa.PATH_WIDE)
     assert ei.value.status == 2

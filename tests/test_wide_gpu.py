@@ -1,5 +1,7 @@
-"""GPU parity of the wide path (head dims above 256, up to 512; the output
-columns are split over four warps per 16-row group) against the oracle."""
+"""GPU parity at head dims above 256 (up to 512) against the oracle: the wide
+path (the output columns split over four warps per 16-row group) and the
+tcgen05 path in column halves (one CTA per 256-column half of V and O, each
+computing the full scores)."""
 import numpy as np
 import pytest
 import torch
@@ -34,8 +36,33 @@ CASES = [
 def test_wide_vs_oracle(cuda_lib, case):
     name, B, Hq, Hkv, L, Sk, Dqk, Dv, dt, causal, W = case
     p = I.Problem(B, Hq, Hkv, L, Sk, Dqk, Dv, dt, causal, W, None, 51, name)
-    _, _, info = check_problem(cuda_lib, p)
+    _, _, info = check_problem(cuda_lib, p, force_path=S.PATH_WIDE)
     assert info["path"] == S.PATH_WIDE
+
+
+@pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
+def test_tc_column_halves_vs_oracle(cuda_lib, case):
+    name, B, Hq, Hkv, L, Sk, Dqk, Dv, dt, causal, W = case
+    p = I.Problem(B, Hq, Hkv, L, Sk, Dqk, Dv, dt, causal, W, None, 55, name)
+    _, _, info = check_problem(cuda_lib, p, force_path=S.PATH_TC)
+    assert info["path"] == S.PATH_TC and info["key_block"] == 32
+
+
+@pytest.mark.parametrize("splits", [1, 3, 0])
+def test_tc_column_halves_key_splits(cuda_lib, splits):
+    p = I.Problem(1, 8, 2, 40, 6000, 512, 512, "bf16", True, 0, None, 56, "halves_split")
+    _, _, info = check_problem(cuda_lib, p, force_path=S.PATH_TC, force_splits=splits)
+    assert info["path"] == S.PATH_TC
+    if splits:
+        assert info["splits"] == splits
+
+
+def test_tc_column_halves_agree_with_wide(cuda_lib):
+    p = I.Problem(1, 4, 2, 200, 700, 512, 512, "bf16", True, 0, None, 57, "halves_agree")
+    q, k, v = I.make_qkv(p)
+    a = run_gpu(cuda_lib, p, q, k, v, force_path=S.PATH_TC)[0].float()
+    b = run_gpu(cuda_lib, p, q, k, v, force_path=S.PATH_WIDE)[0].float()
+    assert agree(a, b, "bf16")
 
 
 @pytest.mark.parametrize("splits", [1, 3, 7, 0])
@@ -55,7 +82,8 @@ def test_wide_splits_agree(cuda_lib):
     assert agree(a, b, "bf16")
 
 
-def test_wide_sinks_offset_lse(cuda_lib):
+@pytest.mark.parametrize("path", [S.PATH_WIDE, S.PATH_TC])
+def test_wide_sinks_offset_lse(cuda_lib, path):
     p = I.Problem(1, 4, 2, 40, 700, 512, 512, "bf16", True, 150, None, 54, "wide_ex")
     q, k, v = I.make_qkv(p)
     sinks = [0.25, -2.0, 1.5, 0.0]
@@ -64,7 +92,7 @@ def test_wide_sinks_offset_lse(cuda_lib):
         out = cuda_lib.forward_ex(q.cuda(), k.cuda(), v.cuda(), scale=p.sm_scale, causal=True,
                                   window_size=150, q_offset=500,
                                   sinks=torch.tensor(sinks, device="cuda"), lse=lse,
-                                  force_splits=fs)
+                                  force_path=path, force_splits=fs)
         cuda_lib.device_status()
         ref, ref_lse = sdpa_oracle(q, k, v, p.sm_scale, True, 150, q_offset=500, sinks=sinks,
                                    return_lse=True)
@@ -80,4 +108,5 @@ def test_wide_bench_workloads(cuda_lib, idx):
     p = I.wide_problems()[idx]
     rows = I.sample_rows(p.L, 256, seed=p.seed) if p.L > 256 else None
     _, _, info = check_problem(cuda_lib, p, rows=rows)
-    assert info["path"] == S.PATH_WIDE
+    # decode on the wide path; the prefill's rows fill 128-row tcgen05 tiles
+    assert info["path"] == (S.PATH_TC if p.L > 64 else S.PATH_WIDE)
