@@ -413,17 +413,23 @@ def secondary(sdpa, probs, steps, warmup, flush, sync_all, device, peaks, kind, 
     """Time a list of problems (one call each per step); return a summary.
     With ``stream``, each problem is also timed back to back (``us_stream``)."""
     cases = [Case(sdpa, p, device) for p in probs]
+    # Each timing pass goes over the list in order, heaviest call last, with a
+    # pause after it: seconds of full tensor load lower the clock under the
+    # power cap for a while, which would slow the next pass's first calls.
+    alone = [time_alone(sdpa, c, flush, reps=max(steps, 20)) for c in cases] if graphs else None
+    time.sleep(1.0)
     call_ms, main_ms, _ = time_cases(sdpa, cases, steps, warmup, flush, sync_all, graphs)
+    time.sleep(1.0)
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     pts = []
-    for c, cm, mm in zip(cases, call_ms, main_ms):
+    for i, (c, cm, mm) in enumerate(zip(cases, call_ms, main_ms)):
         # the call timed alone: a graph holding only the call, replayed after
         # an L2 flush, events on the stream around the replay.  us_events is
         # the same call bracketed by events the library records inside the
         # graph, which carry several microseconds of their own (mean over the
         # timed steps: the device timer's coarse steps make a median jump
         # between neighbouring values)
-        us = time_alone(sdpa, c, flush, reps=max(steps, 20)) if graphs else 1e3 * statistics.mean(cm)
+        us = alone[i] if graphs else 1e3 * statistics.mean(cm)
         d = {"name": c.p.name, "us": round(us, 2),
              "us_events": round(1e3 * statistics.mean(cm), 2),
              "us_events_median": round(1e3 * statistics.median(cm), 2),
