@@ -564,6 +564,14 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t start, uint32_t lbo
   return d;
 }
 
+// A descriptor moved by `bytes` (a multiple of 16) in shared memory: only the
+// start-address field changes, and it cannot carry out of its 14 bits while
+// the address stays below 256 KB, which every shared-memory address does.
+// One add per MMA instead of rebuilding the descriptor from the address.
+__device__ __forceinline__ uint64_t umma_desc_advance(uint64_t desc, uint32_t bytes) {
+  return desc + (uint64_t)(bytes >> 4);
+}
+
 // Same for an MN-major operand: lbo = byte stride between 64-element blocks
 // along M/N, sbo = byte stride between 8-row groups along K.
 __device__ __forceinline__ uint64_t umma_desc_sw128_mn(uint32_t start, uint32_t lbo,

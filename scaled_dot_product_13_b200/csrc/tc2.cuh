@@ -244,13 +244,12 @@ __global__ void __launch_bounds__(224, 1)
         if (!take_slot(slot)) return false;
         const int b = n & 1;
         tc_fence_after();
-        const uint32_t kb = slot_addr + slot * Cfg::kSlotBytes;
+        const uint64_t a0 = umma_desc_sw128(q_addr, 16, 1024);
+        const uint64_t b0 = umma_desc_sw128(slot_addr + slot * Cfg::kSlotBytes, 16, 1024);
 #pragma unroll
         for (int ks = 0; ks < Cfg::kKS; ++ks) {
-          const uint64_t a =
-              umma_desc_sw128(q_addr + (ks >> 2) * (Cfg::kBM * 128) + (ks & 3) * 32, 16, 1024);
-          const uint64_t bd =
-              umma_desc_sw128(kb + (ks >> 2) * ((BN / 2) * 128) + (ks & 3) * 32, 16, 1024);
+          const uint64_t a = umma_desc_advance(a0, (ks >> 2) * (Cfg::kBM * 128) + (ks & 3) * 32);
+          const uint64_t bd = umma_desc_advance(b0, (ks >> 2) * ((BN / 2) * 128) + (ks & 3) * 32);
           tc_mma_ss_pair(tmem + b * BN, a, bd, kIdescS, ks > 0 ? 1u : 0u);
         }
         both(&s_full[b]);
@@ -263,10 +262,10 @@ __global__ void __launch_bounds__(224, 1)
         const int b = j & 1;
         if (!mbar_wait_cluster(&p_full[b], (uint32_t)(j >> 1) & 1u, p.wd, kWdSoftmax)) return false;
         tc_fence_after();
-        const uint32_t vb = slot_addr + slot * Cfg::kSlotBytes;
+        const uint64_t v0 = umma_desc_sw128_mn(slot_addr + slot * Cfg::kSlotBytes, BN * 128, 1024);
 #pragma unroll
         for (int ks = 0; ks < Cfg::kPVK; ++ks) {
-          const uint64_t bd = umma_desc_sw128_mn(vb + ks * 2048, BN * 128, 1024);
+          const uint64_t bd = umma_desc_advance(v0, ks * 2048);
           tc_mma_ts_pair(tmem + Cfg::kOCol, tmem + b * BN + ks * 8, bd, kIdescPV,
                          (j > 0 || ks > 0) ? 1u : 0u);
         }

@@ -267,21 +267,22 @@ __global__ void __launch_bounds__(320, 1)
       };
       auto issue_s = [&](int t, int j) {
         const uint32_t kb = slot_addr + slot_of(2 * j) * Cfg::kSlotBytes;
-        const uint32_t qa = q_addr + t * Cfg::kQTileBytes;
+        const uint64_t a0 = umma_desc_sw128(q_addr + t * Cfg::kQTileBytes, 16, 1024);
+        const uint64_t b0 = umma_desc_sw128(kb, 16, 1024);
 #pragma unroll
         for (int ks = 0; ks < Cfg::kKS; ++ks) {
-          const uint64_t a =
-              umma_desc_sw128(qa + (ks >> 2) * (Cfg::kBM * 128) + (ks & 3) * 32, 16, 1024);
-          const uint64_t bd = umma_desc_sw128(kb + (ks >> 2) * (BN * 128) + (ks & 3) * 32, 16, 1024);
+          const uint64_t a = umma_desc_advance(a0, (ks >> 2) * (Cfg::kBM * 128) + (ks & 3) * 32);
+          const uint64_t bd = umma_desc_advance(b0, (ks >> 2) * (BN * 128) + (ks & 3) * 32);
           tc_mma_ss(tmem + t * Cfg::kTileCols, a, bd, kIdescS, ks > 0 ? 1u : 0u);
         }
         tc_commit(&s_full[t]);
       };
       auto issue_pv = [&](int t, int j) {
         const uint32_t vb = slot_addr + slot_of(2 * j + 1) * Cfg::kSlotBytes;
+        const uint64_t v0 = umma_desc_sw128_mn(vb, BN * 128, 1024);
 #pragma unroll
         for (int ks = 0; ks < Cfg::kPVK; ++ks) {
-          const uint64_t bd = umma_desc_sw128_mn(vb + ks * 2048, BN * 128, 1024);
+          const uint64_t bd = umma_desc_advance(v0, ks * 2048);
           tc_mma_ts(tmem + t * Cfg::kTileCols + BN, tmem + t * Cfg::kTileCols + ks * 8, bd,
                     kIdescPV, (j > 0 || ks > 0) ? 1u : 0u);
         }
@@ -304,23 +305,22 @@ __global__ void __launch_bounds__(320, 1)
           return w;
         };
         auto s_into = [&](int t, int slot) {
-          const uint32_t kb = slot_addr + slot * Cfg::kSlotBytes;
+          const uint64_t a0 = umma_desc_sw128(q_addr, 16, 1024);
+          const uint64_t b0 = umma_desc_sw128(slot_addr + slot * Cfg::kSlotBytes, 16, 1024);
 #pragma unroll
           for (int ks = 0; ks < Cfg::kKS; ++ks) {
-            const uint64_t a =
-                umma_desc_sw128(q_addr + (ks >> 2) * (Cfg::kBM * 128) + (ks & 3) * 32, 16, 1024);
-            const uint64_t bd =
-                umma_desc_sw128(kb + (ks >> 2) * (BN * 128) + (ks & 3) * 32, 16, 1024);
+            const uint64_t a = umma_desc_advance(a0, (ks >> 2) * (Cfg::kBM * 128) + (ks & 3) * 32);
+            const uint64_t bd = umma_desc_advance(b0, (ks >> 2) * (BN * 128) + (ks & 3) * 32);
             tc_mma_ss(tmem + t * Cfg::kTileCols, a, bd, kIdescS, ks > 0 ? 1u : 0u);
           }
           tc_commit(&s_full[t]);
           tc_commit(&slot_empty[slot]);
         };
         auto pv_from = [&](int t, int slot, bool first) {
-          const uint32_t vb = slot_addr + slot * Cfg::kSlotBytes;
+          const uint64_t v0 = umma_desc_sw128_mn(slot_addr + slot * Cfg::kSlotBytes, BN * 128, 1024);
 #pragma unroll
           for (int ks = 0; ks < Cfg::kPVK; ++ks) {
-            const uint64_t bd = umma_desc_sw128_mn(vb + ks * 2048, BN * 128, 1024);
+            const uint64_t bd = umma_desc_advance(v0, ks * 2048);
             tc_mma_ts(tmem + t * Cfg::kTileCols + BN, tmem + t * Cfg::kTileCols + ks * 8, bd,
                       kIdescPV, (!first || ks > 0) ? 1u : 0u);
           }
