@@ -107,9 +107,14 @@ typedef enum {
   SDPA_PATH_TC_DUAL = 5, /* head dims up to 128: two 128-row tiles per CTA
                             share each K/V block, their softmax phases
                             interleaved with each other's MMAs (tcgen05)     */
-  SDPA_PATH_TC_KSPLIT = 6 /* head dims up to 128: one 128-row tile per CTA
+  SDPA_PATH_TC_KSPLIT = 6, /* head dims up to 128: one 128-row tile per CTA
                             whose two softmax groups take alternate key
                             blocks, merged in the epilogue (tcgen05)        */
+  SDPA_PATH_TC2_LOOP = 7  /* the SDPA_PATH_TC2 kernel with at most one CTA
+                            pair per two SMs, each walking several 256-row
+                            tiles: the next tile's Q and first scores run
+                            under the current tile's end.  Never splits the
+                            keys; routed for windows and short key ranges  */
 } sdpa_path;
 
 /*
@@ -244,7 +249,9 @@ typedef struct {
   int row_tiles;     /* row tiles per (batch, KV head)                      */
   int key_block;     /* keys per pipeline stage                             */
   int keys_per_split;/* keys one split covers (a multiple of key_block)     */
-  int ctas;          /* CTAs (CTA pairs on SDPA_PATH_TC2) of the main launch */
+  int ctas;          /* CTAs of the main launch (CTA pairs on SDPA_PATH_TC2;
+                        256-row tiles on SDPA_PATH_TC2_LOOP, whose pairs
+                        walk them)                                          */
   int launches;      /* kernel launches one call makes (1 or 2)             */
   int dqk_pad;       /* head dims the kernel instance is built for          */
   int dv_pad;

@@ -21,13 +21,13 @@ import os
 __all__ = ["forward", "forward_ws", "forward_noalloc", "forward_ex", "Options", "workspace_bytes", "plan", "device_status",
            "set_wait_limit_ns", "watchdog_selftest", "exp2_selftest", "time_next_main_kernel", "time_next_call", "load_library", "library_path",
            "SdpaError", "PATH_AUTO", "PATH_SPLITKV", "PATH_TC", "PATH_TC2", "PATH_WIDE", "PATH_TC_DUAL", "PATH_TC_KSPLIT",
-           "STATUS"]
+           "PATH_TC2_LOOP", "STATUS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB: ctypes.CDLL | None = None
 
-PATH_AUTO, PATH_SPLITKV, PATH_TC, PATH_TC2, PATH_WIDE, PATH_TC_DUAL, PATH_TC_KSPLIT = \
-    0, 1, 2, 3, 4, 5, 6
+PATH_AUTO, PATH_SPLITKV, PATH_TC, PATH_TC2, PATH_WIDE, PATH_TC_DUAL, PATH_TC_KSPLIT, PATH_TC2_LOOP = \
+    0, 1, 2, 3, 4, 5, 6, 7
 STATUS = {0: "SDPA_OK", 1: "SDPA_ERR_INVALID_ARG", 2: "SDPA_ERR_UNSUPPORTED",
           3: "SDPA_ERR_RESOURCES", 4: "SDPA_ERR_CUDA", 5: "SDPA_ERR_TIMEOUT"}
 

@@ -182,6 +182,11 @@ constexpr int kMinBlocksPerSplit = 2;
 constexpr int kMinBlocksPerSplitWide = 8;
 constexpr int kNoSplitBlocks = 4;
 
+// The pair kernel loops over its tiles (SDPA_PATH_TC2_LOOP) when a tile visits
+// at most this many key blocks: there a tile's fill and epilogue are a large
+// share of its time and the loop hides them under the neighbouring tiles.
+constexpr int kLoopMaxTileBlocks = 48;
+
 sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_splits,
                       Plan *out) {
   Plan pl;
@@ -192,7 +197,8 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
     return fail(SDPA_ERR_UNSUPPORTED, "no kernel instance covers Dqk=%d, Dv=%d", pb.Dqk, pb.Dv);
   if (force_path != SDPA_PATH_AUTO && force_path != SDPA_PATH_SPLITKV &&
       force_path != SDPA_PATH_TC && force_path != SDPA_PATH_TC2 && force_path != SDPA_PATH_WIDE &&
-      force_path != SDPA_PATH_TC_DUAL && force_path != SDPA_PATH_TC_KSPLIT)
+      force_path != SDPA_PATH_TC_DUAL && force_path != SDPA_PATH_TC_KSPLIT &&
+      force_path != SDPA_PATH_TC2_LOOP)
     return fail(SDPA_ERR_INVALID_ARG, "unknown path %d", force_path);
   // head dims above 256 run on the column-split warp-tile kernel (decode and
   // short verify windows) or on the tcgen05 kernel in column halves; the
@@ -235,7 +241,8 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
         (long long)pb.B * pb.Hkv * ((pl.rows + 255) / 256) * 2 >= num_sms)
       path = SDPA_PATH_TC_DUAL;
   }
-  if (path == SDPA_PATH_TC2 && !tc2_supports_pair(pl.pair)) {
+  const bool pair_path = path == SDPA_PATH_TC2 || path == SDPA_PATH_TC2_LOOP;
+  if (pair_path && !tc2_supports_pair(pl.pair)) {
     // the smallest two-CTA instance that covers the head dims (zero filled)
     for (int i = pl.pair + 1; i < kNumDimPairs; ++i)
       if (tc2_supports_pair(i) && kDimPairs[i].dqk >= pb.Dqk && kDimPairs[i].dv >= pb.Dv) {
@@ -243,7 +250,7 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
         break;
       }
   }
-  if (path == SDPA_PATH_TC2 && !tc2_supports_pair(pl.pair))
+  if (pair_path && !tc2_supports_pair(pl.pair))
     return fail(SDPA_ERR_UNSUPPORTED,
                 "the two-CTA path is built for head dims 256/256, 192/128 and 128/128 (got %d/%d)",
                 pb.Dqk, pb.Dv);
@@ -266,7 +273,7 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
     pl.wk = 0;
     pl.row_tile = 16 * pl.wr;
     pl.key_block = kWideBN;
-  } else if (path == SDPA_PATH_TC2) {
+  } else if (pair_path) {
     pl.wr = 0; pl.wk = 0;
     pl.row_tile = 2 * kTcRows;
     pl.key_block = 128;
@@ -299,7 +306,7 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
   const int nkb = std::max(1, (kend + bn - 1) / bn - kbeg / bn);
   // CTAs per split: one per row tile, two per pair tile, two per row tile
   // (one per column half) for the tcgen05 kernel at head dims above 256
-  const long long per_tile = pl.path == SDPA_PATH_TC2 ? 2 : 1;
+  const long long per_tile = pair_path ? 2 : 1;
   const bool tc_wide = path == SDPA_PATH_TC && wide;
   const long long base = (long long)pb.B * pb.Hkv * pl.row_tiles * per_tile * pl.col_halves;
   // resident CTAs per SM (the split-KV kernel runs two where they fit)
@@ -309,7 +316,12 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
                                                       kDimPairs[pl.pair].dv, pl.wr)
                                 : 1);
   int splits;
-  if (force_splits > 0) {
+  if (path == SDPA_PATH_TC2_LOOP) {
+    // the looping form writes finished rows only
+    if (force_splits > 1)
+      return fail(SDPA_ERR_UNSUPPORTED, "the looping pair path does not split the keys");
+    splits = 1;
+  } else if (force_splits > 0) {
     splits = std::min(force_splits, nkb);
   } else if (base >= slots || (path == SDPA_PATH_SPLITKV ? nkb * bn <= kNoSplitBlocks * 64
                                 : tc_wide              ? nkb * bn <= kNoSplitBlocks * 128
@@ -331,6 +343,18 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
   pl.splits = splits;
   pl.keys_per_split = bps * bn;
   pl.ctas = (base / per_tile) * splits;  // all CTAs: grid.x * col_halves
+  // Windowed or short unsplit tiles on the pair kernel, more of them than SM
+  // pairs: loop over tiles.  A tile visits at most the window's blocks plus
+  // its own 256 rows' worth (or all of them without a window).
+  if (force_path == SDPA_PATH_AUTO && path == SDPA_PATH_TC2 && splits == 1 &&
+      pl.ctas > num_sms / 2) {
+    const int tile_blocks =
+        pb.window > 0 ? std::min(nkb, (pb.window + pl.row_tile + bn - 1) / bn + 1) : nkb;
+    if (tile_blocks <= kLoopMaxTileBlocks && (pb.window > 0 || !pb.causal))
+      path = pl.path = SDPA_PATH_TC2_LOOP;
+  }
+  if (path == SDPA_PATH_TC2_LOOP)
+    pl.loop_pairs = (int)std::min<long long>(pl.ctas, std::max(1, num_sms / 2));
   if (pl.ctas > 0x7fffffffLL)
     return fail(SDPA_ERR_UNSUPPORTED, "problem needs %lld CTAs, above the grid limit", pl.ctas);
   pl.launches = splits > 1 ? 2 : 1;
@@ -497,7 +521,7 @@ sdpa_status forward_call(const Problem &pb, const void *q, const void *k, const 
   ln.ev_stop = t_ev_stop;
   cudaEvent_t ev_call = t_ev_call;
   t_ev_start = t_ev_stop = t_ev_call = nullptr;
-  st = pl.path == SDPA_PATH_TC2       ? launch_tc2(ln, &err)
+  st = pl.path == SDPA_PATH_TC2 || pl.path == SDPA_PATH_TC2_LOOP ? launch_tc2(ln, &err)
        : pl.path == SDPA_PATH_TC      ? launch_tc(ln, &err)
        : pl.path == SDPA_PATH_TC_DUAL || pl.path == SDPA_PATH_TC_KSPLIT ? launch_tc_pp(ln, &err)
        : pl.path == SDPA_PATH_WIDE    ? launch_wide(ln, &err)

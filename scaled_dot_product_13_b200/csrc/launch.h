@@ -96,7 +96,7 @@ struct Problem {
 };
 
 struct Plan {
-  int path;            // SDPA_PATH_SPLITKV, _TC, _TC2 or _WIDE
+  int path;            // an sdpa_path value other than SDPA_PATH_AUTO
   int pair;            // index into kDimPairs
   int rows;            // g * L
   int wr, wk;          // split-KV warp layout (rows x key slices); wide: row groups
@@ -109,6 +109,7 @@ struct Plan {
   long long ctas;
   int launches;
   int col_halves;      // tcgen05 kernel at head dims above 256: 2 (grid.y), else 1
+  int loop_pairs;      // SDPA_PATH_TC2_LOOP: CTA pairs launched (each walks several tiles)
   size_t ws_o_bytes, ws_lse_bytes, ws_bytes;
 };
 

@@ -6,7 +6,9 @@ namespace sdpa {
 
 namespace {
 
-template <bool kBF16, int DQK, int DV>
+// kLoop: the looping form (two Q buffers, so fewer K/V slots), grid of
+// plan.loop_pairs pairs; otherwise one pair per 256-row tile.
+template <bool kBF16, int DQK, int DV, bool kLoop>
 sdpa_status run_tc2(const Launch &ln, std::string *err) {
   constexpr int kBN = 128;
   constexpr uint32_t kQ = (DQK / 64) * 128 * 128;
@@ -14,11 +16,11 @@ sdpa_status run_tc2(const Launch &ln, std::string *err) {
   constexpr uint32_t kV = (DV / 128) * kBN * 128;
   constexpr uint32_t kSlot = kK > kV ? kK : kV;
   constexpr uint32_t kBudget = 232448u - 48u * 8u - 16u;
-  constexpr int kFit = (int)((kBudget - kQ) / kSlot);
+  constexpr int kFit = (int)((kBudget - (kLoop ? 2u : 1u) * kQ) / kSlot);
   constexpr int kNSlot = kFit > 8 ? 8 : kFit;
-  static_assert(kNSlot >= 2, "at least two K/V slots");
-  using Cfg = Tc2Cfg<DQK, DV, kBN, kNSlot>;
-  auto kern = tc2_attn_kernel<kBF16, DQK, DV, kBN, kNSlot>;
+  static_assert(kNSlot >= 3, "at least three K/V slots");
+  using Cfg = Tc2Cfg<DQK, DV, kBN, kNSlot, kLoop>;
+  auto kern = tc2_attn_kernel<kBF16, DQK, DV, kBN, kNSlot, kLoop>;
   sdpa_status st =
       prepare_kernel((const void *)kern, Cfg::kThreads, Cfg::kSmemBytes, "tc2_attn_kernel", err);
   if (st != SDPA_OK) return st;
@@ -65,7 +67,7 @@ sdpa_status run_tc2(const Launch &ln, std::string *err) {
   p.wd.limit_ns = ln.wd_limit_ns;
 
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(2 * pl.ctas));
+  cfg.gridDim = dim3((unsigned)(2 * (kLoop ? (long long)pl.loop_pairs : pl.ctas)));
   cfg.blockDim = dim3(Cfg::kThreads);
   cfg.dynamicSmemBytes = Cfg::kSmemBytes;
   cfg.stream = ln.stream;
@@ -87,12 +89,12 @@ sdpa_status run_tc2(const Launch &ln, std::string *err) {
   return SDPA_OK;
 }
 
-template <bool kBF16>
+template <bool kBF16, bool kLoop>
 sdpa_status run_dtype(const Launch &ln, std::string *err) {
   switch (ln.plan.pair) {
-    case 2: return run_tc2<kBF16, 128, 128>(ln, err);
-    case 3: return run_tc2<kBF16, 192, 128>(ln, err);
-    case 5: return run_tc2<kBF16, 256, 256>(ln, err);
+    case 2: return run_tc2<kBF16, 128, 128, kLoop>(ln, err);
+    case 3: return run_tc2<kBF16, 192, 128, kLoop>(ln, err);
+    case 5: return run_tc2<kBF16, 256, 256, kLoop>(ln, err);
   }
   *err = "internal: no two-CTA instance for this head-dim pair";
   return SDPA_ERR_UNSUPPORTED;
@@ -101,7 +103,10 @@ sdpa_status run_dtype(const Launch &ln, std::string *err) {
 }  // namespace
 
 sdpa_status launch_tc2(const Launch &ln, std::string *err) {
-  return ln.pb.dtype == SDPA_BF16 ? run_dtype<true>(ln, err) : run_dtype<false>(ln, err);
+  const bool bf16 = ln.pb.dtype == SDPA_BF16;
+  if (ln.plan.path == SDPA_PATH_TC2_LOOP)
+    return bf16 ? run_dtype<true, true>(ln, err) : run_dtype<false, true>(ln, err);
+  return bf16 ? run_dtype<true, false>(ln, err) : run_dtype<false, false>(ln, err);
 }
 
 }  // namespace sdpa

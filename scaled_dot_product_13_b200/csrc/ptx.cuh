@@ -29,6 +29,7 @@ enum : uint32_t {
   kWdDrain = 5,       // teardown wait for in-flight copies expired
   kWdPeer = 6,        // another CTA reported an error; this one unwound
   kWdSmemAlign = 7,   // dynamic shared memory not 1024-byte aligned
+  kWdConfig = 8,      // launch parameters this kernel instance does not take
 };
 
 struct Watchdog {
@@ -364,6 +365,11 @@ __device__ __forceinline__ void bulk_commit_group() {
 }
 __device__ __forceinline__ void bulk_wait_group0() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+// Wait until every committed bulk store has finished reading shared memory
+// (its global writes may still be in flight).
+__device__ __forceinline__ void bulk_wait_group_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
 // Prefetch one box of a tiled tensor into L2 (no shared memory, no barrier).

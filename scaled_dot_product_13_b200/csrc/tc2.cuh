@@ -30,6 +30,18 @@
 // columns of buffer j % 2), O at [2 BN, 2 BN + DV).  A score buffer is reused
 // two blocks later: the MMA for S_{j+2} is issued after P_j V by the same
 // thread, and one thread's tcgen05 MMAs execute in order.
+//
+// Looping form (PERSIST): a grid of at most one pair per two SMs walks the
+// pair tiles (item = pair index, + pairs launched, ...).  Q has two buffers,
+// so the next tile's Q load and its first two score MMAs run under the
+// current tile's last blocks and epilogue, and a pair pays the launch,
+// barrier and TMEM set-up once instead of once per tile.  Block and tile
+// counters run on across tiles, so every barrier's phase follows from them.
+// A tile's output is staged in its own Q buffer (free once the tile's MMAs
+// have completed) and stored from there; the producer refills that buffer
+// for the tile after next only once the store has read it (q_empty).  The
+// next tile's first P V, which overwrites O, waits for P of that tile's
+// first block, which the softmax warps write after they have read O out.
 #pragma once
 
 #include "params.cuh"
@@ -40,11 +52,13 @@
 #define SDPA_TC2_POLY_OF4 1
 #endif
 
+
 namespace sdpa {
 
-template <int DQK, int DV, int BN, int NSLOT>
+template <int DQK, int DV, int BN, int NSLOT, bool PERSIST = false>
 struct Tc2Cfg {
   static constexpr int kBM = 128;              // rows per CTA (256 per pair)
+  static constexpr int kQBufs = PERSIST ? 2 : 1;
   static constexpr int kQBoxes = DQK / 64;
   static constexpr int kVHalf = DV / 2;         // V columns per CTA
   static constexpr int kVBoxes = kVHalf / 64;
@@ -54,7 +68,7 @@ struct Tc2Cfg {
   static constexpr uint32_t kKBytes = kQBoxes * (BN / 2) * 128;  // this CTA's K half
   static constexpr uint32_t kVBytes = kVBoxes * BN * 128;        // this CTA's V half
   static constexpr uint32_t kSlotBytes = kKBytes > kVBytes ? kKBytes : kVBytes;
-  static constexpr uint32_t kSlotOff = kQBytes;
+  static constexpr uint32_t kSlotOff = kQBufs * kQBytes;
   static constexpr uint32_t kBarOff = kSlotOff + NSLOT * kSlotBytes;
   static constexpr int kNumBars = 3 * NSLOT + 16;
   static constexpr uint32_t kSmemBytes = kBarOff + kNumBars * 8 + 16;
@@ -65,36 +79,94 @@ struct Tc2Cfg {
   static_assert(BN == 128, "key block");
   static_assert(2 * BN + DV <= 512, "TMEM columns");
   static_assert(kSmemBytes <= 232448, "shared memory");
-  // the epilogue stages the CTA's 128 output rows in its K/V slots: 64
-  // columns of a 16-bit type, or 32 fp32 split partials, per 16 KB box
+  // the epilogue stages the CTA's 128 output rows, 64 columns of a 16-bit
+  // type or 32 fp32 split partials per 16 KB box: in the K/V slots (one
+  // tile per pair), or in the tile's Q buffer (looping form, 16-bit only)
   static constexpr int kOutBoxes = (DV + 63) / 64;
   static constexpr int kF32Boxes = (DV + 31) / 32;
-  static_assert(kF32Boxes * kBM * 128 <= NSLOT * kSlotBytes, "output staging");
+  static_assert(PERSIST ? kOutBoxes * kBM * 128 <= kQBytes
+                        : kF32Boxes * kBM * 128 <= NSLOT * kSlotBytes,
+                "output staging");
 };
 
-template <bool kBF16, int DQK, int DV, int BN, int NSLOT>
+// One work item of a pair: (batch*KV head) fastest, then split, then the
+// 256-row tile, heaviest first.  Rows are packed head-major (row = head in
+// the group * L + query), so when whole tiles fit a head's L rows, tiles at
+// the same query positions of the group's heads are equally heavy (causal
+// and windowed rows see more keys further down): the order then takes the
+// last positions of every head first.  Both CTAs derive the same key range.
+struct Tc2Tile {
+  int bh, split, k_lo, k_hi, nblk;
+  TileRows tpair;  // the pair's 256 rows
+  TileRows tr;     // this CTA's 128 of them
+};
+
+template <int BN, int kBM>
+__device__ __forceinline__ Tc2Tile tc2_tile(const AttnParams &p, int item, uint32_t rank) {
+  Tc2Tile w;
+  const int BH = p.B * p.Hkv;
+  w.bh = item % BH;
+  item /= BH;
+  w.split = item % p.splits;
+  const int r = item / p.splits;  // rank of the tile, heaviest first
+  const int g = p.R / p.L;
+  int pair_tile;
+  if (g > 1 && p.L % (2 * kBM) == 0) {
+    const int per_head = p.L / (2 * kBM);
+    pair_tile = (r % g) * per_head + (per_head - 1 - r / g);
+  } else {
+    pair_tile = p.row_tiles - 1 - r;
+  }
+  w.tpair = tile_rows(p, pair_tile, 2 * kBM);
+  tile_key_range(p, w.tpair, BN, w.split, w.k_lo, w.k_hi);
+  w.nblk = (w.k_hi - w.k_lo) / BN;
+  w.tr = tile_rows(p, pair_tile * 2 + (int)rank, kBM);
+  if (w.tr.nvalid <= 0) {
+    w.tr.nvalid = 0;
+    w.tr.pos_min = w.tpair.pos_min;
+    w.tr.pos_max = w.tpair.pos_max;
+  }
+  return w;
+}
+
+// The it-th work item of pair `pid` of `npairs`, or -1 when it has no more:
+// round it hands items [it*npairs, (it+1)*npairs) out, every other round in
+// reverse pair order, so that pairs given the heavier items of one round
+// get the lighter ones of the next.
+__device__ __forceinline__ int tc2_item(int it, int pid, int npairs, int n_items) {
+  const long long idx = (long long)it * npairs + ((it & 1) ? npairs - 1 - pid : pid);
+  return idx < n_items ? (int)idx : -1;
+}
+
+template <bool kBF16, int DQK, int DV, int BN, int NSLOT, bool PERSIST>
 __global__ void __launch_bounds__(224, 1)
     tc2_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_o,
                     const __grid_constant__ CUtensorMap tm_p, const AttnParams p) {
-  using Cfg = Tc2Cfg<DQK, DV, BN, NSLOT>;
+  using Cfg = Tc2Cfg<DQK, DV, BN, NSLOT, PERSIST>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // same layout in both CTAs, so both take this exit together
   if ((smem_u32(smem_raw) & 1023u) != 0u) {
     if (threadIdx.x == 0) wd_record(p.wd, kWdSmemAlign);
     return;
   }
+  // the looping form stages 16-bit output rows only (no split partials)
+  if (PERSIST && p.splits != 1) {
+    if (threadIdx.x == 0) wd_record(p.wd, kWdConfig);
+    return;
+  }
   uint8_t *smem = smem_raw;
-  uint8_t *sQ = smem;
+  uint8_t *sQ = smem;  // [kQBufs][kQBytes]
   uint8_t *sSlots = smem + Cfg::kSlotOff;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kBarOff);
   uint64_t *slot_full = bars;                // [NSLOT] this CTA's loads landed
   uint64_t *slot_empty = slot_full + NSLOT;  // [NSLOT] the pair's MMA is done with the slot
   uint64_t *peer_full = slot_empty + NSLOT;  // [NSLOT] even CTA: the odd CTA's loads landed
-  uint64_t *q_full = peer_full + NSLOT;
-  uint64_t *peer_q = q_full + 1;             // even CTA: the odd CTA's Q landed
-  uint64_t *s_full = peer_q + 1;             // [2]
+  uint64_t *q_full = peer_full + NSLOT;      // [2] per Q buffer
+  uint64_t *peer_q = q_full + 2;             // [2] even CTA: the odd CTA's Q landed
+  uint64_t *q_empty = peer_q + 2;            // [2] looping form: the store has read the buffer
+  uint64_t *s_full = q_empty + 2;            // [2]
   uint64_t *p_full = s_full + 2;             // [2] even CTA: P_j of both CTAs written
   uint64_t *o_bar = p_full + 2;
   uint64_t *o_final = o_bar + 1;
@@ -107,24 +179,11 @@ __global__ void __launch_bounds__(224, 1)
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
 
-  // --- work item of the pair: (batch*KV head) fastest, then split, then the
-  // 256-row tile, heaviest first ---
-  int bid = blockIdx.x >> 1;
+  // --- the pair's work items (tc2_item): one per pair unless looping ---
   const int BH = p.B * p.Hkv;
-  const int bh = bid % BH;
-  bid /= BH;
-  const int split = bid % p.splits;
-  const int pair_tile = p.row_tiles - 1 - bid / p.splits;
-  const TileRows tpair = tile_rows(p, pair_tile, 2 * Cfg::kBM);
-  int k_lo, k_hi;
-  tile_key_range(p, tpair, BN, split, k_lo, k_hi);  // identical in both CTAs
-  const int nblk = (k_hi - k_lo) / BN;
-  TileRows tr = tile_rows(p, pair_tile * 2 + (int)rank, Cfg::kBM);  // this CTA's rows
-  if (tr.nvalid <= 0) {
-    tr.nvalid = 0;
-    tr.pos_min = tpair.pos_min;
-    tr.pos_max = tpair.pos_max;
-  }
+  const int n_items = BH * p.splits * p.row_tiles;
+  const int pid = (int)(blockIdx.x >> 1);
+  const int npairs = (int)(gridDim.x >> 1);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NSLOT; ++s) {
@@ -132,9 +191,10 @@ __global__ void __launch_bounds__(224, 1)
       mbar_init(&slot_empty[s], 1);
       mbar_init(&peer_full[s], 1);
     }
-    mbar_init(q_full, 1);
-    mbar_init(peer_q, 1);
     for (int b = 0; b < 2; ++b) {
+      mbar_init(&q_full[b], 1);
+      mbar_init(&peer_q[b], 1);
+      mbar_init(&q_empty[b], 1);
       mbar_init(&s_full[b], 1);
       mbar_init(&p_full[b], 8);
     }
@@ -161,13 +221,27 @@ __global__ void __launch_bounds__(224, 1)
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      const int grow0 = bh * p.R + tpair.row0 + (int)rank * Cfg::kBM;
-      mbar_arrive_expect_tx(q_full, Cfg::kQBytes);
+      int u = 0, it = 0;
+      bool ok = true;
+      for (; ok; ++it) {
+        const int item = tc2_item(it, pid, npairs, n_items);
+        if (item < 0) break;
+      const Tc2Tile w = tc2_tile<BN, Cfg::kBM>(p, item, rank);
+      const int qb = it % Cfg::kQBufs, use = it / Cfg::kQBufs;
+      // a Q buffer is refilled once the store of the output staged in it
+      // (two tiles back) has read it
+      if (PERSIST && use > 0 &&
+          !mbar_wait(&q_empty[qb], (uint32_t)(use - 1) & 1u, p.wd, kWdTmaEmpty)) {
+        ok = false;
+        break;
+      }
+      const int grow0 = w.bh * p.R + w.tpair.row0 + (int)rank * Cfg::kBM;
+      uint8_t *q_dst = sQ + qb * Cfg::kQBytes;
+
+      mbar_arrive_expect_tx(&q_full[qb], Cfg::kQBytes);
 #pragma unroll
       for (int bx = 0; bx < Cfg::kQBoxes; ++bx)
-        tma_load_2d(sQ + bx * (Cfg::kBM * 128), &tm_q, q_full, bx * 64, grow0);
-      int u = 0;
-      bool ok = true;
+        tma_load_2d(q_dst + bx * (Cfg::kBM * 128), &tm_q, &q_full[qb], bx * 64, grow0);
       auto emit = [&](bool is_k, int blk) {
         const int slot = u % NSLOT;
         if (!mbar_wait_cluster(&slot_empty[slot], ((uint32_t)(u / NSLOT) & 1u) ^ 1u, p.wd,
@@ -176,43 +250,60 @@ __global__ void __launch_bounds__(224, 1)
           return;
         }
         uint8_t *dst = sSlots + slot * Cfg::kSlotBytes;
-        const int k0 = k_lo + blk * BN;
+        const int k0 = w.k_lo + blk * BN;
         if (is_k) {
           mbar_arrive_expect_tx(&slot_full[slot], Cfg::kKBytes);
 #pragma unroll
           for (int bx = 0; bx < Cfg::kQBoxes; ++bx)
             tma_load_3d(dst + bx * ((BN / 2) * 128), &tm_k, &slot_full[slot], bx * 64,
-                        k0 + (int)rank * (BN / 2), bh);
+                        k0 + (int)rank * (BN / 2), w.bh);
         } else {
           mbar_arrive_expect_tx(&slot_full[slot], Cfg::kVBytes);
 #pragma unroll
           for (int bx = 0; bx < Cfg::kVBoxes; ++bx)
             tma_load_3d(dst + bx * (BN * 128), &tm_v, &slot_full[slot],
-                        (int)rank * Cfg::kVHalf + bx * 64, k0, bh);
+                        (int)rank * Cfg::kVHalf + bx * 64, k0, w.bh);
         }
         ++u;
       };
+      const int nblk = w.nblk;
       if (nblk > 0) emit(true, 0);
       if (ok && nblk > 1) emit(true, 1);
       for (int j = 0; ok && j < nblk; ++j) {
         emit(false, j);
         if (ok && j + 2 < nblk) emit(true, j + 2);
       }
-      mbar_wait_drain(q_full, 0, p.wd);
+      }
+      // nothing may still land at exit: the last load into each Q buffer
+      // and into each slot
+      for (int qb = 0; qb < Cfg::kQBufs; ++qb) {
+        const int uses = (it - qb + Cfg::kQBufs - 1) / Cfg::kQBufs;
+        if (uses > 0) mbar_wait_drain(&q_full[qb], (uint32_t)(uses - 1) & 1u, p.wd);
+      }
       for (int v = u - NSLOT > 0 ? u - NSLOT : 0; v < u; ++v)
         mbar_wait_drain(&slot_full[v % NSLOT], (uint32_t)(v / NSLOT) & 1u, p.wd);
     }
   } else if (warp == 6) {
     // ============ odd CTA: relay its load completions to the even CTA ============
     if (!leader && lane == 0) {
-      const int nloads = nblk > 0 ? 2 * nblk : 0;
-      const uint32_t leader_peer_q = mapa_shared(smem_u32(peer_q), 0);
-      bool ok = mbar_wait(q_full, 0, p.wd, kWdTmaFull);
-      if (ok) mbar_arrive_cluster(leader_peer_q);
-      for (int u = 0; ok && u < nloads; ++u) {
-        const int slot = u % NSLOT;
-        if (!mbar_wait(&slot_full[slot], (uint32_t)(u / NSLOT) & 1u, p.wd, kWdTmaFull)) break;
-        mbar_arrive_cluster(mapa_shared(smem_u32(&peer_full[slot]), 0));
+      int u = 0, it = 0;
+      bool ok = true;
+      for (; ok; ++it) {
+        const int item = tc2_item(it, pid, npairs, n_items);
+        if (item < 0) break;
+        const int nblk = tc2_tile<BN, Cfg::kBM>(p, item, rank).nblk;
+        const int qb = it % Cfg::kQBufs, use = it / Cfg::kQBufs;
+        if (!mbar_wait(&q_full[qb], (uint32_t)use & 1u, p.wd, kWdTmaFull)) break;
+        mbar_arrive_cluster(mapa_shared(smem_u32(&peer_q[qb]), 0));
+        const int nloads = nblk > 0 ? 2 * nblk : 0;
+        for (int v = 0; v < nloads; ++v, ++u) {
+          const int slot = u % NSLOT;
+          if (!mbar_wait(&slot_full[slot], (uint32_t)(u / NSLOT) & 1u, p.wd, kWdTmaFull)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_cluster(mapa_shared(smem_u32(&peer_full[slot]), 0));
+        }
       }
     }
   } else if (warp == 5) {
@@ -220,7 +311,7 @@ __global__ void __launch_bounds__(224, 1)
     if (leader && lane == 0) {
       constexpr uint32_t kIdescS = umma_idesc_f16(kBF16, 256, BN, false, false);
       constexpr uint32_t kIdescPV = umma_idesc_f16(kBF16, 256, DV, false, true);
-      const uint32_t q_addr = smem_u32(sQ);
+      uint32_t q_addr = smem_u32(sQ);
       const uint32_t slot_addr = smem_u32(sSlots);
       // commit targets in both CTAs
       auto both = [&](uint64_t *bar) {
@@ -228,8 +319,7 @@ __global__ void __launch_bounds__(224, 1)
         tc_commit_pair(mapa_shared(a, 0));
         tc_commit_pair(mapa_shared(a, 1));
       };
-      bool ok = mbar_wait(q_full, 0, p.wd, kWdTmaFull) &&
-                mbar_wait_cluster(peer_q, 0, p.wd, kWdTmaFull);
+      bool ok = true;
       int u = 0;
       auto take_slot = [&](int &slot) -> bool {
         slot = u % NSLOT;
@@ -239,10 +329,11 @@ __global__ void __launch_bounds__(224, 1)
         ++u;
         return true;
       };
-      auto issue_s = [&](int n) -> bool {
+      // x: the key block's index counted over all of the pair's tiles
+      auto issue_s = [&](int x) -> bool {
         int slot;
         if (!take_slot(slot)) return false;
-        const int b = n & 1;
+        const int b = x & 1;
         tc_fence_after();
         const uint64_t a0 = umma_desc_sw128(q_addr, 16, 1024);
         const uint64_t b0 = umma_desc_sw128(slot_addr + slot * Cfg::kSlotBytes, 16, 1024);
@@ -256,11 +347,12 @@ __global__ void __launch_bounds__(224, 1)
         both(&slot_empty[slot]);
         return true;
       };
-      auto issue_pv = [&](int j) -> bool {
+      // j: the block within the tile (the first one overwrites O)
+      auto issue_pv = [&](int j, int x) -> bool {
         int slot;
         if (!take_slot(slot)) return false;
-        const int b = j & 1;
-        if (!mbar_wait_cluster(&p_full[b], (uint32_t)(j >> 1) & 1u, p.wd, kWdSoftmax)) return false;
+        const int b = x & 1;
+        if (!mbar_wait_cluster(&p_full[b], (uint32_t)(x >> 1) & 1u, p.wd, kWdSoftmax)) return false;
         tc_fence_after();
         const uint64_t v0 = umma_desc_sw128_mn(slot_addr + slot * Cfg::kSlotBytes, BN * 128, 1024);
 #pragma unroll
@@ -273,13 +365,24 @@ __global__ void __launch_bounds__(224, 1)
         both(&slot_empty[slot]);
         return true;
       };
-      if (ok && nblk > 0) ok = issue_s(0);
-      if (ok && nblk > 1) ok = issue_s(1);
-      for (int j = 0; ok && j < nblk; ++j) {
-        ok = issue_pv(j);
-        if (ok && j + 2 < nblk) ok = issue_s(j + 2);
+      int it = 0, x0 = 0;
+      for (; ok; ++it) {
+        const int item = tc2_item(it, pid, npairs, n_items);
+        if (item < 0) break;
+        const int nblk = tc2_tile<BN, Cfg::kBM>(p, item, rank).nblk;
+        const int qb = it % Cfg::kQBufs, use = it / Cfg::kQBufs;
+        ok = mbar_wait(&q_full[qb], (uint32_t)use & 1u, p.wd, kWdTmaFull) &&
+             mbar_wait_cluster(&peer_q[qb], (uint32_t)use & 1u, p.wd, kWdTmaFull);
+        q_addr = smem_u32(sQ + qb * Cfg::kQBytes);
+        if (ok && nblk > 0) ok = issue_s(x0);
+        if (ok && nblk > 1) ok = issue_s(x0 + 1);
+        for (int j = 0; ok && j < nblk; ++j) {
+          ok = issue_pv(j, x0 + j);
+          if (ok && j + 2 < nblk) ok = issue_s(x0 + j + 2);
+        }
+        if (ok && nblk > 0) both(o_final);
+        x0 += nblk;
       }
-      if (ok && nblk > 0) both(o_final);
       both(fin_bar);
     }
   } else {
@@ -287,7 +390,6 @@ __global__ void __launch_bounds__(224, 1)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    const int pos = ((tr.row0 + r) % p.L) + p.off;
     const float c = p.scale_log2;
     // scale 0 weighs every visible key the same: the scores are zeroed and 1
     // is used as the factor, so a masked key (set to the neutral value below)
@@ -296,13 +398,36 @@ __global__ void __launch_bounds__(224, 1)
     const float c_eff = c_zero ? 1.f : c;
     const bool c_pos = c >= 0.f;
     const float neutral = c_pos ? -INFINITY : INFINITY;
-    float m_used = -INFINITY, l = 0.f;
+    const long total_rows = (long)p.B * p.Hq * p.L;
+    const bool split_out = p.splits > 1;
     bool ok = true;
+    // looping form: the Q buffer whose staged output a TMA store may still be
+    // reading (warp 0 lane 0 issued the store); handed back to the producer
+    // once the store has read it
+    int pend_q = -1;
+    auto release_q = [&]() {
+      if (PERSIST && warp == 0 && lane == 0 && pend_q >= 0) {
+        bulk_wait_group_read0();
+        mbar_arrive(&q_empty[pend_q]);
+        pend_q = -1;
+      }
+    };
+    int it = 0, x0 = 0, nfin = 0;
+    for (; ok; ++it) {
+      const int item = tc2_item(it, pid, npairs, n_items);
+      if (item < 0) break;
+    const Tc2Tile w = tc2_tile<BN, Cfg::kBM>(p, item, rank);
+    const TileRows &tr = w.tr;
+    const int nblk = w.nblk;
+    const int qb = it % Cfg::kQBufs;
+    const int pos = ((tr.row0 + r) % p.L) + p.off;
+    float m_used = -INFINITY, l = 0.f;
     for (int j = 0; j < nblk; ++j) {
-      const int b = j & 1;
-      bool w = true;
-      if (lane == 0) w = mbar_wait_cluster(&s_full[b], (uint32_t)(j >> 1) & 1u, p.wd, kWdMma);
-      if (!__shfl_sync(0xffffffffu, (int)w, 0)) {
+      const int x = x0 + j;  // block index over the pair's tiles
+      const int b = x & 1;
+      bool wt = true;
+      if (lane == 0) wt = mbar_wait_cluster(&s_full[b], (uint32_t)(x >> 1) & 1u, p.wd, kWdMma);
+      if (!__shfl_sync(0xffffffffu, (int)wt, 0)) {
         ok = false;
         break;
       }
@@ -313,7 +438,7 @@ __global__ void __launch_bounds__(224, 1)
         tmem_ld32(tmem + lane_base + b * BN + c32 * 32, s + c32 * 32);
       tmem_wait_ld();
 
-      const int kbase = k_lo + j * BN;
+      const int kbase = w.k_lo + j * BN;
       const bool masked = block_needs_mask(p, tr, kbase, BN);
       // The common block (positive scale, no masked key) takes the plain
       // reduction; the rare ones (scale 0, masked keys, negative scale) their
@@ -344,11 +469,11 @@ __global__ void __launch_bounds__(224, 1)
         l *= alpha;
       }
       if (j > 0 && __any_sync(0xffffffffu, need)) {
-        // S_j was issued after P_{j-2} V by the same thread, and P_j V waits
-        // for p_full: o_bar is in phase j-1 or j here.  The TMEM loads and
+        // S_x was issued after P_{x-2} V by the same thread, and P_x V waits
+        // for p_full: o_bar is in phase x-1 or x here.  The TMEM loads and
         // stores are warp-wide, so the whole warp rescales its rows.
-        if (lane == 0) w = mbar_wait_cluster(o_bar, (uint32_t)(j - 1) & 1u, p.wd, kWdMma);
-        if (!__shfl_sync(0xffffffffu, (int)w, 0)) {
+        if (lane == 0) wt = mbar_wait_cluster(o_bar, (uint32_t)(x - 1) & 1u, p.wd, kWdMma);
+        if (!__shfl_sync(0xffffffffu, (int)wt, 0)) {
           ok = false;
           break;
         }
@@ -394,17 +519,21 @@ __global__ void __launch_bounds__(224, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&p_full[b]), 0));
+      // the previous tile's store has long read its buffer by now
+      if (j == 0) release_q();
     }
 
     // ------------------------------ epilogue ------------------------------
     if (ok && nblk > 0) {
-      bool w = true;
-      if (lane == 0) w = mbar_wait_cluster(o_final, 0, p.wd, kWdMma);
-      ok = __shfl_sync(0xffffffffu, (int)w, 0) != 0;
+      bool wt = true;
+      if (lane == 0) wt = mbar_wait_cluster(o_final, (uint32_t)nfin & 1u, p.wd, kWdMma);
+      ok = __shfl_sync(0xffffffffu, (int)wt, 0) != 0;
       tc_fence_after();
     }
+    if (nblk > 0) ++nfin;
+    release_q();  // a tile without blocks released nothing above
     const bool valid = r < tr.nvalid;
-    const long grow = (long)bh * p.R + tr.row0 + r;
+    const long grow = (long)w.bh * p.R + tr.row0 + r;
     const bool have_o = ok && nblk > 0;
     // O leaves TMEM kOGroup chunks of 16 columns per wait
     constexpr int kOChunks = DV / 16;
@@ -423,13 +552,12 @@ __global__ void __launch_bounds__(224, 1)
           for (int e = 0; e < 16; ++e) o[k][e] = 0.f;
       }
     };
-    // Output rows are staged in this CTA's K/V slots (free: o_final fired
-    // once every MMA of the pair had completed) in the TMA store's swizzled
-    // box layout, then one thread stores them in boxes of 128 rows; rows past
+    // Output rows are staged in the TMA store's swizzled box layout, in this
+    // CTA's K/V slots (free: o_final fired once every MMA of the pair had
+    // completed) or, looping, in this tile's Q buffer (free for the same
+    // reason), then one thread stores them in boxes of 128 rows; rows past
     // the slab and columns past Dv are clipped by the tensor map.
-    const long total_rows = (long)p.B * p.Hq * p.L;
-    const bool split_out = p.splits > 1;
-    uint8_t *stage = sSlots;
+    uint8_t *stage = PERSIST ? sQ + qb * Cfg::kQBytes : sSlots;
     if (!split_out) {
       const float inv = finish_row(p, grow, m_used, l);  // folds in the sink, if any
       if (p.lse_out != nullptr && valid) p.lse_out[grow] = row_lse(m_used, l);
@@ -446,10 +574,10 @@ __global__ void __launch_bounds__(224, 1)
           stage_16bit_x16(stage, r, g * kOGroup + k, w8);
         }
       }
-    } else {
+    } else if constexpr (!PERSIST) {
       const float inv = l > 0.f ? 1.f / l : 0.f;
       if (valid)
-        p.part_lse[(long)split * total_rows + grow] = have_o ? row_lse(m_used, l) : -INFINITY;
+        p.part_lse[(long)w.split * total_rows + grow] = have_o ? row_lse(m_used, l) : -INFINITY;
 #pragma unroll 1
       for (int g = 0; g < kOChunks / kOGroup; ++g) {
         float o[kOGroup][16];
@@ -464,18 +592,27 @@ __global__ void __launch_bounds__(224, 1)
     }
     fence_proxy_async_smem();
     asm volatile("bar.sync 1, 128;" ::: "memory");  // the four softmax warps
-    if (warp == 0 && lane == 0 && tr.nvalid > 0) {
-      if (!split_out) {
-        for (int bx = 0; bx < Cfg::kOutBoxes && bx * 64 < p.Dv; ++bx)
-          tma_store_3d(&tm_o, stage + bx * (Cfg::kBM * 128), bx * 64, tr.row0, bh);
-      } else {
-        for (int bx = 0; bx < Cfg::kF32Boxes && bx * 32 < p.Dv; ++bx)
-          tma_store_3d(&tm_p, stage + bx * (Cfg::kBM * 128), bx * 32, tr.row0,
-                       split * BH + bh);
+    if (warp == 0 && lane == 0) {
+      if (tr.nvalid > 0) {
+        if (!split_out) {
+          for (int bx = 0; bx < Cfg::kOutBoxes && bx * 64 < p.Dv; ++bx)
+            tma_store_3d(&tm_o, stage + bx * (Cfg::kBM * 128), bx * 64, tr.row0, w.bh);
+        } else {
+          for (int bx = 0; bx < Cfg::kF32Boxes && bx * 32 < p.Dv; ++bx)
+            tma_store_3d(&tm_p, stage + bx * (Cfg::kBM * 128), bx * 32, tr.row0,
+                         w.split * BH + w.bh);
+        }
+        bulk_commit_group();
       }
-      bulk_commit_group();
-      bulk_wait_group0();
+      if (PERSIST)
+        pend_q = qb;  // handed back once read, under the next tile's first block
+      else
+        bulk_wait_group0();
     }
+    x0 += nblk;
+    }
+    // every store has completed before the CTA leaves
+    if (warp == 0 && lane == 0) bulk_wait_group0();
   }
 
   // ------------------------------ teardown ------------------------------

@@ -214,3 +214,34 @@ def test_plan_two_tile_path_for_small_head_dims():
     with pytest.raises(sdpa.SdpaError) as ei:
         sdpa.plan(1, 4, 4, 512, 512, 192, 128, num_sms=148, force_path=sdpa.PATH_TC_DUAL)
     assert ei.value.status == 2
+
+
+def test_plan_looping_pair_path():
+    # sliding windows over more 256-row tiles than SM pairs: the pair kernel
+    # loops over its tiles
+    for n in (2048, 4096, 8192):
+        info = sdpa.plan(1, 16, 8, n, n, 256, 256, causal=True, window_size=1024, num_sms=148)
+        assert info["path"] == sdpa.PATH_TC2_LOOP and info["splits"] == 1
+        assert info["ctas"] == 8 * (2 * n // 256) and info["launches"] == 1
+        assert info["workspace_bytes"] == 0
+    # long causal tiles keep one pair per tile
+    info = sdpa.plan(1, 16, 8, 32768, 32768, 256, 256, causal=True, num_sms=148)
+    assert info["path"] == sdpa.PATH_TC2
+    # fewer tiles than SM pairs: nothing to loop over (the keys are split instead)
+    info = sdpa.plan(1, 4, 2, 2048, 2048, 256, 256, causal=True, window_size=1024, num_sms=148)
+    assert info["path"] == sdpa.PATH_TC2 and info["splits"] > 1
+    # a window wider than a tile's share of short keys still loops; a long one does not
+    info = sdpa.plan(1, 16, 8, 8192, 8192, 256, 256, causal=True, window_size=8000, num_sms=148)
+    assert info["path"] == sdpa.PATH_TC2
+    # forced: never splits, takes the pair instances (head dims zero filled)
+    info = sdpa.plan(1, 4, 4, 512, 512, 64, 64, num_sms=148, force_path=sdpa.PATH_TC2_LOOP)
+    assert info["path"] == sdpa.PATH_TC2_LOOP and info["dqk_pad"] == 128 and info["splits"] == 1
+    info = sdpa.plan(1, 1, 1, 256, 32768, 256, 256, num_sms=148, force_path=sdpa.PATH_TC2_LOOP)
+    assert info["splits"] == 1 and info["ctas"] == 1
+    with pytest.raises(sdpa.SdpaError) as ei:
+        sdpa.plan(1, 1, 1, 256, 32768, 256, 256, num_sms=148, force_path=sdpa.PATH_TC2_LOOP,
+                  force_splits=2)
+    assert ei.value.status == 2 and "split" in ei.value.message
+    with pytest.raises(sdpa.SdpaError) as ei:
+        sdpa.plan(1, 4, 4, 64, 64, 512, 512, num_sms=148, force_path=sdpa.PATH_TC2_LOOP)
+    assert ei.value.status == 2
