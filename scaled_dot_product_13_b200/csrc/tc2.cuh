@@ -21,9 +21,14 @@
 //              BN columns of a block, so a row's max needs no exchange
 //              between warps; lazily moved running max as in tc.cuh.  P_j is
 //              written over the row's own scores in this CTA's TMEM and
-//              signalled to the even CTA's p_full.
+//              signalled with a CTA-scope arrive: on the even CTA's p_full,
+//              or on the odd CTA's p_local.
 //   warp 4     TMA producer for this CTA's halves.
-//   warp 5     TMEM allocation (pair); the MMA issuer in the even CTA.
+//   warp 5     TMEM allocation (pair); the MMA issuer in the even CTA; in
+//              the odd CTA it relays each completed p_local phase to the
+//              even CTA's p_full.  A cluster-scope release costs the issuing
+//              warp several hundred cycles, so it is taken once per block
+//              here instead of once per softmax warp on the softmax's path.
 //   warp 6     odd CTA: forwards its load completions to the even CTA.
 //
 // TMEM per CTA: two score buffers of BN columns (P_j over the first BN/2
@@ -70,7 +75,7 @@ struct Tc2Cfg {
   static constexpr uint32_t kSlotBytes = kKBytes > kVBytes ? kKBytes : kVBytes;
   static constexpr uint32_t kSlotOff = kQBufs * kQBytes;
   static constexpr uint32_t kBarOff = kSlotOff + NSLOT * kSlotBytes;
-  static constexpr int kNumBars = 3 * NSLOT + 16;
+  static constexpr int kNumBars = 3 * NSLOT + 20;
   static constexpr uint32_t kSmemBytes = kBarOff + kNumBars * 8 + 16;
   static constexpr int kThreads = 224;
   static constexpr uint32_t kTmemCols = 512;
@@ -168,7 +173,8 @@ __global__ void __launch_bounds__(224, 1)
   uint64_t *q_empty = peer_q + 2;            // [2] looping form: the store has read the buffer
   uint64_t *s_full = q_empty + 2;            // [2]
   uint64_t *p_full = s_full + 2;             // [2] even CTA: P_j of both CTAs written
-  uint64_t *o_bar = p_full + 2;
+  uint64_t *p_local = p_full + 2;            // [2] odd CTA: P_j of its four warps written
+  uint64_t *o_bar = p_local + 2;
   uint64_t *o_final = o_bar + 1;
   uint64_t *fin_bar = o_final + 1;           // all MMAs of the pair complete
   uint64_t *bye_bar = fin_bar + 1;           // teardown: the other CTA is done with us
@@ -196,7 +202,8 @@ __global__ void __launch_bounds__(224, 1)
       mbar_init(&peer_q[b], 1);
       mbar_init(&q_empty[b], 1);
       mbar_init(&s_full[b], 1);
-      mbar_init(&p_full[b], 8);
+      mbar_init(&p_full[b], 5);  // the even CTA's four warps, the odd CTA's relay
+      mbar_init(&p_local[b], 4);
     }
     mbar_init(o_bar, 1);
     mbar_init(o_final, 1);
@@ -384,6 +391,24 @@ __global__ void __launch_bounds__(224, 1)
         x0 += nblk;
       }
       both(fin_bar);
+    } else if (!leader && lane == 0) {
+      // ============ odd CTA: relay P_x of its softmax warps ============
+      const uint32_t leader_p_full = mapa_shared(smem_u32(p_full), 0);
+      int it = 0, x = 0;
+      bool ok = true;
+      for (; ok; ++it) {
+        const int item = tc2_item(it, pid, npairs, n_items);
+        if (item < 0) break;
+        const int nblk = tc2_tile<BN, Cfg::kBM>(p, item, rank).nblk;
+        for (int j = 0; j < nblk; ++j, ++x) {
+          const int b = x & 1;
+          if (!mbar_wait(&p_local[b], (uint32_t)(x >> 1) & 1u, p.wd, kWdSoftmax)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_cluster(leader_p_full + (uint32_t)b * 8u);
+        }
+      }
     }
   } else {
     // ====== softmax warps 0-3: one row of this CTA's 128 per thread ======
@@ -518,7 +543,7 @@ __global__ void __launch_bounds__(224, 1)
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&p_full[b]), 0));
+      if (lane == 0) mbar_arrive(leader ? &p_full[b] : &p_local[b]);
       // the previous tile's store has long read its buffer by now
       if (j == 0) release_q();
     }
