@@ -556,6 +556,16 @@ __device__ __forceinline__ void tc_commit_pair(uint32_t cluster_addr) {
       : "memory");
 }
 
+// One commit that arrives on the barrier at the same shared-memory offset in
+// both CTAs of the pair (CTA mask 0b11).
+__device__ __forceinline__ void tc_commit_pair_both(uint64_t *bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 "
+      "[%0], %1;" ::"r"(smem_u32(bar)),
+      "h"((uint16_t)3)
+      : "memory");
+}
+
 // Shared-memory matrix descriptor for tcgen05.mma, 128-byte swizzle.
 //   start: smem byte address; lbo/sbo: leading / stride byte offsets.
 // Bits: [0,14) start>>4, [16,30) lbo>>4, [32,46) sbo>>4, [46,48) version 1,
