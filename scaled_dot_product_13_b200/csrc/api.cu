@@ -209,10 +209,10 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
                 "the wide path is built for head dims above 256 (got Dqk=%d, Dv=%d)", pb.Dqk,
                 pb.Dv);
   if (wide && force_path != SDPA_PATH_AUTO && force_path != SDPA_PATH_WIDE &&
-      force_path != SDPA_PATH_TC)
+      force_path != SDPA_PATH_TC && force_path != SDPA_PATH_TC2)
     return fail(SDPA_ERR_UNSUPPORTED,
                 "head dims above 256 (got Dqk=%d, Dv=%d) run on the wide path or the tcgen05 "
-                "path",
+                "paths (one or two SMs per tile)",
                 pb.Dqk, pb.Dv);
   if (force_splits < 0) return fail(SDPA_ERR_INVALID_ARG, "force_splits must be >= 0");
   if (num_sms < 1) num_sms = 148;
@@ -224,9 +224,15 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
   // split-KV kernel on 16-row warp tiles.  Both split the keys when the
   // tiles alone do not fill the GPU.
   int path = force_path;
-  // head dims above 256: packed rows that fill a 128-row tile take tcgen05
-  if (path == SDPA_PATH_AUTO && wide)
+  // head dims above 256: packed rows that fill a 128-row tile take tcgen05;
+  // from one 256-row tile, and with at least one pair's work per two SMs
+  // (that kernel does not split the keys), an SM pair per tile
+  if (path == SDPA_PATH_AUTO && wide) {
     path = pl.rows >= kTcRowThreshold ? SDPA_PATH_TC : SDPA_PATH_WIDE;
+    const long long pair_units = (long long)pb.B * pb.Hkv * ((pl.rows + 255) / 256) *
+                                 ((pb.Dv + kTc2WideHalf - 1) / kTc2WideHalf);
+    if (pl.rows >= kTc2RowThreshold && 2 * pair_units >= num_sms) path = SDPA_PATH_TC2;
+  }
   if (path == SDPA_PATH_AUTO) {
     path = pl.rows >= kTcRowThreshold ? SDPA_PATH_TC : SDPA_PATH_SPLITKV;
     // wide heads with at least one full 256-row pair tile: two SMs per tile
@@ -276,7 +282,9 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
   } else if (pair_path) {
     pl.wr = 0; pl.wk = 0;
     pl.row_tile = 2 * kTcRows;
-    pl.key_block = 128;
+    // head dim 512: 64-key blocks in 256-column halves (grid.y)
+    pl.key_block = wide ? 64 : 128;
+    if (wide) pl.col_halves = (pb.Dv + kTc2WideHalf - 1) / kTc2WideHalf;
   } else if (path == SDPA_PATH_TC) {
     pl.wr = 0; pl.wk = 0;
     pl.row_tile = kTcRows;
@@ -316,10 +324,11 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
                                                       kDimPairs[pl.pair].dv, pl.wr)
                                 : 1);
   int splits;
-  if (path == SDPA_PATH_TC2_LOOP) {
-    // the looping form writes finished rows only
+  if (path == SDPA_PATH_TC2_LOOP || (path == SDPA_PATH_TC2 && wide)) {
+    // the looping form, and the pair kernel at head dims above 256, write
+    // finished rows only
     if (force_splits > 1)
-      return fail(SDPA_ERR_UNSUPPORTED, "the looping pair path does not split the keys");
+      return fail(SDPA_ERR_UNSUPPORTED, "this pair path does not split the keys");
     splits = 1;
   } else if (force_splits > 0) {
     splits = std::min(force_splits, nkb);
@@ -346,7 +355,7 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
   // Windowed or short unsplit tiles on the pair kernel, more of them than SM
   // pairs: loop over tiles.  A tile visits at most the window's blocks plus
   // its own 256 rows' worth (or all of them without a window).
-  if (force_path == SDPA_PATH_AUTO && path == SDPA_PATH_TC2 && splits == 1 &&
+  if (force_path == SDPA_PATH_AUTO && path == SDPA_PATH_TC2 && !wide && splits == 1 &&
       pl.ctas > num_sms / 2) {
     const int tile_blocks =
         pb.window > 0 ? std::min(nkb, (pb.window + pl.row_tile + bn - 1) / bn + 1) : nkb;

@@ -181,7 +181,11 @@ constexpr bool tc_dual_supports_pair(int pair) { return pair <= 2; }
 // Head-dim pairs the two-CTA kernel is built for (index into kDimPairs), and
 // those the router sends to it by itself (where it measured faster than one
 // SM per 128-row tile).
-constexpr bool tc2_supports_pair(int pair) { return pair == 2 || pair == 3 || pair == 5; }
+constexpr bool tc2_supports_pair(int pair) {
+  return pair == 2 || pair == 3 || pair == 5 || pair == kWidePair;
+}
+// Output columns per launch column of the two-CTA kernel at head dim 512.
+constexpr int kTc2WideHalf = 256;
 constexpr bool tc2_preferred_pair(int pair) { return pair == 3 || pair == 5; }
 sdpa_status launch_combine(const Launch &ln, std::string *err);
 

@@ -7,13 +7,14 @@ namespace sdpa {
 namespace {
 
 // kLoop: the looping form (two Q buffers, so fewer K/V slots), grid of
-// plan.loop_pairs pairs; otherwise one pair per 256-row tile.
-template <bool kBF16, int DQK, int DV, bool kLoop>
+// plan.loop_pairs pairs; otherwise one pair per 256-row tile.  DV is the
+// output columns of one launch column (grid.y = plan.col_halves); kBN the
+// key block.
+template <bool kBF16, int DQK, int DV, bool kLoop, int kBN = 128>
 sdpa_status run_tc2(const Launch &ln, std::string *err) {
-  constexpr int kBN = 128;
   constexpr uint32_t kQ = (DQK / 64) * 128 * 128;
   constexpr uint32_t kK = (DQK / 64) * (kBN / 2) * 128;
-  constexpr uint32_t kV = (DV / 128) * kBN * 128;
+  constexpr uint32_t kV = (DV / 128) * kBN * 128;  // this CTA's DV/2 columns
   constexpr uint32_t kSlot = kK > kV ? kK : kV;
   constexpr uint32_t kBudget = 232448u - 48u * 8u - 16u;
   constexpr int kFit = (int)((kBudget - (kLoop ? 2u : 1u) * kQ) / kSlot);
@@ -21,6 +22,10 @@ sdpa_status run_tc2(const Launch &ln, std::string *err) {
   static_assert(kNSlot >= 3, "at least three K/V slots");
   using Cfg = Tc2Cfg<DQK, DV, kBN, kNSlot, kLoop>;
   auto kern = tc2_attn_kernel<kBF16, DQK, DV, kBN, kNSlot, kLoop>;
+  if (!Cfg::kSplitStage && ln.plan.splits != 1) {
+    *err = "internal: this two-CTA instance does not split the keys";
+    return SDPA_ERR_UNSUPPORTED;
+  }
   sdpa_status st =
       prepare_kernel((const void *)kern, Cfg::kThreads, Cfg::kSmemBytes, "tc2_attn_kernel", err);
   if (st != SDPA_OK) return st;
@@ -67,7 +72,8 @@ sdpa_status run_tc2(const Launch &ln, std::string *err) {
   p.wd.limit_ns = ln.wd_limit_ns;
 
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(2 * (kLoop ? (long long)pl.loop_pairs : pl.ctas)));
+  cfg.gridDim = dim3((unsigned)(2 * (kLoop ? (long long)pl.loop_pairs : pl.ctas / pl.col_halves)),
+                     (unsigned)pl.col_halves);
   cfg.blockDim = dim3(Cfg::kThreads);
   cfg.dynamicSmemBytes = Cfg::kSmemBytes;
   cfg.stream = ln.stream;
@@ -95,6 +101,11 @@ sdpa_status run_dtype(const Launch &ln, std::string *err) {
     case 2: return run_tc2<kBF16, 128, 128, kLoop>(ln, err);
     case 3: return run_tc2<kBF16, 192, 128, kLoop>(ln, err);
     case 5: return run_tc2<kBF16, 256, 256, kLoop>(ln, err);
+    case kWidePair:
+      // head dim 512 in two 256-column halves, 64-key blocks (the 128 KB Q
+      // tile leaves room for three 32 KB K/V slots and no second Q buffer)
+      if constexpr (!kLoop) return run_tc2<kBF16, 512, kTc2WideHalf, false, 64>(ln, err);
+      break;
   }
   *err = "internal: no two-CTA instance for this head-dim pair";
   return SDPA_ERR_UNSUPPORTED;

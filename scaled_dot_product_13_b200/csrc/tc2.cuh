@@ -82,7 +82,7 @@ struct Tc2Cfg {
   static constexpr uint32_t kTmemCols = 512;
   static constexpr int kOCol = 2 * BN;
   static_assert(DQK % 64 == 0 && (DV == 128 || DV == 256), "pair split needs 64-column halves");
-  static_assert(BN == 128, "key block");
+  static_assert(BN == 64 || BN == 128, "key block");
   static_assert(2 * BN + DV <= 512, "TMEM columns");
   static_assert(kSmemBytes <= 232448, "shared memory");
   // the epilogue stages the CTA's 128 output rows, 64 columns of a 16-bit
@@ -91,8 +91,10 @@ struct Tc2Cfg {
   static constexpr int kOutBoxes = (DV + 63) / 64;
   static constexpr int kF32Boxes = (DV + 31) / 32;
   static_assert(PERSIST ? kOutBoxes * kBM * 128 <= kQBytes
-                        : kF32Boxes * kBM * 128 <= NSLOT * kSlotBytes,
+                        : kOutBoxes * kBM * 128 <= NSLOT * kSlotBytes,
                 "output staging");
+  // whether split partials fit the slots (head dim 512 per column half: not)
+  static constexpr bool kSplitStage = !PERSIST && kF32Boxes * kBM * 128 <= NSLOT * kSlotBytes;
 };
 
 // One work item of a pair: (batch*KV head) fastest, then split, then the
@@ -157,8 +159,9 @@ __global__ void __launch_bounds__(224, 1)
     if (threadIdx.x == 0) wd_record(p.wd, kWdSmemAlign);
     return;
   }
-  // the looping form stages 16-bit output rows only (no split partials)
-  if (PERSIST && p.splits != 1) {
+  // the looping form, and instances whose slots cannot hold fp32 partials,
+  // write finished 16-bit rows only (no key splits)
+  if (!Cfg::kSplitStage && p.splits != 1) {
     if (threadIdx.x == 0) wd_record(p.wd, kWdConfig);
     return;
   }
@@ -191,6 +194,9 @@ __global__ void __launch_bounds__(224, 1)
   const int n_items = BH * p.splits * p.row_tiles;
   const int pid = (int)(blockIdx.x >> 1);
   const int npairs = (int)(gridDim.x >> 1);
+  // the DV output columns of this launch column (head dims above 256 run in
+  // column halves, grid.y = 2: both halves compute the same scores)
+  const int dv0 = (int)blockIdx.y * DV;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NSLOT; ++s) {
@@ -270,7 +276,7 @@ __global__ void __launch_bounds__(224, 1)
 #pragma unroll
           for (int bx = 0; bx < Cfg::kVBoxes; ++bx)
             tma_load_3d(dst + bx * (BN * 128), &tm_v, &slot_full[slot],
-                        (int)rank * Cfg::kVHalf + bx * 64, k0, w.bh);
+                        dv0 + (int)rank * Cfg::kVHalf + bx * 64, k0, w.bh);
         }
         ++u;
       };
@@ -582,7 +588,7 @@ __global__ void __launch_bounds__(224, 1)
     uint8_t *stage = PERSIST ? sQ + qb * Cfg::kQBytes : sSlots;
     if (!split_out) {
       const float inv = finish_row(p, grow, m_used, l);  // folds in the sink, if any
-      if (p.lse_out != nullptr && valid) p.lse_out[grow] = row_lse(m_used, l);
+      if (p.lse_out != nullptr && valid && dv0 == 0) p.lse_out[grow] = row_lse(m_used, l);
 #pragma unroll 1
       for (int g = 0; g < kOChunks / kOGroup; ++g) {
         float o[kOGroup][16];
@@ -596,9 +602,9 @@ __global__ void __launch_bounds__(224, 1)
           stage_16bit_x16(stage, r, g * kOGroup + k, w8);
         }
       }
-    } else if constexpr (!PERSIST) {
+    } else if constexpr (Cfg::kSplitStage) {
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      if (valid)
+      if (valid && dv0 == 0)
         p.part_lse[(long)w.split * total_rows + grow] = have_o ? row_lse(m_used, l) : -INFINITY;
 #pragma unroll 1
       for (int g = 0; g < kOChunks / kOGroup; ++g) {
@@ -617,11 +623,11 @@ __global__ void __launch_bounds__(224, 1)
     if (warp == 0 && lane == 0) {
       if (tr.nvalid > 0) {
         if (!split_out) {
-          for (int bx = 0; bx < Cfg::kOutBoxes && bx * 64 < p.Dv; ++bx)
-            tma_store_3d(&tm_o, stage + bx * (Cfg::kBM * 128), bx * 64, tr.row0, w.bh);
-        } else {
-          for (int bx = 0; bx < Cfg::kF32Boxes && bx * 32 < p.Dv; ++bx)
-            tma_store_3d(&tm_p, stage + bx * (Cfg::kBM * 128), bx * 32, tr.row0,
+          for (int bx = 0; bx < Cfg::kOutBoxes && dv0 + bx * 64 < p.Dv; ++bx)
+            tma_store_3d(&tm_o, stage + bx * (Cfg::kBM * 128), dv0 + bx * 64, tr.row0, w.bh);
+        } else if constexpr (Cfg::kSplitStage) {
+          for (int bx = 0; bx < Cfg::kF32Boxes && dv0 + bx * 32 < p.Dv; ++bx)
+            tma_store_3d(&tm_p, stage + bx * (Cfg::kBM * 128), dv0 + bx * 32, tr.row0,
                          w.split * BH + w.bh);
         }
         bulk_commit_group();

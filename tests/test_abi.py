@@ -176,10 +176,15 @@ def test_plan_head_dims_above_256():
     assert info["row_tile"] == 16 and info["key_block"] == 32 and info["splits"] > 1
     # short verify windows (fewer than 65 packed rows) stay on the wide path
     assert sdpa.plan(1, 8, 2, 12, 4096, 512, 512, num_sms=148)["path"] == sdpa.PATH_WIDE
-    # prefill: the tcgen05 kernel in two column halves (two CTAs per row tile)
+    # prefill: the pair kernel in two column halves, 64-key blocks, never split
     info = sdpa.plan(1, 8, 8, 4096, 4096, 512, 512, causal=True, num_sms=148)
+    assert info["path"] == sdpa.PATH_TC2 and info["row_tile"] == 256 and info["key_block"] == 64
+    assert info["ctas"] == 8 * 16 * 2 and info["splits"] == 1 and info["workspace_bytes"] == 0
+    # too few pair tiles to give every two SMs one: the one-SM kernel in
+    # column halves (two CTAs per row tile)
+    info = sdpa.plan(1, 4, 4, 512, 512, 512, 512, causal=True, num_sms=148)
     assert info["path"] == sdpa.PATH_TC and info["row_tile"] == 128 and info["key_block"] == 32
-    assert info["ctas"] == 8 * 32 * 2 and info["splits"] == 1
+    assert info["ctas"] == 4 * 4 * 2
     # few row tiles: keys split, each split at least 256 keys
     info = sdpa.plan(1, 8, 2, 64, 8192, 512, 512, num_sms=148)
     assert info["path"] == sdpa.PATH_TC and info["splits"] > 1
@@ -187,14 +192,20 @@ def test_plan_head_dims_above_256():
     # mixed dims above 256 run on the 512/512 instance
     assert sdpa.plan(1, 4, 4, 64, 64, 320, 128, num_sms=148)["path"] == sdpa.PATH_WIDE
     assert sdpa.plan(1, 4, 4, 128, 128, 128, 384, num_sms=148)["path"] == sdpa.PATH_TC
-    # the split-KV and pair kernels do not take them, and the wide path
-    # takes nothing else
-    for path in (sdpa.PATH_SPLITKV, sdpa.PATH_TC2, sdpa.PATH_TC_DUAL):
+    # the split-KV, two-tile and looping pair kernels do not take them, and
+    # the wide path takes nothing else
+    for path in (sdpa.PATH_SPLITKV, sdpa.PATH_TC_DUAL, sdpa.PATH_TC_KSPLIT, sdpa.PATH_TC2_LOOP):
         with pytest.raises(sdpa.SdpaError) as ei:
             sdpa.plan(1, 4, 4, 64, 64, 512, 512, num_sms=148, force_path=path)
         assert ei.value.status == 2 and "wide" in ei.value.message
-    assert sdpa.plan(1, 4, 4, 64, 64, 512, 512, num_sms=148,
-                     force_path=sdpa.PATH_TC)["path"] == sdpa.PATH_TC
+    for path in (sdpa.PATH_TC, sdpa.PATH_TC2):
+        assert sdpa.plan(1, 4, 4, 64, 64, 512, 512, num_sms=148,
+                         force_path=path)["path"] == path
+    # forced onto the pair kernel it never splits
+    with pytest.raises(sdpa.SdpaError) as ei:
+        sdpa.plan(1, 1, 1, 256, 8192, 512, 512, num_sms=148, force_path=sdpa.PATH_TC2,
+                  force_splits=2)
+    assert ei.value.status == 2
     with pytest.raises(sdpa.SdpaError) as ei:
         sdpa.plan(1, 4, 4, 64, 64, 256, 256, num_sms=148, force_path=sdpa.PATH_WIDE)
     assert ei.value.status == 2

@@ -1,7 +1,8 @@
 """GPU parity at head dims above 256 (up to 512) against the oracle: the wide
-path (the output columns split over four warps per 16-row group) and the
+path (the output columns split over four warps per 16-row group), the
 tcgen05 path in column halves (one CTA per 256-column half of V and O, each
-computing the full scores)."""
+computing the full scores) and the pair kernel in column halves (an SM pair
+per 256-row tile and 256-column half, 64-key blocks)."""
 import numpy as np
 import pytest
 import torch
@@ -82,12 +83,13 @@ def test_wide_splits_agree(cuda_lib):
     assert agree(a, b, "bf16")
 
 
-@pytest.mark.parametrize("path", [S.PATH_WIDE, S.PATH_TC])
+@pytest.mark.parametrize("path", [S.PATH_WIDE, S.PATH_TC, S.PATH_TC2])
 def test_wide_sinks_offset_lse(cuda_lib, path):
     p = I.Problem(1, 4, 2, 40, 700, 512, 512, "bf16", True, 150, None, 54, "wide_ex")
     q, k, v = I.make_qkv(p)
     sinks = [0.25, -2.0, 1.5, 0.0]
-    for fs in (1, 4):
+    # the pair kernel does not split the keys at head dims above 256
+    for fs in ((1,) if path == S.PATH_TC2 else (1, 4)):
         lse = torch.full((1, 4, 40), float("nan"), dtype=torch.float32, device="cuda")
         out = cuda_lib.forward_ex(q.cuda(), k.cuda(), v.cuda(), scale=p.sm_scale, causal=True,
                                   window_size=150, q_offset=500,
@@ -108,5 +110,36 @@ def test_wide_bench_workloads(cuda_lib, idx):
     p = I.wide_problems()[idx]
     rows = I.sample_rows(p.L, 256, seed=p.seed) if p.L > 256 else None
     _, _, info = check_problem(cuda_lib, p, rows=rows)
-    # decode on the wide path; the prefill's rows fill 128-row tcgen05 tiles
-    assert info["path"] == (S.PATH_TC if p.L > 64 else S.PATH_WIDE)
+    # decode on the wide path; the prefill's rows fill 256-row pair tiles
+    assert info["path"] == (S.PATH_TC2 if p.L > 64 else S.PATH_WIDE)
+
+
+PAIR_CASES = [
+    # name, B, Hq, Hkv, L, S, Dqk, Dv, dtype, causal, window
+    ("pair_one_tile", 1, 2, 1, 128, 256, 512, 512, "bf16", True, 0),
+    ("pair_ragged_f16", 1, 2, 2, 300, 333, 512, 512, "f16", False, 0),
+    ("pair_window", 1, 4, 2, 400, 700, 512, 512, "bf16", True, 150),
+    ("pair_window_1", 1, 2, 2, 260, 260, 512, 512, "bf16", True, 1),
+    ("pair_dqk320_dv384", 1, 2, 1, 260, 300, 320, 384, "bf16", True, 0),
+    ("pair_dqk512_dv264", 1, 2, 2, 256, 190, 512, 264, "f16", False, 0),
+    ("pair_many_tiles", 2, 8, 4, 512, 512, 512, 512, "bf16", True, 0),
+    ("pair_l_lt_s", 1, 4, 4, 300, 1000, 512, 512, "bf16", True, 0),
+]
+
+
+@pytest.mark.parametrize("case", PAIR_CASES, ids=[c[0] for c in PAIR_CASES])
+def test_pair_column_halves_vs_oracle(cuda_lib, case):
+    name, B, Hq, Hkv, L, Sk, Dqk, Dv, dt, causal, W = case
+    p = I.Problem(B, Hq, Hkv, L, Sk, Dqk, Dv, dt, causal, W, None, 57, name)
+    _, _, info = check_problem(cuda_lib, p, force_path=S.PATH_TC2)
+    assert info["path"] == S.PATH_TC2 and info["key_block"] == 64 and info["splits"] == 1
+
+
+@pytest.mark.parametrize("case", PAIR_CASES[:4], ids=[c[0] for c in PAIR_CASES[:4]])
+def test_pair_column_halves_agree_with_one_sm(cuda_lib, case):
+    name, B, Hq, Hkv, L, Sk, Dqk, Dv, dt, causal, W = case
+    p = I.Problem(B, Hq, Hkv, L, Sk, Dqk, Dv, dt, causal, W, None, 58, name)
+    q, k, v = I.make_qkv(p)
+    a = run_gpu(cuda_lib, p, q, k, v, force_path=S.PATH_TC2)[0].float()
+    b = run_gpu(cuda_lib, p, q, k, v, force_path=S.PATH_TC, force_splits=1)[0].float()
+    assert agree(a, b, dt)
