@@ -37,8 +37,11 @@
 // two blocks later: the MMA for S_{j+2} is issued after P_j V by the same
 // thread, and one thread's tcgen05 MMAs execute in order.
 //
+// Head dims above 256 run in column halves (grid.y): a launch column loads
+// and writes DV of the output columns, and both compute the full scores.
+//
 // Looping form (PERSIST): a grid of at most one pair per two SMs walks the
-// pair tiles (item = pair index, + pairs launched, ...).  Q has two buffers,
+// pair tiles in rounds (tc2_item).  Q has two buffers,
 // so the next tile's Q load and its first two score MMAs run under the
 // current tile's last blocks and epilogue, and a pair pays the launch,
 // barrier and TMEM set-up once instead of once per tile.  Block and tile
@@ -57,7 +60,6 @@
 #ifndef SDPA_TC2_POLY_OF4
 #define SDPA_TC2_POLY_OF4 1
 #endif
-
 
 namespace sdpa {
 
@@ -240,53 +242,52 @@ __global__ void __launch_bounds__(224, 1)
       for (; ok; ++it) {
         const int item = tc2_item(it, pid, npairs, n_items);
         if (item < 0) break;
-      const Tc2Tile w = tc2_tile<BN, Cfg::kBM>(p, item, rank);
-      const int qb = it % Cfg::kQBufs, use = it / Cfg::kQBufs;
-      // a Q buffer is refilled once the store of the output staged in it
-      // (two tiles back) has read it
-      if (PERSIST && use > 0 &&
-          !mbar_wait(&q_empty[qb], (uint32_t)(use - 1) & 1u, p.wd, kWdTmaEmpty)) {
-        ok = false;
-        break;
-      }
-      const int grow0 = w.bh * p.R + w.tpair.row0 + (int)rank * Cfg::kBM;
-      uint8_t *q_dst = sQ + qb * Cfg::kQBytes;
-
-      mbar_arrive_expect_tx(&q_full[qb], Cfg::kQBytes);
-#pragma unroll
-      for (int bx = 0; bx < Cfg::kQBoxes; ++bx)
-        tma_load_2d(q_dst + bx * (Cfg::kBM * 128), &tm_q, &q_full[qb], bx * 64, grow0);
-      auto emit = [&](bool is_k, int blk) {
-        const int slot = u % NSLOT;
-        if (!mbar_wait_cluster(&slot_empty[slot], ((uint32_t)(u / NSLOT) & 1u) ^ 1u, p.wd,
-                               kWdTmaEmpty)) {
+        const Tc2Tile w = tc2_tile<BN, Cfg::kBM>(p, item, rank);
+        const int qb = it % Cfg::kQBufs, use = it / Cfg::kQBufs;
+        // a Q buffer is refilled once the store of the output staged in it
+        // (two tiles back) has read it
+        if (PERSIST && use > 0 &&
+            !mbar_wait(&q_empty[qb], (uint32_t)(use - 1) & 1u, p.wd, kWdTmaEmpty)) {
           ok = false;
-          return;
+          break;
         }
-        uint8_t *dst = sSlots + slot * Cfg::kSlotBytes;
-        const int k0 = w.k_lo + blk * BN;
-        if (is_k) {
-          mbar_arrive_expect_tx(&slot_full[slot], Cfg::kKBytes);
+        const int grow0 = w.bh * p.R + w.tpair.row0 + (int)rank * Cfg::kBM;
+        uint8_t *q_dst = sQ + qb * Cfg::kQBytes;
+        mbar_arrive_expect_tx(&q_full[qb], Cfg::kQBytes);
 #pragma unroll
-          for (int bx = 0; bx < Cfg::kQBoxes; ++bx)
-            tma_load_3d(dst + bx * ((BN / 2) * 128), &tm_k, &slot_full[slot], bx * 64,
-                        k0 + (int)rank * (BN / 2), w.bh);
-        } else {
-          mbar_arrive_expect_tx(&slot_full[slot], Cfg::kVBytes);
+        for (int bx = 0; bx < Cfg::kQBoxes; ++bx)
+          tma_load_2d(q_dst + bx * (Cfg::kBM * 128), &tm_q, &q_full[qb], bx * 64, grow0);
+        auto emit = [&](bool is_k, int blk) {
+          const int slot = u % NSLOT;
+          if (!mbar_wait_cluster(&slot_empty[slot], ((uint32_t)(u / NSLOT) & 1u) ^ 1u, p.wd,
+                                 kWdTmaEmpty)) {
+            ok = false;
+            return;
+          }
+          uint8_t *dst = sSlots + slot * Cfg::kSlotBytes;
+          const int k0 = w.k_lo + blk * BN;
+          if (is_k) {
+            mbar_arrive_expect_tx(&slot_full[slot], Cfg::kKBytes);
 #pragma unroll
-          for (int bx = 0; bx < Cfg::kVBoxes; ++bx)
-            tma_load_3d(dst + bx * (BN * 128), &tm_v, &slot_full[slot],
-                        dv0 + (int)rank * Cfg::kVHalf + bx * 64, k0, w.bh);
+            for (int bx = 0; bx < Cfg::kQBoxes; ++bx)
+              tma_load_3d(dst + bx * ((BN / 2) * 128), &tm_k, &slot_full[slot], bx * 64,
+                          k0 + (int)rank * (BN / 2), w.bh);
+          } else {
+            mbar_arrive_expect_tx(&slot_full[slot], Cfg::kVBytes);
+#pragma unroll
+            for (int bx = 0; bx < Cfg::kVBoxes; ++bx)
+              tma_load_3d(dst + bx * (BN * 128), &tm_v, &slot_full[slot],
+                          dv0 + (int)rank * Cfg::kVHalf + bx * 64, k0, w.bh);
+          }
+          ++u;
+        };
+        const int nblk = w.nblk;
+        if (nblk > 0) emit(true, 0);
+        if (ok && nblk > 1) emit(true, 1);
+        for (int j = 0; ok && j < nblk; ++j) {
+          emit(false, j);
+          if (ok && j + 2 < nblk) emit(true, j + 2);
         }
-        ++u;
-      };
-      const int nblk = w.nblk;
-      if (nblk > 0) emit(true, 0);
-      if (ok && nblk > 1) emit(true, 1);
-      for (int j = 0; ok && j < nblk; ++j) {
-        emit(false, j);
-        if (ok && j + 2 < nblk) emit(true, j + 2);
-      }
       }
       // nothing may still land at exit: the last load into each Q buffer
       // and into each slot
@@ -444,200 +445,200 @@ __global__ void __launch_bounds__(224, 1)
     for (; ok; ++it) {
       const int item = tc2_item(it, pid, npairs, n_items);
       if (item < 0) break;
-    const Tc2Tile w = tc2_tile<BN, Cfg::kBM>(p, item, rank);
-    const TileRows &tr = w.tr;
-    const int nblk = w.nblk;
-    const int qb = it % Cfg::kQBufs;
-    const int pos = ((tr.row0 + r) % p.L) + p.off;
-    float m_used = -INFINITY, l = 0.f;
-    for (int j = 0; j < nblk; ++j) {
-      const int x = x0 + j;  // block index over the pair's tiles
-      const int b = x & 1;
-      bool wt = true;
-      if (lane == 0) wt = mbar_wait_cluster(&s_full[b], (uint32_t)(x >> 1) & 1u, p.wd, kWdMma);
-      if (!__shfl_sync(0xffffffffu, (int)wt, 0)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      float s[BN];
-#pragma unroll
-      for (int c32 = 0; c32 < BN / 32; ++c32)
-        tmem_ld32(tmem + lane_base + b * BN + c32 * 32, s + c32 * 32);
-      tmem_wait_ld();
-
-      const int kbase = w.k_lo + j * BN;
-      const bool masked = block_needs_mask(p, tr, kbase, BN);
-      // The common block (positive scale, no masked key) takes the plain
-      // reduction; the rare ones (scale 0, masked keys, negative scale) their
-      // own copy, so that their per-element work is not folded into it.
-      float mr[1];
-      if (!masked && c_pos && !c_zero) {
-        mr[0] = row_reduce_max(s);
-      } else {
-        if (c_zero) {
-#pragma unroll
-          for (int i = 0; i < BN; ++i) s[i] = 0.f;
-        }
-        if (masked) {
-          const VisibleRange vis = visible_range(p, pos, kbase);
-#pragma unroll
-          for (int i = 0; i < BN; ++i)
-            if (!vis(i)) s[i] = neutral;
-        }
-        mr[0] = c_pos ? row_reduce_max(s) : row_reduce_min(s);
-      }
-      const float mblk = isinf(mr[0]) ? -INFINITY : mr[0] * c_eff;
-      const float m_new = fmaxf(m_used, mblk);
-      const bool need = m_new > m_used + 8.0f;
-      float alpha = 1.f;
-      if (need) {
-        alpha = fast_exp2(m_used - m_new);
-        m_used = m_new;
-        l *= alpha;
-      }
-      if (j > 0 && __any_sync(0xffffffffu, need)) {
-        // S_x was issued after P_{x-2} V by the same thread, and P_x V waits
-        // for p_full: o_bar is in phase x-1 or x here.  The TMEM loads and
-        // stores are warp-wide, so the whole warp rescales its rows.
-        if (lane == 0) wt = mbar_wait_cluster(o_bar, (uint32_t)(x - 1) & 1u, p.wd, kWdMma);
+      const Tc2Tile w = tc2_tile<BN, Cfg::kBM>(p, item, rank);
+      const TileRows &tr = w.tr;
+      const int nblk = w.nblk;
+      const int qb = it % Cfg::kQBufs;
+      const int pos = ((tr.row0 + r) % p.L) + p.off;
+      float m_used = -INFINITY, l = 0.f;
+      for (int j = 0; j < nblk; ++j) {
+        const int x = x0 + j;  // block index over the pair's tiles
+        const int b = x & 1;
+        bool wt = true;
+        if (lane == 0) wt = mbar_wait_cluster(&s_full[b], (uint32_t)(x >> 1) & 1u, p.wd, kWdMma);
         if (!__shfl_sync(0xffffffffu, (int)wt, 0)) {
           ok = false;
           break;
         }
         tc_fence_after();
-#pragma unroll 1
-        for (int c16 = 0; c16 < DV / 16; ++c16) {
-          float o[16];
-          tmem_ld16(tmem + lane_base + Cfg::kOCol + c16 * 16, o);
-          tmem_wait_ld();
+        float s[BN];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) o[e] *= alpha;
-          tmem_st16(tmem + lane_base + Cfg::kOCol + c16 * 16, o);
-        }
-      }
-      // ---- P = exp2(s c - m), row sum, P packed over the row's own scores ----
-      const float mref = m_used == -INFINITY ? 0.f : m_used;
-      const float2 c2 = make_float2(c_eff, c_eff), nm2 = make_float2(-mref, -mref);
-      float2 acc[4];
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) acc[q4] = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int c32 = 0; c32 < BN / 32; ++c32) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int i2 = 0; i2 < 16; ++i2) {
-          const int i = c32 * 32 + 2 * i2;
-          float2 t = fma2(make_float2(s[i], s[i + 1]), c2, nm2);
-          if ((i2 & 3) < SDPA_TC2_POLY_OF4) {
-            t = exp2_poly2(t);  // FMA / ALU pipes
-          } else {
-            t.x = fast_exp2(t.x);  // MUFU
-            t.y = fast_exp2(t.y);
-          }
-          acc[i2 & 3] = add2(acc[i2 & 3], t);
-          pk[i2] = pack2<kBF16>(t.x, t.y);
-        }
-        tmem_st_u16x(tmem + lane_base + b * BN + c32 * 16, pk);
-      }
-      const float2 a01 = add2(acc[0], acc[1]), a23 = add2(acc[2], acc[3]);
-      const float2 at = add2(a01, a23);
-      l += at.x + at.y;
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(leader ? &p_full[b] : &p_local[b]);
-      // the previous tile's store has long read its buffer by now
-      if (j == 0) release_q();
-    }
-
-    // ------------------------------ epilogue ------------------------------
-    if (ok && nblk > 0) {
-      bool wt = true;
-      if (lane == 0) wt = mbar_wait_cluster(o_final, (uint32_t)nfin & 1u, p.wd, kWdMma);
-      ok = __shfl_sync(0xffffffffu, (int)wt, 0) != 0;
-      tc_fence_after();
-    }
-    if (nblk > 0) ++nfin;
-    release_q();  // a tile without blocks released nothing above
-    const bool valid = r < tr.nvalid;
-    const long grow = (long)w.bh * p.R + tr.row0 + r;
-    const bool have_o = ok && nblk > 0;
-    // O leaves TMEM kOGroup chunks of 16 columns per wait
-    constexpr int kOChunks = DV / 16;
-    constexpr int kOGroup = kOChunks <= 5 ? kOChunks : 4;
-    static_assert(kOChunks % kOGroup == 0, "whole groups of O chunks");
-    auto load_o = [&](int g, float (&o)[kOGroup][16]) {
-      if (have_o) {
-    #pragma unroll
-        for (int k = 0; k < kOGroup; ++k)
-          tmem_ld16(tmem + lane_base + Cfg::kOCol + (g * kOGroup + k) * 16, o[k]);
+        for (int c32 = 0; c32 < BN / 32; ++c32)
+          tmem_ld32(tmem + lane_base + b * BN + c32 * 32, s + c32 * 32);
         tmem_wait_ld();
-      } else {
-    #pragma unroll
-        for (int k = 0; k < kOGroup; ++k)
-    #pragma unroll
-          for (int e = 0; e < 16; ++e) o[k][e] = 0.f;
-      }
-    };
-    // Output rows are staged in the TMA store's swizzled box layout, in this
-    // CTA's K/V slots (free: o_final fired once every MMA of the pair had
-    // completed) or, looping, in this tile's Q buffer (free for the same
-    // reason), then one thread stores them in boxes of 128 rows; rows past
-    // the slab and columns past Dv are clipped by the tensor map.
-    uint8_t *stage = PERSIST ? sQ + qb * Cfg::kQBytes : sSlots;
-    if (!split_out) {
-      const float inv = finish_row(p, grow, m_used, l);  // folds in the sink, if any
-      if (p.lse_out != nullptr && valid && dv0 == 0) p.lse_out[grow] = row_lse(m_used, l);
+
+        const int kbase = w.k_lo + j * BN;
+        const bool masked = block_needs_mask(p, tr, kbase, BN);
+        // The common block (positive scale, no masked key) takes the plain
+        // reduction; the rare ones (scale 0, masked keys, negative scale) their
+        // own copy, so that their per-element work is not folded into it.
+        float mr[1];
+        if (!masked && c_pos && !c_zero) {
+          mr[0] = row_reduce_max(s);
+        } else {
+          if (c_zero) {
+#pragma unroll
+            for (int i = 0; i < BN; ++i) s[i] = 0.f;
+          }
+          if (masked) {
+            const VisibleRange vis = visible_range(p, pos, kbase);
+#pragma unroll
+            for (int i = 0; i < BN; ++i)
+              if (!vis(i)) s[i] = neutral;
+          }
+          mr[0] = c_pos ? row_reduce_max(s) : row_reduce_min(s);
+        }
+        const float mblk = isinf(mr[0]) ? -INFINITY : mr[0] * c_eff;
+        const float m_new = fmaxf(m_used, mblk);
+        const bool need = m_new > m_used + 8.0f;
+        float alpha = 1.f;
+        if (need) {
+          alpha = fast_exp2(m_used - m_new);
+          m_used = m_new;
+          l *= alpha;
+        }
+        if (j > 0 && __any_sync(0xffffffffu, need)) {
+          // S_x was issued after P_{x-2} V by the same thread, and P_x V waits
+          // for p_full: o_bar is in phase x-1 or x here.  The TMEM loads and
+          // stores are warp-wide, so the whole warp rescales its rows.
+          if (lane == 0) wt = mbar_wait_cluster(o_bar, (uint32_t)(x - 1) & 1u, p.wd, kWdMma);
+          if (!__shfl_sync(0xffffffffu, (int)wt, 0)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
 #pragma unroll 1
-      for (int g = 0; g < kOChunks / kOGroup; ++g) {
-        float o[kOGroup][16];
-        load_o(g, o);
+          for (int c16 = 0; c16 < DV / 16; ++c16) {
+            float o[16];
+            tmem_ld16(tmem + lane_base + Cfg::kOCol + c16 * 16, o);
+            tmem_wait_ld();
 #pragma unroll
-        for (int k = 0; k < kOGroup; ++k) {
-          uint32_t w8[8];
+            for (int e = 0; e < 16; ++e) o[e] *= alpha;
+            tmem_st16(tmem + lane_base + Cfg::kOCol + c16 * 16, o);
+          }
+        }
+        // ---- P = exp2(s c - m), row sum, P packed over the row's own scores ----
+        const float mref = m_used == -INFINITY ? 0.f : m_used;
+        const float2 c2 = make_float2(c_eff, c_eff), nm2 = make_float2(-mref, -mref);
+        float2 acc[4];
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            w8[e] = pack2<kBF16>(o[k][2 * e] * inv, o[k][2 * e + 1] * inv);
-          stage_16bit_x16(stage, r, g * kOGroup + k, w8);
+        for (int q4 = 0; q4 < 4; ++q4) acc[q4] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int c32 = 0; c32 < BN / 32; ++c32) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i2 = 0; i2 < 16; ++i2) {
+            const int i = c32 * 32 + 2 * i2;
+            float2 t = fma2(make_float2(s[i], s[i + 1]), c2, nm2);
+            if ((i2 & 3) < SDPA_TC2_POLY_OF4) {
+              t = exp2_poly2(t);  // FMA / ALU pipes
+            } else {
+              t.x = fast_exp2(t.x);  // MUFU
+              t.y = fast_exp2(t.y);
+            }
+            acc[i2 & 3] = add2(acc[i2 & 3], t);
+            pk[i2] = pack2<kBF16>(t.x, t.y);
+          }
+          tmem_st_u16x(tmem + lane_base + b * BN + c32 * 16, pk);
+        }
+        const float2 a01 = add2(acc[0], acc[1]), a23 = add2(acc[2], acc[3]);
+        const float2 at = add2(a01, a23);
+        l += at.x + at.y;
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(leader ? &p_full[b] : &p_local[b]);
+        // the previous tile's store has long read its buffer by now
+        if (j == 0) release_q();
+      }
+
+      // ------------------------------ epilogue ------------------------------
+      if (ok && nblk > 0) {
+        bool wt = true;
+        if (lane == 0) wt = mbar_wait_cluster(o_final, (uint32_t)nfin & 1u, p.wd, kWdMma);
+        ok = __shfl_sync(0xffffffffu, (int)wt, 0) != 0;
+        tc_fence_after();
+      }
+      if (nblk > 0) ++nfin;
+      release_q();  // a tile without blocks released nothing above
+      const bool valid = r < tr.nvalid;
+      const long grow = (long)w.bh * p.R + tr.row0 + r;
+      const bool have_o = ok && nblk > 0;
+      // O leaves TMEM kOGroup chunks of 16 columns per wait
+      constexpr int kOChunks = DV / 16;
+      constexpr int kOGroup = kOChunks <= 5 ? kOChunks : 4;
+      static_assert(kOChunks % kOGroup == 0, "whole groups of O chunks");
+      auto load_o = [&](int g, float (&o)[kOGroup][16]) {
+        if (have_o) {
+    #pragma unroll
+          for (int k = 0; k < kOGroup; ++k)
+            tmem_ld16(tmem + lane_base + Cfg::kOCol + (g * kOGroup + k) * 16, o[k]);
+          tmem_wait_ld();
+        } else {
+    #pragma unroll
+          for (int k = 0; k < kOGroup; ++k)
+    #pragma unroll
+            for (int e = 0; e < 16; ++e) o[k][e] = 0.f;
+        }
+      };
+      // Output rows are staged in the TMA store's swizzled box layout, in this
+      // CTA's K/V slots (free: o_final fired once every MMA of the pair had
+      // completed) or, looping, in this tile's Q buffer (free for the same
+      // reason), then one thread stores them in boxes of 128 rows; rows past
+      // the slab and columns past Dv are clipped by the tensor map.
+      uint8_t *stage = PERSIST ? sQ + qb * Cfg::kQBytes : sSlots;
+      if (!split_out) {
+        const float inv = finish_row(p, grow, m_used, l);  // folds in the sink, if any
+        if (p.lse_out != nullptr && valid && dv0 == 0) p.lse_out[grow] = row_lse(m_used, l);
+#pragma unroll 1
+        for (int g = 0; g < kOChunks / kOGroup; ++g) {
+          float o[kOGroup][16];
+          load_o(g, o);
+#pragma unroll
+          for (int k = 0; k < kOGroup; ++k) {
+            uint32_t w8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              w8[e] = pack2<kBF16>(o[k][2 * e] * inv, o[k][2 * e + 1] * inv);
+            stage_16bit_x16(stage, r, g * kOGroup + k, w8);
+          }
+        }
+      } else if constexpr (Cfg::kSplitStage) {
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        if (valid && dv0 == 0)
+          p.part_lse[(long)w.split * total_rows + grow] = have_o ? row_lse(m_used, l) : -INFINITY;
+#pragma unroll 1
+        for (int g = 0; g < kOChunks / kOGroup; ++g) {
+          float o[kOGroup][16];
+          load_o(g, o);
+#pragma unroll
+          for (int k = 0; k < kOGroup; ++k)
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4)
+              stage_f32_x4(stage, r, (g * kOGroup + k) * 4 + q4, o[k][q4 * 4] * inv,
+                           o[k][q4 * 4 + 1] * inv, o[k][q4 * 4 + 2] * inv, o[k][q4 * 4 + 3] * inv);
         }
       }
-    } else if constexpr (Cfg::kSplitStage) {
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      if (valid && dv0 == 0)
-        p.part_lse[(long)w.split * total_rows + grow] = have_o ? row_lse(m_used, l) : -INFINITY;
-#pragma unroll 1
-      for (int g = 0; g < kOChunks / kOGroup; ++g) {
-        float o[kOGroup][16];
-        load_o(g, o);
-#pragma unroll
-        for (int k = 0; k < kOGroup; ++k)
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4)
-            stage_f32_x4(stage, r, (g * kOGroup + k) * 4 + q4, o[k][q4 * 4] * inv,
-                         o[k][q4 * 4 + 1] * inv, o[k][q4 * 4 + 2] * inv, o[k][q4 * 4 + 3] * inv);
-      }
-    }
-    fence_proxy_async_smem();
-    asm volatile("bar.sync 1, 128;" ::: "memory");  // the four softmax warps
-    if (warp == 0 && lane == 0) {
-      if (tr.nvalid > 0) {
-        if (!split_out) {
-          for (int bx = 0; bx < Cfg::kOutBoxes && dv0 + bx * 64 < p.Dv; ++bx)
-            tma_store_3d(&tm_o, stage + bx * (Cfg::kBM * 128), dv0 + bx * 64, tr.row0, w.bh);
-        } else if constexpr (Cfg::kSplitStage) {
-          for (int bx = 0; bx < Cfg::kF32Boxes && dv0 + bx * 32 < p.Dv; ++bx)
-            tma_store_3d(&tm_p, stage + bx * (Cfg::kBM * 128), dv0 + bx * 32, tr.row0,
-                         w.split * BH + w.bh);
+      fence_proxy_async_smem();
+      asm volatile("bar.sync 1, 128;" ::: "memory");  // the four softmax warps
+      if (warp == 0 && lane == 0) {
+        if (tr.nvalid > 0) {
+          if (!split_out) {
+            for (int bx = 0; bx < Cfg::kOutBoxes && dv0 + bx * 64 < p.Dv; ++bx)
+              tma_store_3d(&tm_o, stage + bx * (Cfg::kBM * 128), dv0 + bx * 64, tr.row0, w.bh);
+          } else if constexpr (Cfg::kSplitStage) {
+            for (int bx = 0; bx < Cfg::kF32Boxes && dv0 + bx * 32 < p.Dv; ++bx)
+              tma_store_3d(&tm_p, stage + bx * (Cfg::kBM * 128), dv0 + bx * 32, tr.row0,
+                           w.split * BH + w.bh);
+          }
+          bulk_commit_group();
         }
-        bulk_commit_group();
+        if (PERSIST)
+          pend_q = qb;  // handed back once read, under the next tile's first block
+        else
+          bulk_wait_group0();
       }
-      if (PERSIST)
-        pend_q = qb;  // handed back once read, under the next tile's first block
-      else
-        bulk_wait_group0();
-    }
-    x0 += nblk;
+      x0 += nblk;
     }
     // every store has completed before the CTA leaves
     if (warp == 0 && lane == 0) bulk_wait_group0();
