@@ -16,7 +16,7 @@ sdpa_status run_tc_pp(const Launch &ln, std::string *err) {
   constexpr uint32_t kV = ((DV + 63) / 64) * kBN * 128;
   constexpr uint32_t kSlot = kK > kV ? kK : kV;
   constexpr uint32_t kBudget =
-      232448u - (2u * 8u + 10u) * 8u - 16u - (kKSplit ? 2u * 128u * 8u : 0u);
+      232448u - (2u * 8u + 14u) * 8u - 16u - (kKSplit ? 2u * 128u * 8u : 0u);
   constexpr int kFit = (int)((kBudget - kQ) / kSlot);
   constexpr int kNSlot = kFit > 8 ? 8 : kFit;
   static_assert(kNSlot >= 2, "at least two K/V slots");

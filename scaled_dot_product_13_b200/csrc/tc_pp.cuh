@@ -50,6 +50,14 @@
 // thread's MMAs run in issue order.  For the same reason, once S_t(j) is
 // complete, P_t(j-1) V is complete too, so the softmax may rescale O_t in
 // tensor memory without waiting for anything else.
+//
+// Separate P (row pairs, BN + BN/2 + DV <= 256, i.e. head dims <= 64): P has
+// its own columns [256 t + BN, 256 t + 3 BN/2) and O follows it.  The tile's
+// softmax signals s_free once it has loaded S_t(j), and the next scores
+// S_t(j+1) are issued then, ahead of P_t(j) V, so they compute during the
+// softmax instead of after it: MMA order S_A(j+1), P_A(j) V, S_B(j+1),
+// P_B(j) V.  P_t(j) V now completes after S_t(j+1), so the softmax of block
+// j+1 waits for it (pv_done) before it rescales O_t or writes P_t(j+1).
 #pragma once
 
 #include "params.cuh"
@@ -73,7 +81,7 @@ struct PpCfg {
   static constexpr uint32_t kXOff = kSlotOff + NSLOT * kSlotBytes;
   static constexpr uint32_t kXBytes = KSPLIT ? 2 * kBM * 8 : 0;
   static constexpr uint32_t kBarOff = kXOff + kXBytes;
-  static constexpr int kNumBars = 2 * NSLOT + 10;
+  static constexpr int kNumBars = 2 * NSLOT + 14;
   static constexpr uint32_t kSmemBytes = kBarOff + kNumBars * 8 + 16;
   static constexpr int kThreads = 320;
   static constexpr uint32_t kTmemCols = 512;
@@ -82,6 +90,10 @@ struct PpCfg {
   static_assert(DQK % 16 == 0 && DV % 16 == 0 && DV >= 16, "head dims");
   static_assert(BN == 128, "key block");
   static_assert(BN + DV <= kTileCols, "TMEM columns per tile");
+  // P in its own columns (see above) where the tile's TMEM has room for it
+  static constexpr bool kSepP = !KSPLIT && BN + BN / 2 + DV <= kTileCols;
+  static constexpr int kPCol = kSepP ? BN : 0;           // P within the tile's columns
+  static constexpr int kOCol = kSepP ? BN + BN / 2 : BN;  // O within the tile's columns
   static_assert(kSmemBytes <= 232448, "shared memory");
   // the epilogue stages each tile's output rows in the K/V slots: 64 columns
   // of a 16-bit type, or 32 fp32 split partials, per 16 KB box
@@ -115,7 +127,9 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t *p_full = s_full + 2;              // [2] P_t(j) in TMEM (4 warps each)
   uint64_t *o_final = p_full + 2;             // [2] every P_t V complete
   uint64_t *fin_bar = o_final + 2;            // all MMAs complete (teardown)
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(fin_bar + 1);
+  uint64_t *s_free = fin_bar + 1;             // [2] separate P: S_t(j) loaded (4 warps each)
+  uint64_t *pv_done = s_free + 2;             // [2] separate P: P_t(j) V complete
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(pv_done + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -143,6 +157,8 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&s_full[t], 1);
       mbar_init(&p_full[t], 4);
       mbar_init(&o_final[t], 1);
+      mbar_init(&s_free[t], 4);
+      mbar_init(&pv_done[t], 1);
     }
     mbar_init(fin_bar, 1);
     fence_barrier_init();
@@ -283,9 +299,11 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
         for (int ks = 0; ks < Cfg::kPVK; ++ks) {
           const uint64_t bd = umma_desc_advance(v0, ks * 2048);
-          tc_mma_ts(tmem + t * Cfg::kTileCols + BN, tmem + t * Cfg::kTileCols + ks * 8, bd,
-                    kIdescPV, (j > 0 || ks > 0) ? 1u : 0u);
+          tc_mma_ts(tmem + t * Cfg::kTileCols + Cfg::kOCol,
+                    tmem + t * Cfg::kTileCols + Cfg::kPCol + ks * 8, bd, kIdescPV,
+                    (j > 0 || ks > 0) ? 1u : 0u);
         }
+        if constexpr (Cfg::kSepP) tc_commit(&pv_done[t]);
       };
       auto wait_p = [&](int t, int j) -> bool {
         if (!mbar_wait(&p_full[t], (uint32_t)j & 1u, p.wd, kWdSoftmax)) return false;
@@ -345,6 +363,44 @@ __global__ void __launch_bounds__(320, 1)
             s_into(t, slot);
           }
         }
+      } else if constexpr (Cfg::kSepP) {
+        if (ok && nblk > 0) {
+          ok = wait_load(0);
+          if (ok) {
+            tc_fence_after();
+            issue_s(0, 0);
+            issue_s(1, 0);
+            tc_commit(&slot_empty[slot_of(0)]);
+          }
+        }
+        auto wait_s_free = [&](int t, int j) -> bool {
+          if (!mbar_wait(&s_free[t], (uint32_t)j & 1u, p.wd, kWdSoftmax)) return false;
+          tc_fence_after();
+          return true;
+        };
+        for (int j = 0; ok && j < nblk; ++j) {
+          const bool more = j + 1 < nblk;
+          // tile A: S_A(j+1) once its softmax has loaded S_A(j), then P_A(j) V
+          if (more) {
+            ok = wait_load(2 * j + 2) && wait_s_free(0, j);
+            if (!ok) break;
+            issue_s(0, j + 1);
+          }
+          ok = wait_load(2 * j + 1) && wait_p(0, j);
+          if (!ok) break;
+          issue_pv(0, j);
+          // tile B the same; each slot's second use frees it
+          if (more) {
+            ok = wait_s_free(1, j);
+            if (!ok) break;
+            issue_s(1, j + 1);
+            tc_commit(&slot_empty[slot_of(2 * j + 2)]);
+          }
+          ok = wait_p(1, j);
+          if (!ok) break;
+          issue_pv(1, j);
+          tc_commit(&slot_empty[slot_of(2 * j + 1)]);
+        }
       } else {
         if (ok && nblk > 0) {
           ok = wait_load(0);
@@ -392,7 +448,8 @@ __global__ void __launch_bounds__(320, 1)
     const int r = quarter * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const uint32_t s_col = (uint32_t)(t * Cfg::kTileCols);
-    const uint32_t o_col = s_col + BN;
+    const uint32_t p_col = s_col + Cfg::kPCol;
+    const uint32_t o_col = s_col + Cfg::kOCol;
     TileRows tr = KSPLIT ? tpair : tile_rows(p, pair_tile * 2 + t, Cfg::kBM);
     if (tr.nvalid <= 0) {  // past the slab: compute on zeros, store nothing
       tr.nvalid = 0;
@@ -426,6 +483,12 @@ __global__ void __launch_bounds__(320, 1)
       for (int c32 = 0; c32 < BN / 32; ++c32)
         tmem_ld32(tmem + lane_base + s_col + c32 * 32, s + c32 * 32);
       tmem_wait_ld();
+      if constexpr (Cfg::kSepP) {
+        // S_t(j) is in registers: the next scores may overwrite it
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_free[t]);
+      }
 
       const int kbase = k_lo + (KSPLIT ? 2 * j + t : j) * BN;
       const bool masked = block_needs_mask(p, tr, kbase, BN);
@@ -460,7 +523,19 @@ __global__ void __launch_bounds__(320, 1)
       // The TMEM loads and stores are warp-wide (.sync.aligned): the rescale
       // runs for the whole warp when any of its rows moved its max.  O_t holds
       // P_t(0..j-1) V and is stable: S_t(j) was issued after P_t(j-1) V by the
-      // same thread and has completed.
+      // same thread and has completed; with separate P, P_t(j-1) V is waited
+      // for here (it also frees the P columns for P_t(j)).
+      if constexpr (Cfg::kSepP) {
+        if (j > 0) {
+          bool w = true;
+          if (lane == 0) w = mbar_wait(&pv_done[t], (uint32_t)(j - 1) & 1u, p.wd, kWdMma);
+          if (!__shfl_sync(0xffffffffu, (int)w, 0)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+      }
       if (j > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll 1
         for (int c16 = 0; c16 < DV / 16; ++c16) {
@@ -490,7 +565,7 @@ __global__ void __launch_bounds__(320, 1)
           acc[i2 & 3] = add2(acc[i2 & 3], e2);
           pk[i2] = pack2<kBF16>(e2.x, e2.y);
         }
-        tmem_st_u16x(tmem + lane_base + s_col + c32 * 16, pk);
+        tmem_st_u16x(tmem + lane_base + p_col + c32 * 16, pk);
       }
       const float2 a01 = add2(acc[0], acc[1]), a23 = add2(acc[2], acc[3]);
       const float2 at = add2(a01, a23);
