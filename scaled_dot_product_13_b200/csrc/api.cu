@@ -268,11 +268,11 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
   if (path == SDPA_PATH_TC_DUAL) {
     pl.wr = 0; pl.wk = 0;
     pl.row_tile = 2 * kTcRows;
-    pl.key_block = 128;
+    pl.key_block = tc_pp_key_block(pl.pair, false);
   } else if (path == SDPA_PATH_TC_KSPLIT) {
     pl.wr = 0; pl.wk = 0;
     pl.row_tile = kTcRows;
-    pl.key_block = 128;
+    pl.key_block = tc_pp_key_block(pl.pair, true);
   } else if (path == SDPA_PATH_WIDE) {
     // one 16-row group (four warps) for decode-sized problems, two otherwise
     pl.wr = pl.rows <= 16 ? 1 : 2;

@@ -177,6 +177,10 @@ sdpa_status launch_tc_pp(const Launch &ln, std::string *err);
 
 // Head-dim pairs the two-tile kernel is built for (index into kDimPairs).
 constexpr bool tc_dual_supports_pair(int pair) { return pair <= 2; }
+// Key block of the two-tile kernel: 96 keys for row pairs at head dims 80
+// (score, P and O columns of a tile then fit its 256 TMEM columns apart),
+// 128 otherwise.
+constexpr int tc_pp_key_block(int pair, bool key_split) { return (!key_split && pair == 1) ? 96 : 128; }
 
 // Head-dim pairs the two-CTA kernel is built for (index into kDimPairs), and
 // those the router sends to it by itself (where it measured faster than one

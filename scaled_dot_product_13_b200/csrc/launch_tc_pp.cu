@@ -10,7 +10,12 @@ namespace {
 
 template <bool kBF16, int DQK, int DV, bool kKSplit>
 sdpa_status run_tc_pp(const Launch &ln, std::string *err) {
-  constexpr int kBN = 128;
+  constexpr int kPair = DQK == 64 ? 0 : DQK == 80 ? 1 : 2;
+  constexpr int kBN = tc_pp_key_block(kPair, kKSplit);
+  if (ln.plan.key_block != kBN) {
+    *err = "internal: the plan's key block does not match the two-tile instance";
+    return SDPA_ERR_UNSUPPORTED;
+  }
   constexpr uint32_t kQ = (kKSplit ? 1u : 2u) * ((DQK + 63) / 64) * 128 * 128;
   constexpr uint32_t kK = ((DQK + 63) / 64) * kBN * 128;
   constexpr uint32_t kV = ((DV + 63) / 64) * kBN * 128;

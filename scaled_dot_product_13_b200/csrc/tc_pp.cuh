@@ -88,7 +88,7 @@ struct PpCfg {
   static constexpr int kTileCols = 256;  // TMEM columns per tile
   static constexpr int kPrefetch = 4;    // K/V blocks prefetched into L2 ahead of the loads
   static_assert(DQK % 16 == 0 && DV % 16 == 0 && DV >= 16, "head dims");
-  static_assert(BN == 128, "key block");
+  static_assert(BN == 128 || (BN == 96 && !KSPLIT), "key block");
   static_assert(BN + DV <= kTileCols, "TMEM columns per tile");
   // P in its own columns (see above) where the tile's TMEM has room for it
   static constexpr bool kSepP = !KSPLIT && BN + BN / 2 + DV <= kTileCols;

@@ -19,6 +19,8 @@ CASES = [
     ("d64_half_pair", 1, 1, 1, 130, 300, 64, 64, "bf16", True, 0),
     ("d72_ragged", 1, 3, 3, 333, 371, 72, 72, "bf16", False, 0),
     ("d80_f16_causal_gqa", 2, 8, 2, 200, 260, 80, 80, "f16", True, 0),
+    ("d72_window", 1, 4, 2, 500, 500, 72, 72, "bf16", True, 100),
+    ("d72_causal_long", 1, 2, 2, 1000, 2000, 72, 72, "bf16", True, 0),
     ("d128_window", 1, 4, 2, 700, 700, 128, 128, "bf16", True, 150),
     ("d128_window_1", 1, 2, 1, 300, 300, 128, 128, "f16", True, 1),
     ("d128_l_lt_s", 1, 4, 4, 257, 1000, 128, 128, "bf16", True, 0),
