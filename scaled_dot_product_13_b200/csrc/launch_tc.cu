@@ -71,11 +71,21 @@ sdpa_status run_tc(const Launch &ln, std::string *err) {
   p.wd.word = ln.wd_word;
   p.wd.limit_ns = ln.wd_limit_ns;
   if (ln.ev_start) record_event(ln.ev_start, ln.stream);
-  // head dims above 256: one CTA per half of V and O (grid.y)
-  const dim3 grid((unsigned)(pl.ctas / pl.col_halves), (unsigned)pl.col_halves);
-  kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, ln.stream>>>(tq, tk, tv, to, tp, p);
+  // head dims above 256: one CTA per half of V and O (grid.y); programmatic
+  // stream serialization: the set-up overlaps the previous grid's tail
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(pl.ctas / pl.col_halves), (unsigned)pl.col_halves);
+  cfg.blockDim = dim3(Cfg::kThreads);
+  cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+  cfg.stream = ln.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, to, tp, p);
   if (ln.ev_stop) record_event(ln.ev_stop, ln.stream);
-  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) {
     *err = std::string("tc_attn_kernel launch failed: ") + cudaGetErrorString(e);
     return SDPA_ERR_CUDA;

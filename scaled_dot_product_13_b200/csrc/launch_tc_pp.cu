@@ -72,9 +72,21 @@ sdpa_status run_tc_pp(const Launch &ln, std::string *err) {
   p.wd.word = ln.wd_word;
   p.wd.limit_ns = ln.wd_limit_ns;
   if (ln.ev_start) record_event(ln.ev_start, ln.stream);
-  kern<<<(unsigned)pl.ctas, Cfg::kThreads, Cfg::kSmemBytes, ln.stream>>>(tq, tk, tv, to, tp, p);
+  // programmatic stream serialization: the set-up overlaps the previous
+  // grid's tail
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)pl.ctas);
+  cfg.blockDim = dim3(Cfg::kThreads);
+  cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+  cfg.stream = ln.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, to, tp, p);
   if (ln.ev_stop) record_event(ln.ev_stop, ln.stream);
-  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) {
     *err = std::string("tc_pp_attn_kernel launch failed: ") + cudaGetErrorString(e);
     return SDPA_ERR_CUDA;

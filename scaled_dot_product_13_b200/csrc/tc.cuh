@@ -179,6 +179,10 @@ __global__ void __launch_bounds__(TcCfg<DQK, DV, BN, NSLOT>::kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   // Let a dependent combine launch now (it waits for this grid to finish).
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // Launched as a programmatic dependent of the previous grid on the stream:
+  // the set-up above ran under that grid's tail; nothing below touches
+  // global memory before that grid has completed.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (warp == Cfg::kProducerWarp) {
     // ============================ TMA producer ============================

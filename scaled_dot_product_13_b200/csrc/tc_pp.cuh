@@ -172,6 +172,10 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // Launched as a programmatic dependent of the previous grid on the stream:
+  // the set-up above ran under that grid's tail; nothing below touches
+  // global memory before that grid has completed.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (warp == 8) {
     // ============================ TMA producer ============================
