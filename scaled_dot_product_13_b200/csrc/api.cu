@@ -238,11 +238,12 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
     // wide heads with at least one full 256-row pair tile: two SMs per tile
     if (path == SDPA_PATH_TC && tc2_preferred_pair(pl.pair) && pl.rows >= kTc2RowThreshold)
       path = SDPA_PATH_TC2;
-    // head dims <= 128: two 128-row tiles per CTA, when the 256-row tiles
-    // alone occupy at least half of the SMs (fewer would rather take the
-    // one-tile kernel's twice as many CTAs) and no window trims the tiles'
-    // key ranges differently (the pair walks the union of both ranges)
-    if (path == SDPA_PATH_TC && tc_dual_supports_pair(pl.pair) && pb.window == 0 &&
+    // head dims <= 80 (where P has TMEM columns of its own): two 128-row
+    // tiles per CTA, when the 256-row tiles alone occupy at least half of the
+    // SMs (fewer would rather take the one-tile kernel's twice as many CTAs)
+    // and no window trims the tiles' key ranges differently (the pair walks
+    // the union of both ranges)
+    if (path == SDPA_PATH_TC && tc_dual_preferred_pair(pl.pair) && pb.window == 0 &&
         pl.rows >= kTc2RowThreshold &&
         (long long)pb.B * pb.Hkv * ((pl.rows + 255) / 256) * 2 >= num_sms)
       path = SDPA_PATH_TC_DUAL;

@@ -177,6 +177,9 @@ sdpa_status launch_tc_pp(const Launch &ln, std::string *err);
 
 // Head-dim pairs the two-tile kernel is built for (index into kDimPairs).
 constexpr bool tc_dual_supports_pair(int pair) { return pair <= 2; }
+// ... and those the router sends to it by itself: at head dims 128 the
+// one-tile kernel measured faster (P shares the scores' columns there)
+constexpr bool tc_dual_preferred_pair(int pair) { return pair <= 1; }
 // Key block of the two-tile kernel: 96 keys for row pairs at head dims 80
 // (score, P and O columns of a tile then fit its 256 TMEM columns apart),
 // 128 otherwise.

@@ -218,6 +218,10 @@ def test_plan_two_tile_path_for_small_head_dims():
     # too few 256-row tiles to fill half the SMs: one tile per CTA
     info = sdpa.plan(1, 16, 16, 1024, 1024, 72, 72, causal=False, num_sms=148)
     assert info["path"] == sdpa.PATH_TC
+    # head dims 128: the one-tile kernel (P shares the scores' TMEM columns in
+    # the two-tile kernel there, and it measured slower)
+    info = sdpa.plan(1, 16, 16, 4096, 4096, 128, 128, causal=False, num_sms=148)
+    assert info["path"] == sdpa.PATH_TC
     # a window trims the two tiles' key ranges differently: one tile per CTA
     info = sdpa.plan(1, 16, 8, 4096, 4096, 128, 128, causal=True, window_size=1024, num_sms=148)
     assert info["path"] == sdpa.PATH_TC
