@@ -50,7 +50,7 @@
 #define SDPA_TC_PARTS 1
 #endif
 #ifndef SDPA_TC_POLY_OF4
-#define SDPA_TC_POLY_OF4 1
+#define SDPA_TC_POLY_OF4 0
 #endif
 // blocks prefetched into L2 beyond the one being loaded
 #ifndef SDPA_TC_PREFETCH
