@@ -169,8 +169,12 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 constexpr int kMaxSplits = 4096;
 
 // Packed rows per (batch, KV head) from which the tcgen05 path is taken:
-// above four 16-row warp tiles, one 128-row tensor-memory tile costs less.
-constexpr int kTcRowThreshold = 65;
+// above two 16-row warp tiles, one 128-row tensor-memory tile costs less
+// (measured on the verify sweep: 48 and 64 rows faster there, 32 slower).
+constexpr int kTcRowThreshold = 33;
+// ... and, at head dims above 256, from which it takes over from the
+// column-split warp-tile kernel.
+constexpr int kTcRowThresholdWide = 65;
 // ... and from which head dims 256/256 and 192/128 take the two-CTA kernel.
 constexpr int kTc2RowThreshold = 256;
 
@@ -228,7 +232,7 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
   // from one 256-row tile, and with at least one pair's work per two SMs
   // (that kernel does not split the keys), an SM pair per tile
   if (path == SDPA_PATH_AUTO && wide) {
-    path = pl.rows >= kTcRowThreshold ? SDPA_PATH_TC : SDPA_PATH_WIDE;
+    path = pl.rows >= kTcRowThresholdWide ? SDPA_PATH_TC : SDPA_PATH_WIDE;
     const long long pair_units = (long long)pb.B * pb.Hkv * ((pl.rows + 255) / 256) *
                                  ((pb.Dv + kTc2WideHalf - 1) / kTc2WideHalf);
     if (pl.rows >= kTc2RowThreshold && 2 * pair_units >= num_sms) path = SDPA_PATH_TC2;

@@ -22,8 +22,8 @@
 //              in the order the MMA consumes them (K0, K1, K2, then V_j,
 //              K_{j+3} for j = 0, 1, ...) through a FIFO ring of NSLOT
 //              shared-memory slots (128-byte swizzle, zero fill past S and
-//              past the head dim), and L2 prefetches of the blocks further
-//              ahead.
+//              past the head dim).  No L2 prefetch ahead of the loads: it
+//              measured slower (the TMA unit serves prefetches before loads).
 //   MMA        (the last warp) allocates TMEM and issues tcgen05.mma from
 //              one thread: S_j = Q K_j^T (A = Q from shared memory) into
 //              score buffer j % 3, and O += P_j V_j with A = P_j read from
@@ -51,10 +51,6 @@
 #endif
 #ifndef SDPA_TC_POLY_OF4
 #define SDPA_TC_POLY_OF4 0
-#endif
-// blocks prefetched into L2 beyond the one being loaded
-#ifndef SDPA_TC_PREFETCH
-#define SDPA_TC_PREFETCH 4
 #endif
 
 namespace sdpa {
@@ -86,7 +82,6 @@ struct TcCfg {
   static constexpr int kCols = BN / kParts;  // key columns per softmax thread
   static constexpr uint32_t kTmemCols = 512;
   static constexpr int kOCol = kBufs * BN;
-  static constexpr int kPrefetch = SDPA_TC_PREFETCH;
   static_assert(DQK % 16 == 0 && DV % 16 == 0 && DV >= 16 && DV <= 256, "head dims");
   static_assert(BN == 32 || BN == 64 || BN == 128, "key block");
   static_assert(kCols == 16 || kCols % 32 == 0, "TMEM load / store widths");
@@ -197,7 +192,7 @@ __global__ void __launch_bounds__(TcCfg<DQK, DV, BN, NSLOT>::kThreads, 1)
         tma_load_2d(sQ + bx * (Cfg::kBM * 128), &tm_q, q_full, bx * 64, grow0);
       int u = 0;
       bool ok = true;
-      // one load into the next ring slot, plus an L2 prefetch further ahead
+      // one load into the next ring slot
       auto emit = [&](bool is_k, int blk) {
         const int slot = u % NSLOT;
         const uint32_t ph = (uint32_t)(u / NSLOT) & 1u;
@@ -212,15 +207,6 @@ __global__ void __launch_bounds__(TcCfg<DQK, DV, BN, NSLOT>::kThreads, 1)
 #pragma unroll
           for (int bx = 0; bx < Cfg::kQBoxes; ++bx)
             tma_load_3d(dst + bx * (BN * 128), &tm_k, &slot_full[slot], bx * 64, k0, bh);
-          const int pf = blk + Cfg::kPrefetch;
-          if (pf < nblk) {
-#pragma unroll
-            for (int bx = 0; bx < Cfg::kQBoxes; ++bx)
-              tma_prefetch_l2_3d(&tm_k, bx * 64, k_lo + pf * BN, bh);
-#pragma unroll
-            for (int bx = 0; bx < Cfg::kVBoxes; ++bx)
-              tma_prefetch_l2_3d(&tm_v, bx * 64, k_lo + pf * BN, bh);
-          }
         } else {
           mbar_arrive_expect_tx(&slot_full[slot], Cfg::kVBytes);
 #pragma unroll

@@ -25,7 +25,7 @@
 //              16-bit input type and written over the row's own scores.
 //   warps 4-7  softmax of tile B, the same on lanes 32 (w-4) .. +31.
 //   warp 8     TMA producer: Q of both tiles once, then K_0, V_0, K_1, V_1,
-//              ... through a ring of NSLOT slots, plus L2 prefetches ahead.
+//              ... through a ring of NSLOT slots.
 //   warp 9     allocates TMEM and issues every MMA from one thread, in the
 //              order S_A(0), S_B(0), then per block j: P_A(j) V_j, S_A(j+1),
 //              P_B(j) V_j, S_B(j+1).  Each K/V slot is released after its
@@ -86,7 +86,6 @@ struct PpCfg {
   static constexpr int kThreads = 320;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr int kTileCols = 256;  // TMEM columns per tile
-  static constexpr int kPrefetch = 4;    // K/V blocks prefetched into L2 ahead of the loads
   static_assert(DQK % 16 == 0 && DV % 16 == 0 && DV >= 16, "head dims");
   static_assert(BN == 128 || (BN == 96 && !KSPLIT), "key block");
   static_assert(BN + DV <= kTileCols, "TMEM columns per tile");
@@ -210,15 +209,6 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
             for (int bx = 0; bx < Cfg::kQBoxes; ++bx)
               tma_load_3d(dst + bx * (BN * 128), &tm_k, &slot_full[slot], bx * 64, k0, bh);
-            const int pf = blk + Cfg::kPrefetch;
-            if (pf < nblk) {
-#pragma unroll
-              for (int bx = 0; bx < Cfg::kQBoxes; ++bx)
-                tma_prefetch_l2_3d(&tm_k, bx * 64, k_lo + pf * BN, bh);
-#pragma unroll
-              for (int bx = 0; bx < Cfg::kVBoxes; ++bx)
-                tma_prefetch_l2_3d(&tm_v, bx * 64, k_lo + pf * BN, bh);
-            }
           } else {
             mbar_arrive_expect_tx(&slot_full[slot], Cfg::kVBytes);
 #pragma unroll
@@ -249,15 +239,6 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
             for (int bx = 0; bx < Cfg::kQBoxes; ++bx)
               tma_load_3d(dst + bx * (BN * 128), &tm_k, &slot_full[slot], bx * 64, k0, bh);
-            const int pf = j + Cfg::kPrefetch;
-            if (pf < nblk) {
-#pragma unroll
-              for (int bx = 0; bx < Cfg::kQBoxes; ++bx)
-                tma_prefetch_l2_3d(&tm_k, bx * 64, k_lo + pf * BN, bh);
-#pragma unroll
-              for (int bx = 0; bx < Cfg::kVBoxes; ++bx)
-                tma_prefetch_l2_3d(&tm_v, bx * 64, k_lo + pf * BN, bh);
-            }
           } else {
             mbar_arrive_expect_tx(&slot_full[slot], Cfg::kVBytes);
 #pragma unroll

@@ -123,11 +123,19 @@ def test_plan_packs_verify_rows_per_kv_head():
 
 def test_plan_two_split_kv_ctas_per_sm_only_for_the_64_row_layout():
     # 33..64 packed rows (four row warps, no key slices) run two CTAs per SM,
-    # so the planner fills twice the SM count; 16- and 32-row layouts one
+    # so the planner fills twice the SM count; 16- and 32-row layouts one.
+    # The router sends 33..64 rows to the tcgen05 kernel, so that layout is
+    # forced here.
     for L, per_sm in ((4, 1), (8, 1), (12, 2), (16, 2)):
-        info = sdpa.plan(1, 32, 8, L, 32768, 128, 128, causal=False, dtype="f16", num_sms=148)
+        info = sdpa.plan(1, 32, 8, L, 32768, 128, 128, causal=False, dtype="f16", num_sms=148,
+                         force_path=sdpa.PATH_SPLITKV)
         assert info["path"] == sdpa.PATH_SPLITKV
         assert per_sm * 148 - 8 < info["ctas"] <= per_sm * 148, (L, info)
+    # routed: up to 32 packed rows on the split-KV kernel, from 33 on tcgen05
+    for L, path in ((4, sdpa.PATH_SPLITKV), (8, sdpa.PATH_SPLITKV), (9, sdpa.PATH_TC),
+                    (12, sdpa.PATH_TC), (16, sdpa.PATH_TC)):
+        info = sdpa.plan(1, 32, 8, L, 32768, 128, 128, causal=False, dtype="f16", num_sms=148)
+        assert info["path"] == path, (L, info)
     # head dims whose stages do not fit half the shared memory stay at one per SM
     info = sdpa.plan(1, 32, 8, 16, 32768, 256, 256, causal=False, num_sms=148)
     assert info["ctas"] <= 148
