@@ -1,105 +1,106 @@
 // Log-sum-exp combine of split partials (mlx issue #3826: split over S, then
 // a log-sum-exp merge; mlx PR #3637: the 2-pass kernel's aggregation).
-// One CTA of 128 threads per output row and 128 output columns:
 //   LSE = max_s LSE_s + ln sum_s exp(LSE_s - max),  O = sum_s exp(LSE_s - LSE) O_s
 // Splits that saw no visible key carry LSE_s = -inf and weight 0.  A head's
 // sink (when given) joins as one more term with weight exp(sink - LSE) and
-// no value row.  Every thread loads its column's partials of the first 64
-// splits and one split LSE in the same round trip to L2; two block
-// reductions (max, then the weight sum) form the weights in shared memory,
-// and each thread accumulates its output column.
+// no value row.
+//
+// One warp per output row and 128 output columns, four rows per CTA: each
+// lane owns four adjacent columns (one 16-byte load per split) and holds the
+// LSE of split `lane` of each round of 32.  The first round's partials and
+// LSEs are requested together, so up to 32 splits cost one round trip to L2
+// before the reductions; the LSE max and the weight sum are warp shuffles
+// (no shared memory, no block barrier), and each split's weight reaches the
+// lanes by one more shuffle.
 // Launched as a programmatic dependent of the split pass: it waits for that
 // grid (griddepcontrol.wait) before touching the partials.
 #pragma once
 
 #include "params.cuh"
 
-// splits loaded per round trip to L2 after the first kPre
-#ifndef SDPA_COMBINE_BATCH
-#define SDPA_COMBINE_BATCH 16
-#endif
-
 namespace sdpa {
 
+constexpr int kCombineRowsPerCta = 4;
+
 template <bool kBF16>
-__global__ void __launch_bounds__(128) combine_kernel(const float *__restrict__ part_o,
-                                                      const float *__restrict__ part_lse,
-                                                      void *__restrict__ out, float *lse_out,
-                                                      const float *__restrict__ sinks,
-                                                      long total_rows, int Dv, int splits, int L,
-                                                      int Hq) {
-  extern __shared__ float s_w[];  // [splits]: the split LSEs, then their weights
-  __shared__ float s_red[2][4];   // per-warp max, per-warp weight sum
-  constexpr int kPre = 64;        // splits whose partials go out in the first round trip
+__global__ void __launch_bounds__(32 * kCombineRowsPerCta)
+    combine_kernel(const float *__restrict__ part_o, const float *__restrict__ part_lse,
+                   void *__restrict__ out, float *lse_out, const float *__restrict__ sinks,
+                   long total_rows, int Dv, int splits, int L, int Hq) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   // the next split pass on the stream may start its setup now; it waits for
   // this grid before it reads or writes global memory
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const long row = blockIdx.x;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int col = blockIdx.y * 128 + tid;  // this thread's output column
-  const bool live = col < Dv;
-  const long stride = total_rows * Dv;
+  const int lane = threadIdx.x & 31;
+  const long row = (long)blockIdx.x * kCombineRowsPerCta + (threadIdx.x >> 5);
+  if (row >= total_rows) return;  // whole warps
+  const int col = blockIdx.y * 128 + lane * 4;  // this lane's four output columns
+  const bool live = col < Dv;                   // Dv is a multiple of 8
+  const long stride = total_rows * Dv;          // floats between two splits' partials
   const float *src = part_o + row * Dv + col;
-  // One round trip to L2: each thread's partials of the first kPre splits and
-  // one split LSE per thread (up to 128 splits; more take further rounds).
-  float v[kPre];
+  const float *lse = part_lse + row;
+
+  // ---- first round: the partials of splits 0..31 and their LSEs (lane s
+  // holds split s's) go out together, before any reduction ----
+  float4 v[32];
 #pragma unroll
-  for (int t = 0; t < kPre; ++t) v[t] = (t < splits && live) ? __ldcg(src + (long)t * stride) : 0.f;
-  float mx = -INFINITY;
-  for (int s = tid; s < splits; s += 128) {
-    const float x = __ldcg(part_lse + (long)s * total_rows + row);
-    s_w[s] = x;
-    mx = fmaxf(mx, x);
-  }
-  // block max of the split LSEs and the sink
+  for (int k = 0; k < 32; ++k)
+    v[k] = (live && k < splits)
+               ? __ldcg(reinterpret_cast<const float4 *>(src + (long)k * stride))
+               : make_float4(0.f, 0.f, 0.f, 0.f);
+  const float lse0 = lane < splits ? __ldcg(lse + (long)lane * total_rows) : -INFINITY;
+  // the LSE max over all splits (and the sink)
+  float mx = lse0;
+  for (int s = lane + 32; s < splits; s += 32) mx = fmaxf(mx, __ldcg(lse + (long)s * total_rows));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  if (lane == 0) s_red[0][warp] = mx;
-  __syncthreads();
   const float sink = sinks != nullptr ? sinks[(int)((row / L) % Hq)] : -INFINITY;
-  mx = fmaxf(fmaxf(fmaxf(s_red[0][0], s_red[0][1]), fmaxf(s_red[0][2], s_red[0][3])), sink);
+  mx = fmaxf(mx, sink);
   const float ref = mx == -INFINITY ? 0.f : mx;
-  // weights exp(LSE_s - ref); each thread rereads the entries it wrote
-  float den = 0.f;
-  for (int s = tid; s < splits; s += 128) {
-    const float w = __expf(s_w[s] - ref);
-    s_w[s] = w;
-    den += w;
+
+  // ---- weighted sum: lane s's weight is shuffled out to every lane ----
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float w_own = lane < splits ? __expf(lse0 - ref) : 0.f;
+  float den = w_own;
+#pragma unroll
+  for (int k = 0; k < 32; ++k) {
+    const float w = __shfl_sync(0xffffffffu, w_own, k);
+    acc.x += w * v[k].x;
+    acc.y += w * v[k].y;
+    acc.z += w * v[k].z;
+    acc.w += w * v[k].w;
+  }
+  // further rounds of 32 splits
+  for (int s0 = 32; s0 < splits; s0 += 32) {
+    const int s = s0 + lane;
+#pragma unroll
+    for (int k = 0; k < 32; ++k)
+      v[k] = (live && s0 + k < splits)
+                 ? __ldcg(reinterpret_cast<const float4 *>(src + (long)(s0 + k) * stride))
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
+    w_own = s < splits ? __expf(__ldcg(lse + (long)s * total_rows) - ref) : 0.f;
+    den += w_own;
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+      const float w = __shfl_sync(0xffffffffu, w_own, k);
+      acc.x += w * v[k].x;
+      acc.y += w * v[k].y;
+      acc.z += w * v[k].z;
+      acc.w += w * v[k].w;
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-  if (lane == 0) s_red[1][warp] = den;
-  __syncthreads();
-  den = (s_red[1][0] + s_red[1][1]) + (s_red[1][2] + s_red[1][3]);
   if (sinks != nullptr) den += __expf(sink - ref);
-  float acc = 0.f;
-#pragma unroll
-  for (int t = 0; t < kPre; ++t) {
-    const float w = t < splits ? s_w[t] : 0.f;
-    acc += w * v[t];
-  }
-  // splits past kPre, kBatch per round trip
-  constexpr int kBatch = SDPA_COMBINE_BATCH;
-  for (int s0 = kPre; s0 < splits; s0 += kBatch) {
-    float x[kBatch];
-#pragma unroll
-    for (int t = 0; t < kBatch; ++t)
-      x[t] = (s0 + t < splits && live) ? __ldcg(src + (long)(s0 + t) * stride) : 0.f;
-#pragma unroll
-    for (int t = 0; t < kBatch; ++t) {
-      const float w = s0 + t < splits ? s_w[s0 + t] : 0.f;
-      acc += w * x[t];
-    }
-  }
+
+  const float inv = den > 0.f ? 1.f / den : 0.f;
   if (live) {
-    const float o = den > 0.f ? acc / den : 0.f;
-    if constexpr (kBF16)
-      reinterpret_cast<__nv_bfloat16 *>(out)[row * Dv + col] = __float2bfloat16_rn(o);
-    else
-      reinterpret_cast<__half *>(out)[row * Dv + col] = __float2half_rn(o);
+    uint2 w;
+    w.x = pack2<kBF16>(acc.x * inv, acc.y * inv);
+    w.y = pack2<kBF16>(acc.z * inv, acc.w * inv);
+    *reinterpret_cast<uint2 *>(reinterpret_cast<uint16_t *>(out) + row * Dv + col) = w;
   }
-  if (lse_out != nullptr && blockIdx.y == 0 && tid == 0)
+  if (lse_out != nullptr && blockIdx.y == 0 && lane == 0)
     lse_out[row] = den > 0.f ? ref + logf(den) : -INFINITY;
 }
 

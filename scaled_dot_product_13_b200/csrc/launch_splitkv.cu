@@ -127,9 +127,11 @@ sdpa_status launch_combine(const Launch &ln, std::string *err) {
   // it, which hides the second launch's latency.
   const long total = (long)ln.pb.B * ln.pb.Hq * ln.pb.L;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)total, (unsigned)((ln.pb.Dv + 127) / 128));
-  cfg.blockDim = dim3(128);
-  cfg.dynamicSmemBytes = (size_t)ln.plan.splits * sizeof(float);
+  // one warp per output row and 128 columns, kCombineRowsPerCta rows per CTA
+  cfg.gridDim = dim3((unsigned)((total + kCombineRowsPerCta - 1) / kCombineRowsPerCta),
+                     (unsigned)((ln.pb.Dv + 127) / 128));
+  cfg.blockDim = dim3(32 * kCombineRowsPerCta);
+  cfg.dynamicSmemBytes = 0;
   cfg.stream = ln.stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
