@@ -38,7 +38,10 @@
 // when a block's max exceeds it by more than 8 (log2 units), so O in TMEM is
 // rescaled rarely.  exp2(s - m) then stays below 2^8, which bf16/fp16 P and
 // the fp32 sums hold without loss; l and O share the same reference, so the
-// final O / l is the same softmax.
+// final O / l is the same softmax.  An unmasked block first takes P against
+// the reference in use: a row sum below 224 shows that no score passed it by
+// 8, and the block's row max (about a fifth of the softmax's time per block)
+// is only taken when some row's sum reaches 224.
 #pragma once
 
 #include "params.cuh"
@@ -323,116 +326,149 @@ __global__ void __launch_bounds__(TcCfg<DQK, DV, BN, NSLOT>::kThreads, 1)
       }
       tc_fence_after();
       float s[kH];
-      if constexpr (kH == 16) {
-        float s16[16];
-        tmem_ld16(tmem + lane_base + b * BN + part * kH, s16);
+      auto load_s = [&]() {
+        if constexpr (kH == 16) {
+          float s16[16];
+          tmem_ld16(tmem + lane_base + b * BN + part * kH, s16);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) s[i] = s16[i];
-      } else {
+          for (int i = 0; i < 16; ++i) s[i] = s16[i];
+        } else {
 #pragma unroll
-        for (int c32 = 0; c32 < kH / 32; ++c32)
-          tmem_ld32(tmem + lane_base + b * BN + part * kH + c32 * 32, s + c32 * 32);
-      }
-      tmem_wait_ld();
+          for (int c32 = 0; c32 < kH / 32; ++c32)
+            tmem_ld32(tmem + lane_base + b * BN + part * kH + c32 * 32, s + c32 * 32);
+        }
+        tmem_wait_ld();
+      };
+      load_s();
 
-      // ---- this part's raw row max (masked keys excluded) ----
+      // ---- P = exp2(s * c - m) (two lanes per FMA) against the reference m
+      // in use, packed to the 16-bit type; returns the row sum ----
+      uint32_t pk[kH / 2];
+      auto exp_pack = [&]() -> float {
+        const float mref = m_used == -INFINITY ? 0.f : m_used;
+        const float2 c2 = make_float2(c_eff, c_eff), nm2 = make_float2(-mref, -mref);
+        float2 acc[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) acc[t] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < kH; i += 2) {
+          float2 t = fma2(make_float2(s[i], s[i + 1]), c2, nm2);
+          if (((i >> 1) & 3) < SDPA_TC_POLY_OF4) {
+            t = exp2_poly2(t);  // FMA / ALU pipes
+          } else {
+            t.x = fast_exp2(t.x);  // MUFU
+            t.y = fast_exp2(t.y);
+          }
+          acc[(i >> 1) & 3] = add2(acc[(i >> 1) & 3], t);
+          pk[i >> 1] = pack2<kBF16>(t.x, t.y);
+        }
+        const float2 a01 = add2(acc[0], acc[1]), a23 = add2(acc[2], acc[3]);
+        const float2 at = add2(a01, a23);
+        return at.x + at.y;
+      };
+
       const int kbase = k_lo + j * BN;
       const bool masked = block_needs_mask(p, tr, kbase, BN);
-      // The common block (positive scale, no masked key) takes the plain
-      // reduction; the rare ones (scale 0, masked keys, negative scale) their
-      // own copy, so that their per-element work is not folded into it.
-      float mr[1];
-      if (!masked && c_pos && !c_zero) {
-        mr[0] = row_reduce_max(s);
-      } else {
-        if (c_zero) {
-#pragma unroll
-          for (int i = 0; i < kH; ++i) s[i] = 0.f;
-        }
-        if (masked) {
-          const VisibleRange vis = visible_range(p, pos, kbase + part * kH);
-#pragma unroll
-          for (int i = 0; i < kH; ++i)
-            if (!vis(i)) s[i] = neutral;
-        }
-        mr[0] = c_pos ? row_reduce_max(s) : row_reduce_min(s);
+      // Plain blocks (positive scale, no masked key, a reference already
+      // set) first take P against the current reference.  The reference only
+      // moves when a score exceeds it by more than 8 (log2 units): then some
+      // P is above 2^7.875 (the rounding of s * c - m stays below 1/8 while
+      // |m| < 2^20), so a row sum below 224 rules it out and the row max is
+      // needed only for the rare block whose sum reaches 224 (or is NaN).
+      // (A row of equal scores, zero-filled padding rows included, sums to at
+      // most BN and stays on the fast side.)
+      // Either way P, the reference and the sum are those of the max-first
+      // order below, bit for bit.
+      const bool optimistic = kParts == 1 && !masked && c_pos && !c_zero &&
+                              !__any_sync(0xffffffffu, m_used == -INFINITY);
+      float lsum = 0.f;
+      bool by_max = true;
+      if (optimistic) {
+        lsum = exp_pack();
+        by_max = __any_sync(0xffffffffu, !(lsum < 224.f));
+        if (by_max) load_s();  // the scores are still in TMEM (P not stored)
       }
-      // ---- combine with the other parts of the row (bounded barrier).  The
-      // barrier also orders every part's score reads before any part
-      // overwrites them with P. ----
-      float mraw = mr[0];
-      if constexpr (kParts > 1) {
-        xmax[((j & 1) * kParts + part) * Cfg::kBM + r] = mr[0];
-        tc_fence_before();
-        mbar_arrive(&part_bar[quarter]);
-        if (!mbar_wait(&part_bar[quarter], part_phase & 1u, p.wd, kWdSoftmax)) {
-          ok = false;
-          break;
-        }
-        ++part_phase;
-        tc_fence_after();
-#pragma unroll
-        for (int q = 0; q < kParts; ++q) {
-          const float other = xmax[((j & 1) * kParts + q) * Cfg::kBM + r];
-          mraw = c_pos ? fmaxf(mraw, other) : fminf(mraw, other);
-        }
-      }
-      const float mblk = isinf(mraw) ? -INFINITY : mraw * c_eff;
-      const float m_new = fmaxf(m_used, mblk);
-      const bool need = m_new > m_used + 8.0f;
-      float alpha = 1.f;
-      if (need) {
-        alpha = fast_exp2(m_used - m_new);
-        m_used = m_new;
-        l *= alpha;
-      }
-      if (j > 0 && __any_sync(0xffffffffu, need)) {
-        // O holds P_0..P_{j-1} V: wait for the last P V, then rescale this
-        // warp's columns in TMEM.  P_{j-1} V commits to o_bar[(j-1) % 2] as
-        // that barrier's phase (j-1) / 2.  The parity is unambiguous: S_j was
-        // issued after P_{j-3} V by the same thread, so S_j's completion
-        // implies the barrier's previous phase (P_{j-3} V) completed, and its
-        // next one (P_{j+1} V) waits for p_full of a block not yet done.
-        if (lane == 0)
-          w = mbar_wait(&o_bar[(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1u, p.wd, kWdMma);
-        if (!__shfl_sync(0xffffffffu, (int)w, 0)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-#pragma unroll 1
-        for (int c16 = oc_begin; c16 < oc_end; ++c16) {
-          float o[16];
-          tmem_ld16(tmem + lane_base + Cfg::kOCol + c16 * 16, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 16; ++e) o[e] *= alpha;
-          tmem_st16(tmem + lane_base + Cfg::kOCol + c16 * 16, o);
-        }
-        tmem_wait_st();
-      }
-      // ---- P = exp2(s * c - m) (two lanes per FMA), row sums ----
-      const float mref = m_used == -INFINITY ? 0.f : m_used;
-      const float2 c2 = make_float2(c_eff, c_eff), nm2 = make_float2(-mref, -mref);
-      float2 acc[4];
-#pragma unroll
-      for (int t = 0; t < 4; ++t) acc[t] = make_float2(0.f, 0.f);
-      uint32_t pk[kH / 2];
-#pragma unroll
-      for (int i = 0; i < kH; i += 2) {
-        float2 t = fma2(make_float2(s[i], s[i + 1]), c2, nm2);
-        if (((i >> 1) & 3) < SDPA_TC_POLY_OF4) {
-          t = exp2_poly2(t);  // FMA / ALU pipes
+      if (by_max) {
+        // ---- this part's raw row max (masked keys excluded) ----
+        // The common block (positive scale, no masked key) takes the plain
+        // reduction; the rare ones (scale 0, masked keys, negative scale)
+        // their own copy, so that their per-element work is not folded in.
+        float mr[1];
+        if (!masked && c_pos && !c_zero) {
+          mr[0] = row_reduce_max(s);
         } else {
-          t.x = fast_exp2(t.x);  // MUFU
-          t.y = fast_exp2(t.y);
+          if (c_zero) {
+#pragma unroll
+            for (int i = 0; i < kH; ++i) s[i] = 0.f;
+          }
+          if (masked) {
+            const VisibleRange vis = visible_range(p, pos, kbase + part * kH);
+#pragma unroll
+            for (int i = 0; i < kH; ++i)
+              if (!vis(i)) s[i] = neutral;
+          }
+          mr[0] = c_pos ? row_reduce_max(s) : row_reduce_min(s);
         }
-        acc[(i >> 1) & 3] = add2(acc[(i >> 1) & 3], t);
-        pk[i >> 1] = pack2<kBF16>(t.x, t.y);
+        // ---- combine with the other parts of the row (bounded barrier).
+        // The barrier also orders every part's score reads before any part
+        // overwrites them with P. ----
+        float mraw = mr[0];
+        if constexpr (kParts > 1) {
+          xmax[((j & 1) * kParts + part) * Cfg::kBM + r] = mr[0];
+          tc_fence_before();
+          mbar_arrive(&part_bar[quarter]);
+          if (!mbar_wait(&part_bar[quarter], part_phase & 1u, p.wd, kWdSoftmax)) {
+            ok = false;
+            break;
+          }
+          ++part_phase;
+          tc_fence_after();
+#pragma unroll
+          for (int q = 0; q < kParts; ++q) {
+            const float other = xmax[((j & 1) * kParts + q) * Cfg::kBM + r];
+            mraw = c_pos ? fmaxf(mraw, other) : fminf(mraw, other);
+          }
+        }
+        const float mblk = isinf(mraw) ? -INFINITY : mraw * c_eff;
+        const float m_new = fmaxf(m_used, mblk);
+        const bool need = m_new > m_used + 8.0f;
+        float alpha = 1.f;
+        if (need) {
+          alpha = fast_exp2(m_used - m_new);
+          m_used = m_new;
+          l *= alpha;
+        }
+        const bool any_need = __any_sync(0xffffffffu, need);
+        if (j > 0 && any_need) {
+          // O holds P_0..P_{j-1} V: wait for the last P V, then rescale this
+          // warp's columns in TMEM.  P_{j-1} V commits to o_bar[(j-1) % 2] as
+          // that barrier's phase (j-1) / 2.  The parity is unambiguous: S_j was
+          // issued after P_{j-3} V by the same thread, so S_j's completion
+          // implies the barrier's previous phase (P_{j-3} V) completed, and its
+          // next one (P_{j+1} V) waits for p_full of a block not yet done.
+          if (lane == 0)
+            w = mbar_wait(&o_bar[(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1u, p.wd, kWdMma);
+          if (!__shfl_sync(0xffffffffu, (int)w, 0)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll 1
+          for (int c16 = oc_begin; c16 < oc_end; ++c16) {
+            float o[16];
+            tmem_ld16(tmem + lane_base + Cfg::kOCol + c16 * 16, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) o[e] *= alpha;
+            tmem_st16(tmem + lane_base + Cfg::kOCol + c16 * 16, o);
+          }
+          tmem_wait_st();
+        }
+        // P again where the reference moved (every lane recomputes: an
+        // unchanged reference gives the same P and sum)
+        if (!optimistic || any_need) lsum = exp_pack();
       }
-      const float2 a01 = add2(acc[0], acc[1]), a23 = add2(acc[2], acc[3]);
-      const float2 at = add2(a01, a23);
-      l += at.x + at.y;
+      l += lsum;
       // P_j into this warp's packed columns of buffer b (over the first
       // BN/2 score columns)
       if constexpr (kH == 16) {

@@ -1,6 +1,7 @@
 """GPU parity of the tcgen05 path (128-row tensor-memory tiles) with the route
 pinned, against the oracle, and agreement between the two routes."""
 import pytest
+import torch
 
 import scaled_dot_product_13_b200 as S
 from scaled_dot_product_13_b200 import inputs as I
@@ -59,3 +60,31 @@ def test_routes_agree(cuda_lib, case):
     a = run_gpu(cuda_lib, p, q, k, v, force_path=S.PATH_TC)[0].float()
     b = run_gpu(cuda_lib, p, q, k, v, force_path=S.PATH_SPLITKV)[0].float()
     assert agree(a, b, dt)
+
+
+@pytest.mark.parametrize("kind,dt", [("rising", "bf16"), ("rising", "f16"), ("falling", "bf16"),
+                                     ("flat_rows", "bf16")])
+def test_tc_reference_moves_inside_plain_blocks(cuda_lib, kind, dt):
+    """Unmasked blocks first take P against the reference in use and take the
+    row max only when the block's row sum reaches 224.  Keys whose scale
+    grows along the sequence move the reference in later unmasked blocks
+    (sums far above 224, with and without a move); keys whose scale shrinks
+    leave every later block far below the reference (P near underflow);
+    query heads of zeros give rows of equal scores, whose sums are exactly
+    the block width.  All against the oracle, on the one-tile route."""
+    from oracle import sdpa_oracle
+    from tests.gpu_util import TOL_MAX, TOL_MEAN, compare
+    p = I.Problem(1, 4, 2, 256, 2048, 128, 128, dt, False, 0, None, 31, kind)
+    q, k, v = I.make_qkv(p)
+    if kind in ("rising", "falling"):
+        g = 1.0 + 8.0 * torch.arange(p.S, dtype=torch.float32) / p.S  # x1 .. x9
+        if kind == "falling":
+            g = g.flip(0)
+        k = (k.float() * g[None, None, :, None]).to(k.dtype)
+    else:
+        q[:, ::2] = 0
+    out, info = run_gpu(cuda_lib, p, q, k, v, force_path=S.PATH_TC)
+    assert info["path"] == S.PATH_TC
+    ref = sdpa_oracle(q, k, v, p.sm_scale, p.causal, p.window)
+    mx, mean = compare(p, out.float().cpu().numpy(), ref)
+    assert mx <= TOL_MAX[dt] and mean <= TOL_MEAN, f"{kind}: max {mx:.3e} mean {mean:.3e}"
