@@ -123,14 +123,17 @@ def test_plan_packs_verify_rows_per_kv_head():
 
 def test_plan_two_split_kv_ctas_per_sm_only_for_the_64_row_layout():
     # 33..64 packed rows (four row warps, no key slices) run two CTAs per SM,
-    # so the planner fills twice the SM count; 16- and 32-row layouts one.
+    # so the planner fills twice the SM count; 16- and 32-row layouts one
+    # (less at most a seventh, where the split count is rounded down to a
+    # whole number of the combine's 32-split rounds: 37 -> 32 per KV head).
     # The router sends 33..64 rows to the tcgen05 kernel, so that layout is
     # forced here.
     for L, per_sm in ((4, 1), (8, 1), (12, 2), (16, 2)):
         info = sdpa.plan(1, 32, 8, L, 32768, 128, 128, causal=False, dtype="f16", num_sms=148,
                          force_path=sdpa.PATH_SPLITKV)
         assert info["path"] == sdpa.PATH_SPLITKV
-        assert per_sm * 148 - 8 < info["ctas"] <= per_sm * 148, (L, info)
+        assert per_sm * 148 * 6 // 7 <= info["ctas"] <= per_sm * 148, (L, info)
+        assert (per_sm - 1) * 148 < info["ctas"], (L, info)
     # routed: up to 32 packed rows on the split-KV kernel, from 33 on tcgen05
     for L, path in ((4, sdpa.PATH_SPLITKV), (8, sdpa.PATH_SPLITKV), (9, sdpa.PATH_TC),
                     (12, sdpa.PATH_TC), (16, sdpa.PATH_TC)):
@@ -268,3 +271,19 @@ def test_plan_looping_pair_path():
     with pytest.raises(sdpa.SdpaError) as ei:
         sdpa.plan(1, 4, 4, 64, 64, 512, 512, num_sms=148, force_path=sdpa.PATH_TC2_LOOP)
     assert ei.value.status == 2
+
+
+def test_plan_rounds_split_counts_to_whole_combine_rounds():
+    # the combine merges 32 splits per round: a count within a seventh above a
+    # multiple of 32 is rounded down to it, a larger remainder is kept
+    info = sdpa.plan(1, 64, 4, 1, 32768, 192, 128, causal=True, num_sms=148)
+    assert info["splits"] == 32 and info["ctas"] == 128, info   # 37 -> 32
+    info = sdpa.plan(1, 32, 2, 1, 32768, 128, 128, causal=True, num_sms=148)
+    assert info["splits"] == 64, info                            # 74 -> 64
+    info = sdpa.plan(1, 48, 3, 1, 32768, 128, 128, causal=True, num_sms=148)
+    assert 32 < info["splits"] < 64, info                        # 49 stays above 32
+    info = sdpa.plan(1, 64, 8, 1, 32768, 192, 128, causal=True, num_sms=148)
+    assert info["splits"] == 18, info                            # below 32: unchanged
+    # a pinned split count is kept as given
+    info = sdpa.plan(1, 64, 4, 1, 32768, 192, 128, causal=True, num_sms=148, force_splits=37)
+    assert info["splits"] == 37, info
