@@ -241,9 +241,16 @@ sdpa_status make_plan(const Problem &pb, int num_sms, int force_path, int force_
   }
   if (path == SDPA_PATH_AUTO) {
     path = pl.rows >= kTcRowThreshold ? SDPA_PATH_TC : SDPA_PATH_SPLITKV;
-    // wide heads with at least one full 256-row pair tile: two SMs per tile
-    if (path == SDPA_PATH_TC && tc2_preferred_pair(pl.pair) && pl.rows >= kTc2RowThreshold)
-      path = SDPA_PATH_TC2;
+    // wide heads with at least one full 256-row pair tile: two SMs per tile.
+    // Causal or windowed tiles see key ranges of different lengths; between
+    // one and two of them per SM pair they balance better as twice as many
+    // 128-row tiles on the one-SM kernel (2K calls with 128 pair tiles:
+    // causal 51.2 against 57.4 us, window 512 43.0 against 49.2).
+    if (path == SDPA_PATH_TC && tc2_preferred_pair(pl.pair) && pl.rows >= kTc2RowThreshold) {
+      const long long pair_tiles = (long long)pb.B * pb.Hkv * ((pl.rows + 255) / 256);
+      const bool uneven = pb.causal || pb.window > 0;
+      if (!(uneven && 2 * pair_tiles > num_sms && pair_tiles < num_sms)) path = SDPA_PATH_TC2;
+    }
     // head dims <= 80 (where P has TMEM columns of its own): two 128-row
     // tiles per CTA, when the 256-row tiles alone occupy at least half of the
     // SMs (fewer would rather take the one-tile kernel's twice as many CTAs)

@@ -243,13 +243,24 @@ def test_plan_two_tile_path_for_small_head_dims():
 
 
 def test_plan_looping_pair_path():
-    # sliding windows over more 256-row tiles than SM pairs: the pair kernel
-    # loops over its tiles
-    for n in (2048, 4096, 8192):
+    # sliding windows over at least twice as many 256-row tiles as SM pairs:
+    # the pair kernel loops over its tiles
+    for n in (4096, 8192):
         info = sdpa.plan(1, 16, 8, n, n, 256, 256, causal=True, window_size=1024, num_sms=148)
         assert info["path"] == sdpa.PATH_TC2_LOOP and info["splits"] == 1
         assert info["ctas"] == 8 * (2 * n // 256) and info["launches"] == 1
         assert info["workspace_bytes"] == 0
+    # between one and two causal (or windowed) pair tiles per SM pair: twice as
+    # many 128-row tiles on the one-SM kernel; non-causal tiles keep the pair
+    for window in (1024, 512, 0):
+        info = sdpa.plan(1, 16, 8, 2048, 2048, 256, 256, causal=True, window_size=window,
+                         num_sms=148)
+        assert info["path"] == sdpa.PATH_TC and info["splits"] == 1, (window, info)
+        assert info["ctas"] == 8 * (2 * 2048 // 128)
+    info = sdpa.plan(1, 16, 8, 2048, 2048, 256, 256, causal=False, num_sms=148)
+    assert info["path"] == sdpa.PATH_TC2_LOOP
+    info = sdpa.plan(1, 16, 16, 1536, 1536, 192, 128, causal=True, window_size=1024, num_sms=148)
+    assert info["path"] == sdpa.PATH_TC
     # long causal tiles keep one pair per tile
     info = sdpa.plan(1, 16, 8, 32768, 32768, 256, 256, causal=True, num_sms=148)
     assert info["path"] == sdpa.PATH_TC2
