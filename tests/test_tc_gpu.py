@@ -88,3 +88,18 @@ def test_tc_reference_moves_inside_plain_blocks(cuda_lib, kind, dt):
     ref = sdpa_oracle(q, k, v, p.sm_scale, p.causal, p.window)
     mx, mean = compare(p, out.float().cpu().numpy(), ref)
     assert mx <= TOL_MAX[dt] and mean <= TOL_MEAN, f"{kind}: max {mx:.3e} mean {mean:.3e}"
+
+
+@pytest.mark.parametrize("case", [
+    # causal and windowed calls with one to two 256-row pair tiles per SM pair
+    # take the one-SM kernel's 128-row tiles (router rule), at full size
+    ("d256_causal_2k", 1, 16, 8, 2048, 2048, 256, 256, True, 0),
+    ("d192_128_causal_1536", 1, 16, 16, 1536, 1536, 192, 128, True, 0),
+    ("d192_128_window_1536", 1, 16, 16, 1536, 1536, 192, 128, True, 700),
+], ids=lambda c: c[0])
+def test_balance_rule_routes_to_one_sm_kernel(cuda_lib, case):
+    name, B, Hq, Hkv, L, Sk, Dqk, Dv, causal, W = case
+    p = I.Problem(B, Hq, Hkv, L, Sk, Dqk, Dv, "bf16", causal, W, None, 33, name)
+    rows = I.sample_rows(L, 256, 33, window=W)
+    _, _, info = check_problem(cuda_lib, p, rows=rows)
+    assert info["path"] == S.PATH_TC and info["splits"] == 1, info
