@@ -416,8 +416,20 @@ def secondary(sdpa, probs, steps, warmup, flush, sync_all, device, peaks, kind, 
     # Each timing pass goes over the list in order, heaviest call last, with a
     # pause after it: seconds of full tensor load lower the clock under the
     # power cap for a while, which would slow the next pass's first calls.
-    alone = [time_alone(sdpa, c, flush, reps=max(steps, 20)) for c in cases] if graphs else None
-    time.sleep(1.0)
+    # A call timed alone takes the median of its means over three such passes,
+    # so that a drift of the clock during one pass does not land on one call
+    # (calls of the same work, e.g. verify L = 12..32 on one 128-row tile,
+    # otherwise differed by up to 3.5 %).
+    alone = None
+    if graphs:
+        passes = 3
+        reps = max(steps, 20) // passes + 1
+        per = [[] for _ in cases]
+        for _ in range(passes):
+            for i, c in enumerate(cases):
+                per[i].append(time_alone(sdpa, c, flush, reps=reps))
+            time.sleep(1.0)
+        alone = [statistics.median(x) for x in per]
     call_ms, main_ms, _ = time_cases(sdpa, cases, steps, warmup, flush, sync_all, graphs)
     time.sleep(1.0)
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
