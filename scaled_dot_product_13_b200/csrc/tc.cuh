@@ -375,8 +375,9 @@ __global__ void __launch_bounds__(TcCfg<DQK, DV, BN, NSLOT>::kThreads, 1)
       // P is above 2^7.875 (the rounding of s * c - m stays below 1/8 while
       // |m| < 2^20), so a row sum below 224 rules it out and the row max is
       // needed only for the rare block whose sum reaches 224 (or is NaN).
-      // (A row of equal scores, zero-filled padding rows included, sums to at
-      // most BN and stays on the fast side.)
+      // (A row of equal scores at the reference, such as the zero-filled
+      // padding rows of a partly used tile, sums to BN and stays on the fast
+      // side.)
       // Either way P, the reference and the sum are those of the max-first
       // order below, bit for bit.
       const bool optimistic = kParts == 1 && !masked && c_pos && !c_zero &&
