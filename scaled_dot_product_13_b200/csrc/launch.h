@@ -66,7 +66,8 @@ constexpr int splitkv_stages(int dqk, int dv, int wr, unsigned budget) {
 // registers fit half the file: the second CTA's warps hide the first's
 // latencies (verify L=12..16 at S=32K: 44.4 -> 40.3 us).  The 16- and 32-row
 // layouts keep one per SM: twice the splits cost more in the combine than
-// the pass gains (decode sweep 2113-2125 against 2164-2167 GB/s).
+// the pass gains (decode sweep 3234-3245 against 3406-3408 GB/s with the
+// warp-per-row combine).
 constexpr int splitkv_ctas_per_sm(int dqk, int dv, int wr) {
   return wr == 4 && dqk + dv <= 256 && splitkv_stages(dqk, dv, wr, kSplitKvBudget2) >= 2 ? 2 : 1;
 }
