@@ -298,3 +298,22 @@ def test_plan_rounds_split_counts_to_whole_combine_rounds():
     # a pinned split count is kept as given
     info = sdpa.plan(1, 64, 4, 1, 32768, 192, 128, causal=True, num_sms=148, force_splits=37)
     assert info["splits"] == 37, info
+
+
+def test_plan_balance_rule_bounds():
+    # pair tiles = B * Hkv * ceil(g * L / 256); causal 256/256 calls with more
+    # than num_sms / 2 and fewer than num_sms of them take the one-SM kernel
+    def path(hkv, L, causal=True, window=0, dq=256, dv=256, sms=148):
+        return sdpa.plan(1, hkv, hkv, L, L, dq, dv, causal=causal, window_size=window,
+                         num_sms=sms)["path"]
+    assert path(74, 256) == sdpa.PATH_TC2          # 74 tiles: half the SMs
+    assert path(75, 256) == sdpa.PATH_TC           # 75
+    assert path(147, 256) == sdpa.PATH_TC          # 147
+    assert path(148, 256) == sdpa.PATH_TC2         # 148: two per SM pair
+    assert path(75, 256, causal=False) != sdpa.PATH_TC
+    assert path(75, 256, window=128) == sdpa.PATH_TC
+    assert path(75, 256, dq=192, dv=128) == sdpa.PATH_TC
+    # the bounds follow the SM count it plans for
+    assert path(75, 256, sms=132) == sdpa.PATH_TC and path(66, 256, sms=132) == sdpa.PATH_TC2
+    # head dims that never take the pair kernel are unaffected
+    assert path(100, 256, dq=128, dv=128) == sdpa.PATH_TC
