@@ -466,88 +466,131 @@ __global__ void __launch_bounds__(224, 1)
         }
         tc_fence_after();
         float s[BN];
+        auto load_s = [&]() {
 #pragma unroll
-        for (int c32 = 0; c32 < BN / 32; ++c32)
-          tmem_ld32(tmem + lane_base + b * BN + c32 * 32, s + c32 * 32);
-        tmem_wait_ld();
+          for (int c32 = 0; c32 < BN / 32; ++c32)
+            tmem_ld32(tmem + lane_base + b * BN + c32 * 32, s + c32 * 32);
+          tmem_wait_ld();
+        };
+        load_s();
+
+        // ---- P = exp2(s c - m) against the reference in use, packed to the
+        // 16-bit type, 32 columns at a time; returns the row sum.  The looping
+        // form stores each chunk over the row's own scores as soon as it is
+        // made; the one-tile form holds P until the block's check below ----
+        uint32_t pk[BN / 2];
+        auto exp_block = [&]() -> float {
+          const float mref = m_used == -INFINITY ? 0.f : m_used;
+          const float2 c2 = make_float2(c_eff, c_eff), nm2 = make_float2(-mref, -mref);
+          float2 acc[4];
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) acc[q4] = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int c32 = 0; c32 < BN / 32; ++c32) {
+#pragma unroll
+            for (int i2 = 0; i2 < 16; ++i2) {
+              const int i = c32 * 32 + 2 * i2;
+              float2 t = fma2(make_float2(s[i], s[i + 1]), c2, nm2);
+              if ((i2 & 3) < SDPA_TC2_POLY_OF4) {
+                t = exp2_poly2(t);  // FMA / ALU pipes
+              } else {
+                t.x = fast_exp2(t.x);  // MUFU
+                t.y = fast_exp2(t.y);
+              }
+              acc[i2 & 3] = add2(acc[i2 & 3], t);
+              pk[c32 * 16 + i2] = pack2<kBF16>(t.x, t.y);
+            }
+            if constexpr (PERSIST) tmem_st_u16x(tmem + lane_base + b * BN + c32 * 16, pk + c32 * 16);
+          }
+          const float2 a01 = add2(acc[0], acc[1]), a23 = add2(acc[2], acc[3]);
+          const float2 at = add2(a01, a23);
+          return at.x + at.y;
+        };
 
         const int kbase = w.k_lo + j * BN;
         const bool masked = block_needs_mask(p, tr, kbase, BN);
-        // The common block (positive scale, no masked key) takes the plain
-        // reduction; the rare ones (scale 0, masked keys, negative scale) their
-        // own copy, so that their per-element work is not folded into it.
-        float mr[1];
-        if (!masked && c_pos && !c_zero) {
-          mr[0] = row_reduce_max(s);
-        } else {
-          if (c_zero) {
-#pragma unroll
-            for (int i = 0; i < BN; ++i) s[i] = 0.f;
-          }
-          if (masked) {
-            const VisibleRange vis = visible_range(p, pos, kbase);
-#pragma unroll
-            for (int i = 0; i < BN; ++i)
-              if (!vis(i)) s[i] = neutral;
-          }
-          mr[0] = c_pos ? row_reduce_max(s) : row_reduce_min(s);
+        // One tile per pair: plain blocks (positive scale, no masked key, a
+        // reference already set) first take P against the current reference.
+        // The reference only moves when a score exceeds it by more than 8
+        // (log2 units): then some P is above 2^7.875 (the rounding of s c - m
+        // stays below 1/8 while |m| < 2^20), so a row sum below 224 rules it
+        // out and the row max is taken only for the rare block whose sum
+        // reaches 224 (or is NaN); P, the reference and the sum are those of
+        // the max-first order, bit for bit.  The looping form keeps the
+        // max-first order: its chunked P stores overwrite the scores a
+        // fallback would reload, and holding P instead measured slower there.
+        const bool optimistic = !PERSIST && !masked && c_pos && !c_zero &&
+                                !__any_sync(0xffffffffu, m_used == -INFINITY);
+        float lsum = 0.f;
+        bool by_max = true;
+        if (optimistic) {
+          lsum = exp_block();
+          by_max = __any_sync(0xffffffffu, !(lsum < 224.f));
+          if (by_max) load_s();  // the scores are still in TMEM (P not stored)
         }
-        const float mblk = isinf(mr[0]) ? -INFINITY : mr[0] * c_eff;
-        const float m_new = fmaxf(m_used, mblk);
-        const bool need = m_new > m_used + 8.0f;
-        float alpha = 1.f;
-        if (need) {
-          alpha = fast_exp2(m_used - m_new);
-          m_used = m_new;
-          l *= alpha;
-        }
-        if (j > 0 && __any_sync(0xffffffffu, need)) {
-          // S_x was issued after P_{x-2} V by the same thread, and P_x V waits
-          // for p_full: o_bar is in phase x-1 or x here.  The TMEM loads and
-          // stores are warp-wide, so the whole warp rescales its rows.
-          if (lane == 0) wt = mbar_wait_cluster(o_bar, (uint32_t)(x - 1) & 1u, p.wd, kWdMma);
-          if (!__shfl_sync(0xffffffffu, (int)wt, 0)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-#pragma unroll 1
-          for (int c16 = 0; c16 < DV / 16; ++c16) {
-            float o[16];
-            tmem_ld16(tmem + lane_base + Cfg::kOCol + c16 * 16, o);
-            tmem_wait_ld();
+        if (by_max) {
+          // The common block (positive scale, no masked key) takes the plain
+          // reduction; the rare ones (scale 0, masked keys, negative scale)
+          // their own copy, so that their per-element work is not folded in.
+          float mr[1];
+          if (!masked && c_pos && !c_zero) {
+            mr[0] = row_reduce_max(s);
+          } else {
+            if (c_zero) {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) o[e] *= alpha;
-            tmem_st16(tmem + lane_base + Cfg::kOCol + c16 * 16, o);
-          }
-        }
-        // ---- P = exp2(s c - m), row sum, P packed over the row's own scores ----
-        const float mref = m_used == -INFINITY ? 0.f : m_used;
-        const float2 c2 = make_float2(c_eff, c_eff), nm2 = make_float2(-mref, -mref);
-        float2 acc[4];
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) acc[q4] = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int c32 = 0; c32 < BN / 32; ++c32) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int i2 = 0; i2 < 16; ++i2) {
-            const int i = c32 * 32 + 2 * i2;
-            float2 t = fma2(make_float2(s[i], s[i + 1]), c2, nm2);
-            if ((i2 & 3) < SDPA_TC2_POLY_OF4) {
-              t = exp2_poly2(t);  // FMA / ALU pipes
-            } else {
-              t.x = fast_exp2(t.x);  // MUFU
-              t.y = fast_exp2(t.y);
+              for (int i = 0; i < BN; ++i) s[i] = 0.f;
             }
-            acc[i2 & 3] = add2(acc[i2 & 3], t);
-            pk[i2] = pack2<kBF16>(t.x, t.y);
+            if (masked) {
+              const VisibleRange vis = visible_range(p, pos, kbase);
+#pragma unroll
+              for (int i = 0; i < BN; ++i)
+                if (!vis(i)) s[i] = neutral;
+            }
+            mr[0] = c_pos ? row_reduce_max(s) : row_reduce_min(s);
           }
-          tmem_st_u16x(tmem + lane_base + b * BN + c32 * 16, pk);
+          const float mblk = isinf(mr[0]) ? -INFINITY : mr[0] * c_eff;
+          const float m_new = fmaxf(m_used, mblk);
+          const bool need = m_new > m_used + 8.0f;
+          float alpha = 1.f;
+          if (need) {
+            alpha = fast_exp2(m_used - m_new);
+            m_used = m_new;
+            l *= alpha;
+          }
+          const bool any_need = __any_sync(0xffffffffu, need);
+          if (j > 0 && any_need) {
+            // S_x was issued after P_{x-2} V by the same thread, and P_x V
+            // waits for p_full: o_bar is in phase x-1 or x here.  The TMEM
+            // loads and stores are warp-wide, so the whole warp rescales its
+            // rows.
+            if (lane == 0) wt = mbar_wait_cluster(o_bar, (uint32_t)(x - 1) & 1u, p.wd, kWdMma);
+            if (!__shfl_sync(0xffffffffu, (int)wt, 0)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll 1
+            for (int c16 = 0; c16 < DV / 16; ++c16) {
+              float o[16];
+              tmem_ld16(tmem + lane_base + Cfg::kOCol + c16 * 16, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 16; ++e) o[e] *= alpha;
+              tmem_st16(tmem + lane_base + Cfg::kOCol + c16 * 16, o);
+            }
+          }
+          // P (again, where the reference moved: every lane recomputes, and
+          // an unchanged reference gives the same P and sum)
+          if (!optimistic || any_need) lsum = exp_block();
         }
-        const float2 a01 = add2(acc[0], acc[1]), a23 = add2(acc[2], acc[3]);
-        const float2 at = add2(a01, a23);
-        l += at.x + at.y;
+        // one tile per pair: P over the first BN/2 columns of the row's own
+        // scores, once the block's check has passed
+        if constexpr (!PERSIST) {
+#pragma unroll
+          for (int c32 = 0; c32 < BN / 32; ++c32)
+            tmem_st_u16x(tmem + lane_base + b * BN + c32 * 16, pk + c32 * 16);
+        }
+        l += lsum;
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
