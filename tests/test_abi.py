@@ -7,6 +7,7 @@ import re
 import pytest
 
 import scaled_dot_product_13_b200 as sdpa
+from scaled_dot_product_13_b200 import inputs as I
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -317,3 +318,38 @@ def test_plan_balance_rule_bounds():
     assert path(75, 256, sms=132) == sdpa.PATH_TC and path(66, 256, sms=132) == sdpa.PATH_TC2
     # head dims that never take the pair kernel are unaffected
     assert path(100, 256, dq=128, dv=128) == sdpa.PATH_TC
+
+
+def test_plan_routes_every_benchmark_configuration():
+    # (path, key splits) the router gives each benchmark configuration on 148
+    # SMs, as measured and described with the kernels: a change to the routing
+    # rules that moves one of them has to show up here
+    S, T, P2, W, D, L7 = (sdpa.PATH_SPLITKV, sdpa.PATH_TC, sdpa.PATH_TC2, sdpa.PATH_WIDE,
+                          sdpa.PATH_TC_DUAL, sdpa.PATH_TC2_LOOP)
+    want = {"tiny_causal_gqa": (T, 1)}
+    for s, k4, k8 in ((256, 1, 1), (1024, 8, 8), (4096, 32, 16), (8192, 32, 16),
+                      (16384, 32, 18), (32768, 32, 18)):
+        want[f"decode_hkv4_s{s}"] = (S, k4)
+        want[f"decode_hkv8_s{s}"] = (S, k8)
+    for s, mid in ((16384, 16), (32768, 18)):
+        for l in (1, 2, 4, 8):
+            want[f"verify_s{s}_l{l}"] = (S, 18)
+        for l in (12, 16, 24, 32):
+            want[f"verify_s{s}_l{l}"] = (T, mid)
+        for l in (48, 64):
+            want[f"verify_s{s}_l{l}"] = (T, 9)
+    want.update({
+        "encoder_h20_l1500_d64": (D, 1), "encoder_h16_l1024_d72": (T, 1),
+        "encoder_h16_l4096_d72": (D, 1),
+        "window_l2048_w1024_d256": (T, 1), "window_l4096_w1024_d256": (L7, 1),
+        "window_l8192_w1024_d256": (L7, 1), "causal_l32768_d256": (P2, 1),
+        "wide_decode_d512_s8192": (W, 32), "wide_decode_d512_s32768": (W, 128),
+        "wide_prefill_d512_l4096": (P2, 1),
+    })
+    probs = (I.decode_problems() + I.verify_problems() + I.encoder_problems()
+             + I.window_problems() + I.wide_problems() + [I.tiny_problem()])
+    assert {p.name for p in probs} == set(want)
+    for p in probs:
+        info = sdpa.plan(p.B, p.Hq, p.Hkv, p.L, p.S, p.Dqk, p.Dv, p.causal, p.window, p.dtype,
+                         num_sms=148)
+        assert (info["path"], info["splits"]) == want[p.name], (p.name, info)
